@@ -1,0 +1,171 @@
+/*
+ * CPU ORACLE -- TEST INFRASTRUCTURE ONLY.
+ *
+ * Plain, slow, fp64 reference for the packed-THD sliding-window GQA attention
+ * forward.  Only the tests, the smoke check and the benchmark's CPU-baseline /
+ * reference arm may load it.  It shares no code with the CUDA path.
+ *
+ * What it computes (restated from the NeMo AutoModel API pages):
+ *
+ *   Packed THD tensors -- "muse_spark.magi_cp", MuseMagiPlan.attention
+ *   (query/key/value parameters): q[T, Hq, D], k[T, Hkv, D], v[T, Hkv, D];
+ *   documents delimited by cu_seqlens, "CPU int32 padded document boundaries
+ *   [documents + 1]" (_build_magi_plan, cu_seqlens parameter).
+ *
+ *   Visible keys -- "flint.magi", FlintMagiPlan.attention, window parameter:
+ *   the window counts the current token, zero means full causal.  For a query
+ *   i of document [s, e):   V(i) = { j : s <= j <= i, and W == 0 or j > i - W }.
+ *
+ *   GQA -- "muse_glimmer.model", repeat_kv: each of the Hkv key/value heads is
+ *   repeated Hq/Hkv times to reach the query-head count, so query head h reads
+ *   kv head g = h / (Hq/Hkv).
+ *
+ *   Scores -- MuseMagiPlan.attention, scale parameter:
+ *   s_ij = scale * sum_c q[i,h,c] * k[j,g,c].
+ *
+ *   Sink -- FlintMagiPlan.attention, sink parameter: one fp32 learned logit per
+ *   query head that enters the softmax denominator only (it has no value row):
+ *   Z = sum_{j in V(i)} exp(s_ij) + exp(sink_h);
+ *   out[i,h,:] = sum_{j in V(i)} exp(s_ij) v[j,g,:] / Z;   lse[i,h] = ln Z.
+ *
+ * Readings where the pages leave a step open: the sink is compared unscaled
+ * with the scaled scores; lse is the natural log and includes the sink term;
+ * a row with an empty key set gives out = 0 and lse = -inf (or the sink).
+ *
+ * The max-shift below is only for range safety (the exponentials are taken
+ * relative to the row maximum); it does not change the result in exact
+ * arithmetic.  Parallelised over (token, head) rows with OpenMP; no other
+ * reordering.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+enum { ORACLE_F64 = 0, ORACLE_BF16 = 1 };
+
+static double load_elem(const void *base, int64_t idx, int dtype) {
+    if (dtype == ORACLE_F64) return ((const double *)base)[idx];
+    uint32_t u = ((uint32_t)((const uint16_t *)base)[idx]) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Document containing token i: the d with cu[d] <= i < cu[d+1] (binary search). */
+static int find_doc(const int32_t *cu, int n_docs, int64_t i) {
+    int lo = 0, hi = n_docs - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) / 2;
+        if ((int64_t)cu[mid] <= i) lo = mid; else hi = mid - 1;
+    }
+    while (lo < n_docs - 1 && (int64_t)cu[lo + 1] <= i) lo++; /* skip empty docs */
+    return lo;
+}
+
+static int check_args(const int32_t *cu, int n_docs, int Hq, int Hkv, int D, int window) {
+    if (n_docs < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || window < 0) return -1;
+    if (Hq % Hkv != 0) return -1;
+    if (cu == NULL) return -1;
+    if (cu[0] != 0) return -1;
+    for (int d = 0; d < n_docs; d++)
+        if (cu[d + 1] < cu[d]) return -1;
+    return 0;
+}
+
+/* One output row (token i, query head h).  out_row has D entries. */
+static void attend_row(const void *q, const void *k, const void *v, int dtype,
+                       const int32_t *cu, int n_docs, int Hq, int Hkv, int D,
+                       int window, double scale, const float *sinks,
+                       int64_t i, int h, double *out_row, double *lse_out) {
+    const int G = Hq / Hkv;
+    const int g = h / G;                       /* repeat_kv: contiguous repeats */
+    const int d = find_doc(cu, n_docs, i);
+    const int64_t s = cu[d];
+    int64_t lo = s;                            /* j >= s */
+    if (window > 0 && i - window + 1 > lo) lo = i - window + 1; /* j > i - W */
+    const int64_t n = i - lo + 1;              /* keys lo..i inclusive */
+
+    double *sc = (double *)malloc((size_t)(n > 0 ? n : 1) * sizeof(double));
+    double m = -INFINITY;
+    for (int64_t j = lo; j <= i; j++) {
+        double acc = 0.0;
+        for (int c = 0; c < D; c++)
+            acc += load_elem(q, (i * Hq + h) * (int64_t)D + c, dtype) *
+                   load_elem(k, (j * Hkv + g) * (int64_t)D + c, dtype);
+        sc[j - lo] = scale * acc;
+        if (sc[j - lo] > m) m = sc[j - lo];
+    }
+    const int has_sink = sinks != NULL;
+    const double sink = has_sink ? (double)sinks[h] : -INFINITY;
+    if (has_sink && sink > m) m = sink;
+
+    for (int c = 0; c < D; c++) out_row[c] = 0.0;
+    if (m == -INFINITY) {                      /* empty key set, no sink */
+        *lse_out = -INFINITY;
+        free(sc);
+        return;
+    }
+    double Z = has_sink ? exp(sink - m) : 0.0;
+    for (int64_t j = lo; j <= i; j++) {
+        const double w = exp(sc[j - lo] - m);
+        Z += w;
+        for (int c = 0; c < D; c++)
+            out_row[c] += w * load_elem(v, (j * Hkv + g) * (int64_t)D + c, dtype);
+    }
+    for (int c = 0; c < D; c++) out_row[c] /= Z;
+    *lse_out = m + log(Z);
+    free(sc);
+}
+
+/*
+ * Full forward: out[T, Hq, D] and lse[T, Hq] in fp64.
+ * q/k/v are fp64 (dtype 0) or raw bf16 bit patterns (dtype 1).
+ * sinks may be NULL.  Returns 0, or -1 on invalid arguments.
+ */
+int oracle_thd_attn(const void *q, const void *k, const void *v, int dtype,
+                    const int32_t *cu_seqlens, int n_docs, int Hq, int Hkv, int D,
+                    int window, double scale, const float *sinks,
+                    double *out, double *lse) {
+    if (check_args(cu_seqlens, n_docs, Hq, Hkv, D, window)) return -1;
+    const int64_t T = n_docs > 0 ? cu_seqlens[n_docs] : 0;
+    const int64_t rows = T * Hq;
+#pragma omp parallel for schedule(dynamic, 8)
+    for (int64_t r = 0; r < rows; r++) {
+        const int64_t i = r / Hq;
+        const int h = (int)(r % Hq);
+        attend_row(q, k, v, dtype, cu_seqlens, n_docs, Hq, Hkv, D, window, scale,
+                   sinks, i, h, out + r * D, lse + r);
+    }
+    return 0;
+}
+
+/*
+ * Selected rows only: rows[2*r] = token, rows[2*r+1] = query head.
+ * out[n_rows, D], lse[n_rows].  Used for sampled checks of full-size packs.
+ */
+int oracle_thd_attn_rows(const void *q, const void *k, const void *v, int dtype,
+                         const int32_t *cu_seqlens, int n_docs, int Hq, int Hkv, int D,
+                         int window, double scale, const float *sinks,
+                         const int64_t *rows, int64_t n_rows, double *out, double *lse) {
+    if (check_args(cu_seqlens, n_docs, Hq, Hkv, D, window)) return -1;
+    const int64_t T = n_docs > 0 ? cu_seqlens[n_docs] : 0;
+    for (int64_t r = 0; r < n_rows; r++)
+        if (rows[2 * r] < 0 || rows[2 * r] >= T || rows[2 * r + 1] < 0 || rows[2 * r + 1] >= Hq)
+            return -1;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n_rows; r++)
+        attend_row(q, k, v, dtype, cu_seqlens, n_docs, Hq, Hkv, D, window, scale, sinks,
+                   rows[2 * r], (int)rows[2 * r + 1], out + r * D, lse + r);
+    return 0;
+}
+
+/* Threads OpenMP would use for the calls above. */
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
