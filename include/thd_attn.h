@@ -1,0 +1,138 @@
+/*
+ * thd_attn.h -- C ABI of the B200 (sm_100a) packed-THD sliding-window GQA
+ * attention forward.
+ *
+ * The operation (restated from the NeMo AutoModel API pages):
+ *
+ *   Inputs are packed THD tensors as in MuseMagiPlan.attention and
+ *   FlintMagiPlan.attention ("muse_spark.magi_cp" and "flint.magi" pages,
+ *   query/key/value parameters): q [T, Hq, D], k and v [T, Hkv, D], with the
+ *   documents of the pack delimited by cu_seqlens, "CPU int32 padded document
+ *   boundaries [documents + 1]" (_build_magi_plan, cu_seqlens parameter).
+ *
+ *   For a query token i in document [s, e) and query head h, the visible keys
+ *   are V(i) = { j : s <= j <= i and (window == 0 or j > i - window) }: the
+ *   window counts the current token and zero means full causal
+ *   (FlintMagiPlan.attention, window parameter).  Query head h reads key/value
+ *   head g = h / (Hq / Hkv), the repeat_kv mapping ("muse_glimmer.model" page).
+ *
+ *   s_ij = scale * <q[i,h,:], k[j,g,:]>                       (scale parameter)
+ *   Z    = sum_{j in V(i)} exp(s_ij) + exp(sink[h])           (sink parameter;
+ *          the sink term is present only when sinks are given and has no
+ *          value row)
+ *   out[i,h,:] = sum_{j in V(i)} exp(s_ij) v[j,g,:] / Z       (bf16)
+ *   lse[i,h]   = ln Z                                          (fp32)
+ *
+ *   The output is written in the input token order ("Attention output
+ *   [tokens, query_heads, head_dim] in the local token order").
+ *
+ * Conventions shared by every entry point:
+ *   - Device pointers are CUDA global-memory pointers on the current device;
+ *     q, k, v, out must be 16-byte aligned and dense (row-major, no strides).
+ *   - cu_seqlens is a HOST array; it is read during the call only.
+ *   - The caller owns every buffer.  The library keeps, per device, a small
+ *     cache of tile schedules, one status word and nothing else.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t passed as
+ *     void*; NULL = the legacy default stream).  Argument errors are detected
+ *     on the host before anything is enqueued and return a negative code.
+ *   - A kernel that stops making progress (a bounded wait on the GPU ran out)
+ *     records THD_ERR_TIMEOUT in the device status word and exits cleanly;
+ *     thd_attn_get_error() reports it.
+ */
+#ifndef THD_ATTN_H
+#define THD_ATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum thd_status {
+    THD_OK = 0,
+    THD_ERR_INVALID_ARG = -1,  /* bad pointer, alignment, shape, cu_seqlens, window or scale */
+    THD_ERR_UNSUPPORTED = -2,  /* head_dim not in {64,128,256}, or device is not sm_100 */
+    THD_ERR_CUDA = -3,         /* a CUDA runtime/driver call failed */
+    THD_ERR_TIMEOUT = -4,      /* a bounded wait inside the kernel ran out */
+    THD_ERR_NO_MEMORY = -5     /* the schedule cache could not be allocated */
+};
+
+/*
+ * Forward pass.
+ *
+ *   q          bf16 device [T, Hq, D]        (T = cu_seqlens[n_docs])
+ *   k, v       bf16 device [T, Hkv, D]
+ *   cu_seqlens int32 HOST [n_docs + 1]: cu_seqlens[0] == 0, non-decreasing;
+ *              zero-length documents are allowed; T == 0 or n_docs == 0 is a
+ *              no-op that returns THD_OK.
+ *   Hq, Hkv    query / key-value heads, Hq % Hkv == 0
+ *   D          head dim, one of 64, 128, 256
+ *   window     >= 0; 0 = full causal, W > 0 = the W most recent keys of the
+ *              document including the query's own token
+ *   scale      finite and > 0 (score scale, e.g. D^-0.5)
+ *   sinks_or_null  fp32 device [Hq] learned sink logits, or NULL for none.
+ *              A value of -inf (or very negative) behaves as no sink.
+ *   out        bf16 device [T, Hq, D]; every element is written
+ *   lse        fp32 device [T, Hq] natural-log log-sum-exp (sink included),
+ *              or NULL to skip it
+ *   stream     cudaStream_t as void*
+ *
+ * Returns THD_OK once the kernel is enqueued, or a negative thd_status
+ * (nothing is enqueued on error).
+ */
+int thd_attn_fwd(const void* q, const void* k, const void* v,
+                 const int32_t* cu_seqlens, int n_docs,
+                 int Hq, int Hkv, int D, int window, float scale,
+                 const float* sinks_or_null,
+                 void* out, float* lse,
+                 void* stream);
+
+/*
+ * Synchronises `stream`, returns the status recorded by kernels of this
+ * library on the current device since the last call (THD_OK if none) and
+ * clears it.  Returns THD_ERR_CUDA if the synchronisation itself fails.
+ */
+int thd_attn_get_error(void* stream);
+
+/* Static English description of a thd_status value. */
+const char* thd_attn_status_string(int status);
+
+/*
+ * One unit of work of the tile schedule: a tile of up to 128 query rows of
+ * one document for `n_heads` consecutive query heads that share one kv head,
+ * against the key tiles [kv_start, kv_start + n_kv * block_n).
+ *   q0         first row of the 128-row query tile (may lie before doc_start;
+ *              rows before doc_start are computed but never written)
+ *   q1         one past the last row (<= the document end)
+ *   doc_start  first token of the document
+ *   head0      first query head of the item
+ *   kv_start   first key of the first key tile (may lie before doc_start;
+ *              such keys are masked)
+ *   n_kv       number of key tiles (>= 1)
+ *   n_heads    query heads in the item
+ *   block_n    keys per key tile
+ */
+typedef struct thd_work_item {
+    int32_t q0, q1, doc_start, head0;
+    int32_t kv_start, n_kv, n_heads, block_n;
+} thd_work_item;
+
+/*
+ * Host-only: build the tile schedule thd_attn_fwd uses for these arguments,
+ * ordered longest first (non-increasing n_kv; heads of one kv group adjacent).
+ * No CUDA call is made.  `items` may be NULL to query the count.  Writes
+ * min(count, capacity) items and sets *n_items = count.  Returns THD_OK or
+ * THD_ERR_INVALID_ARG / THD_ERR_UNSUPPORTED for the same argument errors as
+ * thd_attn_fwd.
+ */
+int thd_attn_plan(const int32_t* cu_seqlens, int n_docs, int Hq, int Hkv, int D, int window,
+                  thd_work_item* items, int64_t capacity, int64_t* n_items);
+
+/* ABI version of this header: (major << 16) | minor. */
+int thd_attn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* THD_ATTN_H */

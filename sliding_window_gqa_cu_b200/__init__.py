@@ -1,0 +1,172 @@
+"""B200 (sm_100a) packed-THD sliding-window GQA attention forward.
+
+Python binding over the C ABI in ``include/thd_attn.h`` (``libthdattn.so``,
+built in-tree by :mod:`sliding_window_gqa_cu_b200.build`).  This module only
+marshals arguments: every step of the computation runs in the CUDA library.
+PyTorch supplies device memory and the current stream.
+
+The operation is the local THD attention of ``MuseMagiPlan.attention`` /
+``FlintMagiPlan.attention`` (NeMo AutoModel "muse_spark.magi_cp" and
+"flint.magi" pages): q ``[T, Hq, D]``, k/v ``[T, Hkv, D]`` packed by
+``cu_seqlens``, causal or sliding-window (the window counts the current
+token), GQA by ``repeat_kv`` head mapping, optional per-head sink logits,
+bf16 output ``[T, Hq, D]`` and fp32 log-sum-exp ``[T, Hq]``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+
+__all__ = ["thd_attn_fwd", "thd_attn_get_error", "thd_attn_plan", "ThdAttnError", "library_path",
+           "load_library", "STATUS"]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libthdattn.so"
+_lib = None
+
+STATUS = {0: "THD_OK", -1: "THD_ERR_INVALID_ARG", -2: "THD_ERR_UNSUPPORTED", -3: "THD_ERR_CUDA",
+          -4: "THD_ERR_TIMEOUT", -5: "THD_ERR_NO_MEMORY"}
+
+WORK_ITEM_FIELDS = ("q0", "q1", "doc_start", "head0", "kv_start", "n_kv", "n_heads", "block_n")
+
+
+class ThdAttnError(RuntimeError):
+    def __init__(self, code: int, what: str = ""):
+        self.code = code
+        msg = f"{STATUS.get(code, code)}: {_status_string(code)}"
+        super().__init__(f"{what}: {msg}" if what else msg)
+
+
+class _WorkItem(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_int32) for f in WORK_ITEM_FIELDS]
+
+
+def library_path() -> str:
+    return os.path.join(_PKG, _LIB_NAME)
+
+
+def load_library():
+    """Load ``libthdattn.so``; raises if it has not been built (no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise ImportError(
+            f"{path} is missing: build it with `python -m sliding_window_gqa_cu_b200.build` "
+            "(there is no CPU fallback)")
+    lib = ctypes.CDLL(path)
+    vp, i32p, c_int = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32), ctypes.c_int
+    lib.thd_attn_fwd.argtypes = [vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int,
+                                 ctypes.c_float, vp, vp, vp, vp]
+    lib.thd_attn_fwd.restype = c_int
+    lib.thd_attn_get_error.argtypes = [vp]
+    lib.thd_attn_get_error.restype = c_int
+    lib.thd_attn_status_string.argtypes = [c_int]
+    lib.thd_attn_status_string.restype = ctypes.c_char_p
+    lib.thd_attn_plan.argtypes = [i32p, c_int, c_int, c_int, c_int, c_int,
+                                  ctypes.POINTER(_WorkItem), ctypes.c_int64,
+                                  ctypes.POINTER(ctypes.c_int64)]
+    lib.thd_attn_plan.restype = c_int
+    lib.thd_attn_abi_version.argtypes = []
+    lib.thd_attn_abi_version.restype = c_int
+    _lib = lib
+    return lib
+
+
+def _status_string(code: int) -> str:
+    try:
+        return load_library().thd_attn_status_string(int(code)).decode()
+    except Exception:  # library missing while formatting an error
+        return "?"
+
+
+def _cu_array(cu_seqlens) -> np.ndarray:
+    try:
+        import torch
+        if isinstance(cu_seqlens, torch.Tensor):
+            cu_seqlens = cu_seqlens.detach().cpu().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+    if cu.ndim != 1 or cu.size < 1:
+        raise ValueError("cu_seqlens must be a 1-D array of documents + 1 boundaries")
+    return cu
+
+
+def thd_attn_plan(cu_seqlens, Hq: int, Hkv: int, D: int, window: int) -> np.ndarray:
+    """The tile schedule (structured numpy array, one record per work item)."""
+    lib = load_library()
+    cu = _cu_array(cu_seqlens)
+    n = ctypes.c_int64(0)
+    cup = cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    rc = lib.thd_attn_plan(cup, cu.size - 1, Hq, Hkv, D, window, None, 0, ctypes.byref(n))
+    if rc != 0:
+        raise ThdAttnError(rc, "thd_attn_plan")
+    buf = (_WorkItem * max(1, n.value))()
+    rc = lib.thd_attn_plan(cup, cu.size - 1, Hq, Hkv, D, window, buf, n.value, ctypes.byref(n))
+    if rc != 0:
+        raise ThdAttnError(rc, "thd_attn_plan")
+    dt = np.dtype([(f, np.int32) for f in WORK_ITEM_FIELDS])
+    return np.frombuffer(bytes(buf), dtype=dt, count=n.value).copy()
+
+
+def thd_attn_fwd(q, k, v, cu_seqlens, window: int = 0, scale: Optional[float] = None,
+                 sinks=None, out=None, lse=None, return_lse: bool = True, stream=None):
+    """Packed-THD attention forward on the current CUDA device.
+
+    q: bf16 CUDA tensor [T, Hq, D]; k, v: bf16 CUDA [T, Hkv, D] (contiguous);
+    cu_seqlens: host int32 boundaries [documents + 1] (numpy, list or CPU tensor);
+    window: 0 = full causal, W > 0 = W keys including the query's own token;
+    scale: score scale (default D ** -0.5); sinks: fp32 CUDA [Hq] or None.
+    Returns ``(out, lse)`` (``lse`` is None when ``return_lse`` is False).
+    """
+    import torch
+
+    lib = load_library()
+    if q.dim() != 3 or k.dim() != 3 or v.dim() != 3:
+        raise ValueError("q, k, v must be [tokens, heads, head_dim]")
+    T, Hq, D = q.shape
+    Hkv = k.shape[1]
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    if k.shape != (T, Hkv, D) or v.shape != (T, Hkv, D):
+        raise ValueError("k and v must be [tokens, kv_heads, head_dim] like q")
+    cu = _cu_array(cu_seqlens)
+    if int(cu[-1]) != T:
+        raise ValueError(f"cu_seqlens[-1]={int(cu[-1])} does not match {T} tokens")
+    if scale is None:
+        scale = D ** -0.5
+    if sinks is not None:
+        if sinks.dtype != torch.float32 or not sinks.is_cuda or sinks.numel() != Hq:
+            raise ValueError("sinks must be an fp32 CUDA tensor of Hq values")
+        sinks = sinks.contiguous()
+    if out is None:
+        out = torch.empty((T, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        rc = lib.thd_attn_fwd(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(),
+            cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), cu.size - 1,
+            Hq, Hkv, D, int(window), float(scale),
+            sinks.data_ptr() if sinks is not None else None,
+            out.data_ptr(), lse.data_ptr() if lse is not None else None,
+            ctypes.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise ThdAttnError(rc, "thd_attn_fwd")
+    return out, lse
+
+
+def thd_attn_get_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(load_library().thd_attn_get_error(ctypes.c_void_p(stream.cuda_stream)))

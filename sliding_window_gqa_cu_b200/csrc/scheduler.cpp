@@ -1,0 +1,72 @@
+// Host tile scheduler: see scheduler.h.
+#include "scheduler.h"
+
+#include <algorithm>
+
+namespace thd {
+
+bool choose_kernel_shape(int D, int group, KernelShape* out) {
+    const bool pair = (group % 2) == 0;  // two heads of one kv group per CTA
+    switch (D) {
+        case 64:
+            *out = pair ? KernelShape{64, 2, 1, 128, 4} : KernelShape{64, 1, 2, 128, 4};
+            return true;
+        case 128:
+            *out = pair ? KernelShape{128, 2, 1, 128, 2} : KernelShape{128, 1, 2, 128, 2};
+            return true;
+        case 256:
+            *out = KernelShape{256, 1, 2, 64, 2};
+            return true;
+        default:
+            return false;
+    }
+}
+
+int validate_args(const int32_t* cu_seqlens, int n_docs, int Hq, int Hkv, int D, int window) {
+    if (n_docs < 0 || cu_seqlens == nullptr) return THD_ERR_INVALID_ARG;
+    if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return THD_ERR_INVALID_ARG;
+    if (window < 0) return THD_ERR_INVALID_ARG;
+    if (cu_seqlens[0] != 0) return THD_ERR_INVALID_ARG;
+    for (int d = 0; d < n_docs; ++d)
+        if (cu_seqlens[d + 1] < cu_seqlens[d]) return THD_ERR_INVALID_ARG;
+    if (D != 64 && D != 128 && D != 256) return THD_ERR_UNSUPPORTED;
+    return THD_OK;
+}
+
+std::vector<thd_work_item> build_plan(const int32_t* cu, int n_docs, int Hq, int Hkv, int window,
+                                      const KernelShape& ks) {
+    constexpr int BM = 128;
+    const int G = Hq / Hkv;
+    const int BN = ks.block_n;
+    std::vector<thd_work_item> items;
+    size_t n_tiles = 0;
+    for (int d = 0; d < n_docs; ++d) n_tiles += (cu[d + 1] - cu[d] + BM - 1) / BM;
+    items.reserve(n_tiles * static_cast<size_t>(Hq / ks.nq));
+
+    for (int d = 0; d < n_docs; ++d) {
+        const int s = cu[d], e = cu[d + 1];
+        // Query tiles are aligned to the document END, so a ragged tile is the
+        // document's first (shortest key range) rather than its last.
+        for (int q1 = e; q1 > s; q1 -= BM) {
+            const int q0 = q1 - BM;
+            const int r_lo = q0 > s ? q0 : s;
+            int k_lo = s;  // lowest key any row of the tile can see
+            if (window > 0 && r_lo - window + 1 > k_lo) k_lo = r_lo - window + 1;
+            const int n_kv = (q1 - k_lo + BN - 1) / BN;
+            // Key tiles are aligned to the tile end: the last one sits on the
+            // causal diagonal, keys below k_lo in the first one are masked.
+            const int kv_start = q1 - n_kv * BN;
+            for (int g = 0; g < Hkv; ++g)
+                for (int hp = 0; hp < G / ks.nq; ++hp)
+                    items.push_back(thd_work_item{q0, q1, s, g * G + hp * ks.nq, kv_start, n_kv,
+                                                  ks.nq, BN});
+        }
+    }
+    // Longest first; the stable sort keeps the heads of one kv group (which
+    // read the same K/V tiles) next to each other.
+    std::stable_sort(items.begin(), items.end(),
+                     [](const thd_work_item& a, const thd_work_item& b) { return a.n_kv > b.n_kv; });
+    return items;
+}
+
+}  // namespace thd

@@ -1,0 +1,38 @@
+// Host-side tile scheduler for the packed-THD attention forward.
+//
+// Turns the document boundaries of a pack (cu_seqlens, "CPU int32 padded
+// document boundaries [documents + 1]" in _build_magi_plan) plus the window
+// into the list of work items the kernel runs: one per (128-row query tile,
+// group of query heads sharing a kv head).  The plan is the B200 counterpart
+// of a per-microbatch Magi plan: built once per pack and reused by every
+// layer that shares the same boundaries and window.
+#pragma once
+
+#include <cstdint>
+#include <vector>
+
+#include "../../include/thd_attn.h"
+
+namespace thd {
+
+// Kernel shape chosen for a head dim and GQA group size.
+struct KernelShape {
+    int D;
+    int nq;       // query heads per work item (1 or 2)
+    int nsb;      // S buffers per query tile
+    int block_n;  // keys per key tile
+    int nst;      // K/V ring depth
+};
+
+// Returns false if the head dim is unsupported.
+bool choose_kernel_shape(int D, int group, KernelShape* out);
+
+// Host argument checks shared by every entry point (no CUDA calls).
+int validate_args(const int32_t* cu_seqlens, int n_docs, int Hq, int Hkv, int D, int window);
+
+// Builds the longest-first work list.  cu_seqlens must have passed
+// validate_args.
+std::vector<thd_work_item> build_plan(const int32_t* cu_seqlens, int n_docs, int Hq, int Hkv,
+                                      int window, const KernelShape& ks);
+
+}  // namespace thd

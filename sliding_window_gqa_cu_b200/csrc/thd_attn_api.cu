@@ -1,0 +1,270 @@
+// C ABI of the packed-THD attention forward (declared in include/thd_attn.h):
+// host validation, the per-device schedule cache and status word, TMA
+// descriptor encoding and the kernel launch.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <list>
+#include <mutex>
+#include <unordered_map>
+#include <vector>
+
+#include "../../include/thd_attn.h"
+#include "scheduler.h"
+#include "thd_attn_kernel.cuh"
+
+namespace {
+
+using thd::KernelShape;
+
+// ------------------------------------------------------------ kernel shapes --
+
+using Cfg64x2 = thd::FwdConfig<64, 2, 1, 128, 4>;
+using Cfg64x1 = thd::FwdConfig<64, 1, 2, 128, 4>;
+using Cfg128x2 = thd::FwdConfig<128, 2, 1, 128, 2>;
+using Cfg128x1 = thd::FwdConfig<128, 1, 2, 128, 2>;
+using Cfg256x1 = thd::FwdConfig<256, 1, 2, 64, 2>;
+
+constexpr int kNumVariants = 5;
+
+int variant_index(const KernelShape& ks) {
+    if (ks.D == 64) return ks.nq == 2 ? 0 : 1;
+    if (ks.D == 128) return ks.nq == 2 ? 2 : 3;
+    return 4;
+}
+
+// ---------------------------------------------------------- per-device state --
+
+struct PlanEntry {
+    std::vector<int32_t> cu;
+    int Hq, Hkv, D, window;
+    thd::WorkItem* d_items = nullptr;
+    int64_t n_items = 0;
+};
+
+struct DeviceState {
+    int* d_status = nullptr;
+    bool attr_set[kNumVariants] = {};
+    std::list<PlanEntry> plans;  // most recently used first
+};
+
+constexpr size_t kMaxPlans = 16;
+
+std::mutex g_mu;
+std::unordered_map<int, DeviceState> g_devices;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult qr{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr) ==
+                cudaSuccess &&
+            qr == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 3-D map over a [T, H, D] bf16 tensor: dims (D, H, T), box (64, 1, rows),
+// 128-byte swizzle; out-of-range rows read as zero.
+bool make_map(CUtensorMap* map, const void* base, int64_t T, int H, int D, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                          static_cast<cuuint64_t>(T)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2};
+    cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Returns the device state of the current device (created on first use).
+// Caller holds g_mu.
+int device_state(DeviceState** out, int* dev_out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return THD_ERR_CUDA;
+    auto it = g_devices.find(dev);
+    if (it == g_devices.end()) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return THD_ERR_CUDA;
+        if (major != 10 || minor != 0) return THD_ERR_UNSUPPORTED;
+        DeviceState st;
+        if (cudaMalloc(&st.d_status, sizeof(int)) != cudaSuccess) return THD_ERR_NO_MEMORY;
+        if (cudaMemset(st.d_status, 0, sizeof(int)) != cudaSuccess) return THD_ERR_CUDA;
+        it = g_devices.emplace(dev, std::move(st)).first;
+    }
+    *out = &it->second;
+    if (dev_out) *dev_out = dev;
+    return THD_OK;
+}
+
+// Finds or builds (and uploads) the plan for these arguments.  Caller holds g_mu.
+int get_plan(DeviceState* ds, const int32_t* cu, int n_docs, int Hq, int Hkv, int D, int window,
+             const KernelShape& ks, cudaStream_t stream, const PlanEntry** out) {
+    for (auto it = ds->plans.begin(); it != ds->plans.end(); ++it) {
+        if (it->Hq == Hq && it->Hkv == Hkv && it->D == D && it->window == window &&
+            it->cu.size() == static_cast<size_t>(n_docs) + 1 &&
+            std::memcmp(it->cu.data(), cu, sizeof(int32_t) * (n_docs + 1)) == 0) {
+            ds->plans.splice(ds->plans.begin(), ds->plans, it);
+            *out = &ds->plans.front();
+            return THD_OK;
+        }
+    }
+    std::vector<thd_work_item> items = thd::build_plan(cu, n_docs, Hq, Hkv, window, ks);
+    PlanEntry e;
+    e.cu.assign(cu, cu + n_docs + 1);
+    e.Hq = Hq;
+    e.Hkv = Hkv;
+    e.D = D;
+    e.window = window;
+    e.n_items = static_cast<int64_t>(items.size());
+    if (!items.empty()) {
+        const size_t bytes = items.size() * sizeof(thd::WorkItem);
+        if (cudaMalloc(&e.d_items, bytes) != cudaSuccess) return THD_ERR_NO_MEMORY;
+        if (cudaMemcpyAsync(e.d_items, items.data(), bytes, cudaMemcpyHostToDevice, stream) !=
+                cudaSuccess ||
+            cudaStreamSynchronize(stream) != cudaSuccess) {
+            cudaFree(e.d_items);
+            return THD_ERR_CUDA;
+        }
+    }
+    if (ds->plans.size() >= kMaxPlans) {
+        // cudaFree waits for kernels that may still read the evicted plan.
+        if (ds->plans.back().d_items) cudaFree(ds->plans.back().d_items);
+        ds->plans.pop_back();
+    }
+    ds->plans.push_front(std::move(e));
+    *out = &ds->plans.front();
+    return THD_OK;
+}
+
+template <class C>
+int launch(DeviceState* ds, int vidx, const PlanEntry& plan, const CUtensorMap& mq,
+           const CUtensorMap& mk, const CUtensorMap& mv, const thd::FwdParams& prm,
+           cudaStream_t stream) {
+    auto kern = thd::thd_attn_fwd_kernel<C>;
+    if (!ds->attr_set[vidx]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_ALLOC) != cudaSuccess)
+            return THD_ERR_CUDA;
+        ds->attr_set[vidx] = true;
+    }
+    kern<<<static_cast<unsigned>(plan.n_items), C::NUM_THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv,
+                                                                                      prm);
+    return cudaGetLastError() == cudaSuccess ? THD_OK : THD_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int thd_attn_abi_version(void) { return (1 << 16) | 0; }
+
+const char* thd_attn_status_string(int status) {
+    switch (status) {
+        case THD_OK: return "ok";
+        case THD_ERR_INVALID_ARG: return "invalid argument";
+        case THD_ERR_UNSUPPORTED: return "unsupported head dim or device (needs sm_100 and D in {64,128,256})";
+        case THD_ERR_CUDA: return "CUDA call failed";
+        case THD_ERR_TIMEOUT: return "kernel wait timed out (pipeline stalled)";
+        case THD_ERR_NO_MEMORY: return "out of device memory for the schedule cache";
+        default: return "unknown status";
+    }
+}
+
+int thd_attn_plan(const int32_t* cu_seqlens, int n_docs, int Hq, int Hkv, int D, int window,
+                  thd_work_item* items, int64_t capacity, int64_t* n_items) {
+    if (n_items == nullptr || capacity < 0) return THD_ERR_INVALID_ARG;
+    int rc = thd::validate_args(cu_seqlens, n_docs, Hq, Hkv, D, window);
+    if (rc != THD_OK) return rc;
+    KernelShape ks;
+    if (!thd::choose_kernel_shape(D, Hq / Hkv, &ks)) return THD_ERR_UNSUPPORTED;
+    std::vector<thd_work_item> v = thd::build_plan(cu_seqlens, n_docs, Hq, Hkv, window, ks);
+    *n_items = static_cast<int64_t>(v.size());
+    if (items != nullptr) {
+        const int64_t n = std::min<int64_t>(capacity, static_cast<int64_t>(v.size()));
+        std::memcpy(items, v.data(), sizeof(thd_work_item) * static_cast<size_t>(n));
+    }
+    return THD_OK;
+}
+
+int thd_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                 int n_docs, int Hq, int Hkv, int D, int window, float scale,
+                 const float* sinks_or_null, void* out, float* lse, void* stream_ptr) {
+    int rc = thd::validate_args(cu_seqlens, n_docs, Hq, Hkv, D, window);
+    if (rc != THD_OK) return rc;
+    if (!(std::isfinite(scale) && scale > 0.0f)) return THD_ERR_INVALID_ARG;
+    const int64_t T = cu_seqlens[n_docs];
+    if (T == 0) return THD_OK;
+    if (!q || !k || !v || !out) return THD_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return THD_ERR_INVALID_ARG;
+    if ((lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) ||
+        (sinks_or_null && (reinterpret_cast<uintptr_t>(sinks_or_null) & 3u)))
+        return THD_ERR_INVALID_ARG;
+    KernelShape ks;
+    if (!thd::choose_kernel_shape(D, Hq / Hkv, &ks)) return THD_ERR_UNSUPPORTED;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState* ds = nullptr;
+    rc = device_state(&ds, nullptr);
+    if (rc != THD_OK) return rc;
+    const PlanEntry* plan = nullptr;
+    rc = get_plan(ds, cu_seqlens, n_docs, Hq, Hkv, D, window, ks, stream, &plan);
+    if (rc != THD_OK) return rc;
+    if (plan->n_items == 0) return THD_OK;
+
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, q, T, Hq, D, 128) || !make_map(&mk, k, T, Hkv, D, ks.block_n) ||
+        !make_map(&mv, v, T, Hkv, D, ks.block_n))
+        return THD_ERR_CUDA;
+
+    thd::FwdParams prm;
+    prm.items = plan->d_items;
+    prm.out = static_cast<__nv_bfloat16*>(out);
+    prm.lse = lse;
+    prm.sinks = sinks_or_null;
+    prm.status = ds->d_status;
+    prm.Hq = Hq;
+    prm.G = Hq / Hkv;
+    prm.window = window;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+
+    switch (variant_index(ks)) {
+        case 0: return launch<Cfg64x2>(ds, 0, *plan, mq, mk, mv, prm, stream);
+        case 1: return launch<Cfg64x1>(ds, 1, *plan, mq, mk, mv, prm, stream);
+        case 2: return launch<Cfg128x2>(ds, 2, *plan, mq, mk, mv, prm, stream);
+        case 3: return launch<Cfg128x1>(ds, 3, *plan, mq, mk, mv, prm, stream);
+        default: return launch<Cfg256x1>(ds, 4, *plan, mq, mk, mv, prm, stream);
+    }
+}
+
+int thd_attn_get_error(void* stream_ptr) {
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return THD_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState* ds = nullptr;
+    int rc = device_state(&ds, nullptr);
+    if (rc != THD_OK) return rc;
+    int status = 0;
+    if (cudaMemcpy(&status, ds->d_status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return THD_ERR_CUDA;
+    if (status != 0 && cudaMemset(ds->d_status, 0, sizeof(int)) != cudaSuccess) return THD_ERR_CUDA;
+    return status;
+}
+
+}  // extern "C"

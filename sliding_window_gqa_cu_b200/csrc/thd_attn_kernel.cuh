@@ -1,0 +1,457 @@
+// Packed-THD sliding-window GQA attention forward for B200 (sm_100a).
+//
+// One CTA computes one work item of the host tile schedule: a 128-row query
+// tile of one document for NQ query heads that share one kv head (the
+// repeat_kv grouping of the "muse_glimmer.model" page), against n_kv key
+// tiles of BN keys.  Visible keys follow FlintMagiPlan.attention's window
+// parameter ("flint.magi" page): s <= j <= i and (W == 0 or j > i - W) for a
+// query i of document [s, e).  The per-head sink logit (FlintMagiPlan
+// .attention, sink parameter) starts the running max/sum of every row and so
+// joins the softmax denominator only.
+//
+// Warp roles (warp-specialised, all communication through mbarriers):
+//   warps 0 .. 4*NQ-1  softmax: warpgroup q owns query tile q; thread t owns
+//                      row t (= TMEM lane t).  Reads S from TMEM, masks edge
+//                      tiles, keeps the running max / sum, writes P (bf16)
+//                      back over S in TMEM, rescales O in TMEM when the max
+//                      grows by more than 2^8, and writes O/l and the LSE.
+//   warp 4*NQ          TMA producer: Q tiles once, then K/V tiles through an
+//                      NST-deep shared-memory ring (128-byte swizzle).
+//   warp 4*NQ+1        MMA issuer: S = Q K^T (both operands from shared
+//                      memory, K-major) and O += P V (P from TMEM, V from
+//                      shared memory, MN-major), fp32 accumulators in TMEM.
+//
+// TMEM columns: S[q][b] at (q*NSB + b)*BN (b < NSB buffers), O[q] after them.
+// With NSB = 1 the MMA order QK(j) PV(j) QK(j+1) keeps S/P of one tile live;
+// with NSB = 2, QK(j+1) runs while the softmax works on tile j.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+
+namespace thd {
+
+struct WorkItem {  // identical layout to thd_work_item in thd_attn.h
+    int32_t q0, q1, doc_start, head0;
+    int32_t kv_start, n_kv, n_heads, block_n;
+};
+
+// Error codes recorded in the device status word (THD_ERR_TIMEOUT family).
+constexpr int kStatusTimeout = -4;
+
+template <int D_, int NQ_, int NSB_, int BN_, int NST_>
+struct FwdConfig {
+    static constexpr int D = D_;
+    static constexpr int NQ = NQ_;    // query tiles (heads) per CTA
+    static constexpr int NSB = NSB_;  // S buffers per query tile
+    static constexpr int BN = BN_;    // keys per key tile
+    static constexpr int NST = NST_;  // K/V ring depth
+    static constexpr int BM = 128;    // query rows per tile (= TMEM lanes)
+
+    static constexpr int KCH = D / 64;                 // 128-byte column chunks
+    static constexpr int Q_BOX_BYTES = BM * 128;       // one chunk of a Q tile
+    static constexpr int Q_TILE_BYTES = BM * D * 2;
+    static constexpr int KV_BOX_BYTES = BN * 128;      // one chunk of a K/V tile
+    static constexpr int KV_TILE_BYTES = BN * D * 2;
+
+    static constexpr int TMEM_S = 0;
+    static constexpr int TMEM_O = NQ * NSB * BN;
+    static constexpr int TMEM_USED = TMEM_O + NQ * D;
+    static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64
+                                   : TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
+
+    static constexpr int NUM_SOFTMAX_WARPS = 4 * NQ;
+    static constexpr int PRODUCER_WARP = NUM_SOFTMAX_WARPS;
+    static constexpr int MMA_WARP = NUM_SOFTMAX_WARPS + 1;
+    static constexpr int NUM_THREADS = (NUM_SOFTMAX_WARPS + 2) * 32;
+
+    // mbarrier indices
+    static constexpr int B_Q_FULL = 0;
+    static constexpr int B_K_FULL = 1;
+    static constexpr int B_K_EMPTY = B_K_FULL + NST;
+    static constexpr int B_V_FULL = B_K_EMPTY + NST;
+    static constexpr int B_V_EMPTY = B_V_FULL + NST;
+    static constexpr int B_S_FULL = B_V_EMPTY + NST;   // [NQ][NSB]
+    static constexpr int B_P_FULL = B_S_FULL + NQ * NSB;
+    static constexpr int B_O_FULL = B_P_FULL + NQ;
+    static constexpr int B_DRAIN = B_O_FULL + NQ;
+    static constexpr int NUM_BARS = B_DRAIN + 1;
+
+    // shared memory layout (offsets from a 1024-byte aligned base)
+    static constexpr int SMEM_Q = 0;
+    static constexpr int SMEM_K = SMEM_Q + NQ * Q_TILE_BYTES;
+    static constexpr int SMEM_V = SMEM_K + NST * KV_TILE_BYTES;
+    static constexpr int SMEM_BAR = SMEM_V + NST * KV_TILE_BYTES;
+    static constexpr int SMEM_TMEM_SLOT = SMEM_BAR + NUM_BARS * 8;
+    static constexpr int SMEM_ABORT = SMEM_TMEM_SLOT + 4;
+    static constexpr int SMEM_BYTES = SMEM_ABORT + 4;
+    static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+
+    static_assert(D % 64 == 0 && D <= 256, "head dim must be 64, 128 or 256");
+    static_assert(BN % 32 == 0 && BN <= 256, "key tile must be a multiple of 32");
+    static_assert(TMEM_USED <= 512, "TMEM budget exceeded");
+    static_assert(SMEM_ALLOC <= 232448, "shared memory budget exceeded");
+};
+
+struct FwdParams {
+    const WorkItem* items;
+    __nv_bfloat16* out;  // [T, Hq, D]
+    float* lse;          // [T, Hq] or null
+    const float* sinks;  // [Hq] or null
+    int* status;         // device status word
+    int Hq;
+    int G;               // Hq / Hkv
+    int window;
+    float scale_log2;    // scale * log2(e)
+};
+
+// Wait by lane 0 of the calling warp; the result is broadcast to the warp so
+// that the warp-collective tcgen05 instructions after it stay convergent.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          int* status) {
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, status, kStatusTimeout);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
+// Bounded wait that ignores the abort flag: used while unwinding, to let
+// operations already in flight finish before the CTA exits.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > kWaitLimitNs) return;
+    }
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::NUM_THREADS, 1)
+thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                    const __grid_constant__ CUtensorMap tmap_k,
+                    const __grid_constant__ CUtensorMap tmap_v,
+                    const FwdParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = smem_addr(smem_raw);
+    uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
+    const uint32_t sbase = smem_addr(smem);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const WorkItem it = p.items[blockIdx.x];
+    const int n = it.n_kv;
+
+    auto bar = [&](int idx) -> uint32_t { return sbase + C::SMEM_BAR + 8u * idx; };
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::SMEM_ABORT);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SMEM_TMEM_SLOT);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(C::B_Q_FULL), 1);
+        for (int s = 0; s < C::NST; ++s) {
+            mbar_init(bar(C::B_K_FULL + s), 1);
+            mbar_init(bar(C::B_K_EMPTY + s), 1);
+            mbar_init(bar(C::B_V_FULL + s), 1);
+            mbar_init(bar(C::B_V_EMPTY + s), 1);
+        }
+        for (int i = 0; i < C::NQ * C::NSB; ++i) mbar_init(bar(C::B_S_FULL + i), 1);
+        for (int q = 0; q < C::NQ; ++q) {
+            mbar_init(bar(C::B_P_FULL + q), 4);
+            mbar_init(bar(C::B_O_FULL + q), 1);
+        }
+        mbar_init(bar(C::B_DRAIN), 1);
+        // A timeout recorded by an earlier CTA (or launch) makes every later
+        // CTA skip its work until the host reads and clears the status.
+        *abort_flag = *reinterpret_cast<volatile int*>(p.status) != 0 ? 1 : 0;
+        fence_barrier_init();
+    }
+    if (warp == C::MMA_WARP) {
+        tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const bool skip = *abort_flag != 0;
+
+    if (warp == C::PRODUCER_WARP) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0 && !skip) {
+            tma_prefetch_desc(&tmap_q);
+            tma_prefetch_desc(&tmap_k);
+            tma_prefetch_desc(&tmap_v);
+            const int g = it.head0 / p.G;
+            mbar_arrive_expect_tx(bar(C::B_Q_FULL), C::NQ * C::Q_TILE_BYTES);
+            for (int q = 0; q < C::NQ; ++q)
+                for (int c = 0; c < C::KCH; ++c)
+                    tma_load_3d(sbase + C::SMEM_Q + q * C::Q_TILE_BYTES + c * C::Q_BOX_BYTES,
+                                &tmap_q, bar(C::B_Q_FULL), c * 64, it.head0 + q, it.q0);
+            int last_k[C::NST], last_v[C::NST];
+            for (int s = 0; s < C::NST; ++s) last_k[s] = last_v[s] = -1;
+            bool ok = true;
+            for (int j = 0; j < n && ok; ++j) {
+                const int st = j % C::NST;
+                const uint32_t ph = (j / C::NST) & 1;
+                const int kt = it.kv_start + j * C::BN;
+                ok = mbar_wait(bar(C::B_K_EMPTY + st), ph ^ 1, abort_flag, p.status, kStatusTimeout);
+                if (!ok) break;
+                mbar_arrive_expect_tx(bar(C::B_K_FULL + st), C::KV_TILE_BYTES);
+                for (int c = 0; c < C::KCH; ++c)
+                    tma_load_3d(sbase + C::SMEM_K + st * C::KV_TILE_BYTES + c * C::KV_BOX_BYTES,
+                                &tmap_k, bar(C::B_K_FULL + st), c * 64, g, kt);
+                last_k[st] = j;
+                ok = mbar_wait(bar(C::B_V_EMPTY + st), ph ^ 1, abort_flag, p.status, kStatusTimeout);
+                if (!ok) break;
+                mbar_arrive_expect_tx(bar(C::B_V_FULL + st), C::KV_TILE_BYTES);
+                for (int c = 0; c < C::KCH; ++c)
+                    tma_load_3d(sbase + C::SMEM_V + st * C::KV_TILE_BYTES + c * C::KV_BOX_BYTES,
+                                &tmap_v, bar(C::B_V_FULL + st), c * 64, g, kt);
+                last_v[st] = j;
+            }
+            if (!ok) {
+                // Unwinding: let the loads already issued land before exit.
+                drain_wait(bar(C::B_Q_FULL), 0);
+                for (int s = 0; s < C::NST; ++s) {
+                    if (last_k[s] >= 0) drain_wait(bar(C::B_K_FULL + s), (last_k[s] / C::NST) & 1);
+                    if (last_v[s] >= 0) drain_wait(bar(C::B_V_FULL + s), (last_v[s] / C::NST) & 1);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == C::MMA_WARP) {
+        // -------------------------------------------------------- MMA issuer
+        if (lane == 0 && !skip) {
+            constexpr uint32_t idesc_qk = idesc_bf16_f32(128, C::BN, false);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::D, true);
+            auto issue_qk = [&](int q, int b, int st) {
+                const uint32_t d_tmem = tmem_base + C::TMEM_S + (q * C::NSB + b) * C::BN;
+                const uint32_t qa = sbase + C::SMEM_Q + q * C::Q_TILE_BYTES;
+                const uint32_t ka = sbase + C::SMEM_K + st * C::KV_TILE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < C::D / 16; ++kk) {
+                    const uint32_t koff = (kk & 3) * 32;  // 16 bf16 = 32 bytes along K
+                    const uint64_t a = smem_desc_sw128(qa + (kk >> 2) * C::Q_BOX_BYTES + koff, 16, 1024);
+                    const uint64_t b_ = smem_desc_sw128(ka + (kk >> 2) * C::KV_BOX_BYTES + koff, 16, 1024);
+                    mma_bf16_ss(d_tmem, a, b_, idesc_qk, kk > 0 ? 1u : 0u);
+                }
+            };
+            auto issue_pv = [&](int q, int b, int st, bool acc) {
+                const uint32_t d_tmem = tmem_base + C::TMEM_O + q * C::D;
+                const uint32_t p_tmem = tmem_base + C::TMEM_S + (q * C::NSB + b) * C::BN;
+                const uint32_t va = sbase + C::SMEM_V + st * C::KV_TILE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; ++kk) {
+                    const uint64_t b_ = smem_desc_sw128(va + kk * 16 * 128, C::KV_BOX_BYTES, 1024);
+                    mma_bf16_ts(d_tmem, p_tmem + kk * 8, b_, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+                }
+            };
+
+            bool ok = mbar_wait(bar(C::B_Q_FULL), 0, abort_flag, p.status, kStatusTimeout);
+            for (int jj = 0; ok && jj < C::NSB && jj < n; ++jj) {
+                const int st = jj % C::NST;
+                ok = mbar_wait(bar(C::B_K_FULL + st), (jj / C::NST) & 1, abort_flag, p.status,
+                               kStatusTimeout);
+                if (!ok) break;
+                tc_fence_after();
+                for (int q = 0; q < C::NQ; ++q) {
+                    issue_qk(q, jj % C::NSB, st);
+                    mma_commit(bar(C::B_S_FULL + q * C::NSB + jj % C::NSB));
+                }
+                mma_commit(bar(C::B_K_EMPTY + st));
+            }
+            for (int j = 0; ok && j < n; ++j) {
+                const int st = j % C::NST;
+                ok = mbar_wait(bar(C::B_V_FULL + st), (j / C::NST) & 1, abort_flag, p.status,
+                               kStatusTimeout);
+                if (!ok) break;
+                const int jn = j + C::NSB;
+                const bool has_next = jn < n;
+                const int stn = jn % C::NST;
+                for (int q = 0; q < C::NQ && ok; ++q) {
+                    ok = mbar_wait(bar(C::B_P_FULL + q), j & 1, abort_flag, p.status, kStatusTimeout);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(q, j % C::NSB, st, j > 0);
+                    mma_commit(bar(C::B_O_FULL + q));
+                    if (has_next) {
+                        if (q == 0) {
+                            ok = mbar_wait(bar(C::B_K_FULL + stn), (jn / C::NST) & 1, abort_flag,
+                                           p.status, kStatusTimeout);
+                            if (!ok) break;
+                            tc_fence_after();
+                        }
+                        issue_qk(q, jn % C::NSB, stn);
+                        mma_commit(bar(C::B_S_FULL + q * C::NSB + jn % C::NSB));
+                    }
+                }
+                if (!ok) break;
+                mma_commit(bar(C::B_V_EMPTY + st));
+                if (has_next) mma_commit(bar(C::B_K_EMPTY + stn));
+            }
+            // Every MMA issued by this thread has completed once this lands.
+            mma_commit(bar(C::B_DRAIN));
+            drain_wait(bar(C::B_DRAIN), 0);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax
+        const int q = warp >> 2;
+        const int wq = warp & 3;
+        const int row = wq * 32 + lane;
+        const int h = it.head0 + q;
+        const int i = it.q0 + row;  // token of this row
+        const int s_doc = it.doc_start;
+        const int r_lo = it.q0 > s_doc ? it.q0 : s_doc;
+        const int r_hi = it.q1 - 1;
+        const bool row_valid = i >= r_lo && i <= r_hi;
+        const int W = p.window;
+        const int lo_i = (W > 0 && i - W + 1 > s_doc) ? i - W + 1 : s_doc;
+        const float sl2 = p.scale_log2;
+        constexpr float kTau = 8.0f;  // rescale only when the max grows by > 2^8
+
+        float m_ref = -INFINITY;
+        float l = 0.0f;
+        if (p.sinks != nullptr) {
+            m_ref = p.sinks[h] * 1.4426950408889634f;
+            l = 1.0f;
+        }
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(wq * 32) << 16);
+        const uint32_t o_tmem = lane_base + C::TMEM_O + q * C::D;
+
+        bool ok = !skip;
+        for (int j = 0; ok && j < n; ++j) {
+            const int b = j % C::NSB;
+            ok = warp_wait(bar(C::B_S_FULL + q * C::NSB + b), (j / C::NSB) & 1, abort_flag, p.status);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t s_tmem = lane_base + C::TMEM_S + (q * C::NSB + b) * C::BN;
+            uint32_t sr[C::BN];
+#pragma unroll
+            for (int c = 0; c < C::BN / 32; ++c)
+                tmem_ld32(s_tmem + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < C::BN / 32; ++c)
+                reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+            float sv[C::BN];
+#pragma unroll
+            for (int c = 0; c < C::BN; ++c) sv[c] = __uint_as_float(sr[c]);
+
+            const int kt = it.kv_start + j * C::BN;
+            const bool full_tile = kt >= s_doc && kt + C::BN - 1 <= r_lo &&
+                                   (W == 0 || kt >= r_hi - W + 1);
+            if (!full_tile) {
+                const int c_lo = lo_i - kt;
+                const int c_hi = i - kt;
+#pragma unroll
+                for (int c = 0; c < C::BN; ++c)
+                    if (c < c_lo || c > c_hi) sv[c] = -INFINITY;
+            }
+            float mx[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) mx[u] = sv[u];
+#pragma unroll
+            for (int c = 8; c < C::BN; ++c) mx[c & 7] = fmaxf(mx[c & 7], sv[c]);
+            const float smax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            const float m_tile = smax * sl2;
+
+            float alpha = 1.0f;
+            bool rescale_o = false;
+            if (j == 0) {
+                if (m_tile > m_ref) {
+                    alpha = ex2_approx(m_ref - m_tile);
+                    m_ref = m_tile;
+                }
+            } else if (m_tile > m_ref + kTau) {
+                alpha = ex2_approx(m_ref - m_tile);
+                m_ref = m_tile;
+                rescale_o = true;
+            }
+            l *= alpha;
+            const float neg_m = (m_ref == -INFINITY) ? 0.0f : -m_ref;
+
+            float rs[4] = {0.f, 0.f, 0.f, 0.f};
+            uint32_t pk[C::BN / 2];
+#pragma unroll
+            for (int c = 0; c < C::BN / 2; ++c) {
+                const float p0 = ex2_approx(fmaf(sv[2 * c], sl2, neg_m));
+                const float p1 = ex2_approx(fmaf(sv[2 * c + 1], sl2, neg_m));
+                rs[c & 3] += p0 + p1;
+                pk[c] = pack_bf16x2(p0, p1);
+            }
+            l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+#pragma unroll
+            for (int c = 0; c < C::BN / 64; ++c)
+                tmem_st32(s_tmem + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[c * 32]));
+            if constexpr ((C::BN / 2) % 32 == 16)
+                tmem_st16(s_tmem + (C::BN / 64) * 32,
+                          *reinterpret_cast<const uint32_t(*)[16]>(&pk[(C::BN / 64) * 32]));
+            tmem_wait_st();
+
+            if (j > 0) {
+                // O must hold PV(j-1) before it is rescaled (and before PV(j)).
+                ok = warp_wait(bar(C::B_O_FULL + q), (j - 1) & 1, abort_flag, p.status);
+                if (!ok) break;
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, rescale_o)) {
+#pragma unroll 1
+                    for (int c = 0; c < C::D / 32; ++c) {
+                        uint32_t r[32];
+                        tmem_ld32(o_tmem + c * 32, r);
+                        tmem_wait_ld();
+                        reg_fence32(r);
+#pragma unroll
+                        for (int u = 0; u < 32; ++u)
+                            r[u] = __float_as_uint(__uint_as_float(r[u]) * alpha);
+                        tmem_st32(o_tmem + c * 32, r);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_P_FULL + q));
+        }
+
+        if (ok) ok = warp_wait(bar(C::B_O_FULL + q), (n - 1) & 1, abort_flag, p.status);
+        if (ok) {
+            tc_fence_after();
+            const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
+            __nv_bfloat16* orow = p.out + (static_cast<int64_t>(i) * p.Hq + h) * C::D;
+#pragma unroll 1
+            for (int c = 0; c < C::D / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(o_tmem + c * 32, r);
+                tmem_wait_ld();
+                reg_fence32(r);
+                uint32_t w[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u)
+                    w[u] = pack_bf16x2(__uint_as_float(r[2 * u]) * inv_l,
+                                       __uint_as_float(r[2 * u + 1]) * inv_l);
+                if (row_valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        dst[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+                }
+            }
+            if (row_valid && p.lse != nullptr)
+                p.lse[static_cast<int64_t>(i) * p.Hq + h] =
+                    l > 0.0f ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == C::MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+}  // namespace thd
