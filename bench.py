@@ -1,0 +1,386 @@
+#!/usr/bin/env python
+"""Benchmark of the packed-THD sliding-window GQA attention forward on B200.
+
+One step = one forward (thd_attn_fwd through the C ABI) over one synthetic
+pack.  Default workload: the 65,536-token pack (log-uniform document lengths
+in [1024, 32768], Hq=64, Hkv=8, D=128, full causal, learned sinks).  Metric:
+TFLOP/s over valid (unmasked) query-key pairs, FLOP = 4 * pairs * D * Hq.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line on stdout (rank 0).  Multi-GPU runs are launched with
+torchrun, one process per GPU; every rank runs its own pack of the same shape
+(no data-path collective), the timed region is bracketed by a barrier and a
+device synchronisation, and the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sliding_window_gqa_cu_b200 import metrics, multirank, workloads  # noqa: E402
+
+DEFAULT_WORKLOAD = "pack64k_gqa8_d128_causal_sink"
+METRIC = "THD varlen attention fwd TFLOP/s (valid pairs) and % of B200 BF16 peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DATASHEET_BF16_TFLOPS = 2250.0
+KERNEL_NAME = "thd_attn_fwd_kernel"
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=workloads.CONFIG_ORDER)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="truncate the pack to its first N tokens (small profiling cases)")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ------------------------------------------------------------------ helpers --
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sliding_window_gqa_cu_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".cpp", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_per_launch(workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = d.get(workload)
+    if not e or e.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken during the timed region."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, device: torch.device):
+        self.samples = []  # (host time, fields)
+        self.proc = None
+        self.error = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            t0 = time.time()
+            while not self.samples and time.time() - t0 < 10 and self.proc.poll() is None:
+                time.sleep(0.05)
+        except Exception as e:  # no nvidia-smi
+            self.error = str(e)
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) == len(self.FIELDS):
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.error}
+        win = [p for (t, p) in self.samples if t0 <= t <= t1] or [p for (_, p) in self.samples[-3:]]
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(p[0]) for p in win if num(p[0]) is not None]
+        mx = [num(p[1]) for p in win if num(p[1]) is not None]
+        pw = [num(p[2]) for p in win if num(p[2]) is not None]
+        reasons = sorted({r for p in win for r, v in zip(self.REASONS, p[3:]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(win),
+                "power_w_max": max(pw) if pw else None}
+
+
+# ------------------------------------------------------------ CPU baseline --
+
+def cpu_oracle_sample(pack, target_seconds: float, seed: int, max_rows: int = 1 << 20):
+    """Time the fp64 CPU oracle on random (token, head) rows of the pack until
+    about `target_seconds` of work is done.  Returns (TFLOP/s, seconds, rows,
+    flops, threads)."""
+    import oracle  # test infrastructure: only the CPU-baseline leg uses it
+    cfg = pack["config"]
+    T, Hq, D = pack["T"], cfg.Hq, cfg.D
+    rng = np.random.default_rng(seed)
+    lib = oracle.load()
+    done_rows, flops, spent = 0, 0, 0.0
+    batch = 64
+    while spent < target_seconds and done_rows < max_rows:
+        rows = np.stack([rng.integers(0, T, size=batch), rng.integers(0, Hq, size=batch)], axis=1)
+        t0 = time.perf_counter()
+        oracle.attention_rows(pack["q"], pack["k"], pack["v"], pack["cu_seqlens"], cfg.window,
+                              cfg.scale, rows, pack["sinks"], lib=lib)
+        spent += time.perf_counter() - t0
+        flops += metrics.row_flops(metrics.visible_keys(pack["cu_seqlens"], cfg.window, rows[:, 0]), D)
+        done_rows += batch
+        if spent < target_seconds / 8:
+            batch *= 2
+    return flops / spent / 1e12, spent, done_rows, flops, oracle.num_threads(lib)
+
+
+def workload_config(cfg, cu, pairs, extra=None):
+    d = {"workload": cfg.name, "tokens": int(cu[-1]), "documents": int(len(cu) - 1),
+         "Hq": cfg.Hq, "Hkv": cfg.Hkv, "head_dim": cfg.D, "window": cfg.window,
+         "sinks": cfg.sinks, "valid_pairs": int(pairs), "seed": 0,
+         "l2": "inputs larger than L2 (Q+K+V = %.2f GB > 126 MB), no flush"
+               % (int(cu[-1]) * (cfg.Hq + 2 * cfg.Hkv) * cfg.D * 2 / 1e9)}
+    if extra:
+        d.update(extra)
+    return d
+
+
+# ----------------------------------------------------------- reference arm --
+
+def run_reference(args, info):
+    """The fp64 CPU oracle timed as the reference arm (rank 0 only)."""
+    if not info.is_root:
+        return 0
+    cfg = workloads.CONFIGS[args.workload]
+    pack = workloads.make_pack(cfg, args.seed, T_override=args.tokens)
+    cu = pack["cu_seqlens"]
+    pairs = metrics.valid_pairs(cu, cfg.window)
+    # size one step to about 2 s of CPU work so the whole run stays within minutes
+    per_step = max(0.25, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_oracle_sample(pack, per_step, seed=1000 + _)
+    tot_flops, tot_s, tot_rows, threads = 0, 0.0, 0, 1
+    for s in range(args.steps):
+        _, spent, rows, flops, threads = cpu_oracle_sample(pack, per_step, seed=s)
+        tot_flops += flops
+        tot_s += spent
+        tot_rows += rows
+    value = tot_flops / tot_s / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": workload_config(cfg, cu, pairs),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{tot_rows} random (token, head) rows of the pack over "
+                                   f"{args.steps} steps (~{per_step:.2f} s each)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm --
+
+def run_ours(args, info):
+    import sliding_window_gqa_cu_b200 as swa
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the CUDA path has no CPU fallback)")
+    multirank.init("nccl")
+    device = torch.device("cuda", info.local_rank)
+    torch.cuda.set_device(device)
+    swa.load_library()
+
+    cfg = workloads.CONFIGS[args.workload]
+    pack = workloads.make_pack(cfg, args.seed, tensor_seed=multirank.tensor_seed(args.seed, info.rank),
+                               T_override=args.tokens)
+    cu = pack["cu_seqlens"]
+    T = pack["T"]
+    pairs = metrics.valid_pairs(cu, cfg.window)
+    flops = 4 * pairs * cfg.D * cfg.Hq
+    q, k, v = (pack[n].to(device) for n in "qkv")
+    sinks = pack["sinks"].to(device) if pack["sinks"] is not None else None
+    out = torch.empty((T, cfg.Hq, cfg.D), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((T, cfg.Hq), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        swa.thd_attn_fwd(q, k, v, cu, cfg.window, cfg.scale, sinks, out=out, lse=lse, stream=stream)
+
+    t_plan0 = time.perf_counter()
+    step()  # first call builds and uploads the tile schedule
+    torch.cuda.synchronize(device)
+    first_call_ms = (time.perf_counter() - t_plan0) * 1e3
+    status = swa.thd_attn_get_error(stream)
+    if status != 0:
+        raise RuntimeError(f"kernel reported status {status}")
+
+    clocks = ClockSampler(device)
+    for _ in range(args.warmup):
+        step()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    multirank.barrier(device)
+    torch.cuda.synchronize(device)
+    h0 = time.time()
+    start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    h1 = time.time()
+    multirank.barrier(device)
+    clocks.stop()
+    status = swa.thd_attn_get_error(stream)
+    if status != 0:
+        raise RuntimeError(f"kernel reported status {status}")
+    elapsed_ms = start.elapsed_time(end)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    max_ms = multirank.max_over_ranks(elapsed_ms, device)
+    max_launch = multirank.max_over_ranks(statistics.mean(launch_ms), device)
+    value = multirank.aggregate_rate(flops * args.steps, info.world, max_ms / 1e3) / 1e12
+
+    # end to end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (pack[n].pin_memory() for n in "qkv")
+        sh = pack["sinks"].pin_memory() if pack["sinks"] is not None else None
+        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        lh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh) + ((sh,) if sh is not None else ()))
+        d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
+
+        def e2e_step():
+            q.copy_(qh, non_blocking=True)
+            k.copy_(kh, non_blocking=True)
+            v.copy_(vh, non_blocking=True)
+            if sh is not None:
+                sinks.copy_(sh, non_blocking=True)
+            swa.thd_attn_fwd(q, k, v, cu, cfg.window, cfg.scale, sinks, out=out, lse=lse, stream=stream)
+            oh.copy_(out, non_blocking=True)
+            lh.copy_(lse, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        multirank.barrier(device)
+        torch.cuda.synchronize(device)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e2e_ms = multirank.max_over_ranks(e0.elapsed_time(e1), device)
+        e2e = {"value": multirank.aggregate_rate(flops * args.e2e_steps, info.world, e2e_ms / 1e3) / 1e12,
+               "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e2e_ms / args.e2e_steps}
+
+    peaks, peak_src = measured_peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = flops / (max_launch / 1e3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic_per_launch(cfg.name),
+                "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)" if peak_src == "measured"
+                else "fallback 1.59 PFLOP/s",
+                "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
+                "frac_of_datasheet_2250": achieved / DATASHEET_BF16_TFLOPS,
+                "kernel": KERNEL_NAME,
+                "algorithmic_flops_per_launch": flops,
+                "algorithmic_bytes_per_launch": metrics.algorithmic_bytes(T, cfg.Hq, cfg.Hkv, cfg.D)}
+
+    cpu = None
+    if info.is_root and info.world == 1 and not args.no_cpu_baseline:
+        tf, spent, rows, fl, threads = cpu_oracle_sample(pack, args.cpu_seconds, seed=12345)
+        cpu = {"value": tf, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"{rows} random (token, head) rows of the same pack, fp64, "
+                         f"{fl / 1e9:.1f} GFLOP in {spent:.1f} s"}
+
+    csum = clocks.summary(h0, h1)
+    if info.is_root:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": info.world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": workload_config(cfg, cu, pairs, {"parallelism": f"pack-parallel x{info.world}",
+                                                       "per_rank_tflop": flops / 1e12}),
+            "pct_of_peak": 100.0 * value / info.world / peak,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": args.steps, "clocks": {k: csum[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+            "first_call_ms_with_schedule_build": first_call_ms,
+        }
+        log(f"[bench] {cfg.name}: {max_ms / args.steps:.3f} ms/step, {value:.1f} TFLOP/s "
+            f"({100 * value / info.world / peak:.1f}% of measured {peak:.0f}, "
+            f"{100 * value / info.world / DATASHEET_BF16_TFLOPS:.1f}% of 2250), clocks {csum}")
+        print(json.dumps(line), flush=True)
+    multirank.shutdown()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    info = multirank.rank_info()
+    if args.impl == "reference":
+        return run_reference(args, info)
+    return run_ours(args, info)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
