@@ -54,7 +54,8 @@ enum thd_status {
     THD_ERR_UNSUPPORTED = -2,  /* head_dim not in {64,128,256}, or device is not sm_100 */
     THD_ERR_CUDA = -3,         /* a CUDA runtime/driver call failed */
     THD_ERR_TIMEOUT = -4,      /* a bounded wait inside the kernel ran out */
-    THD_ERR_NO_MEMORY = -5     /* the schedule cache could not be allocated */
+    THD_ERR_NO_MEMORY = -5,    /* the schedule cache could not be allocated */
+    THD_ERR_TOO_LARGE = -6     /* thd_attn_fwd_noalloc: the schedule exceeds its fixed scratch */
 };
 
 /*
@@ -127,6 +128,43 @@ typedef struct thd_work_item {
  */
 int thd_attn_plan(const int32_t* cu_seqlens, int n_docs, int Hq, int Hkv, int D, int window,
                   thd_work_item* items, int64_t capacity, int64_t* n_items);
+
+/*
+ * Allocation-free variant of thd_attn_fwd.  The pages have no counterpart of
+ * this entry point: it exists for callers that may not allocate device
+ * memory -- runtimes that reserve all device memory up front and hand out
+ * only pre-planned buffers, and latency-critical loops that cannot take the
+ * device-wide synchronisation cudaMalloc/cudaFree may cause.
+ *
+ * Arguments and results are those of thd_attn_fwd, plus
+ *   device_status_or_null  optional caller-owned device int.  If given, a
+ *              kernel stall is recorded there as THD_ERR_TIMEOUT (the caller
+ *              zeroes it; while it is non-zero, launches skip their work).
+ *              If NULL, the scratch's own status word is used and cleared
+ *              before each launch.
+ *
+ * Scratch: a fixed array inside the library's device image (one per GPU that
+ * loads the library, kept until the process exits) holds a 256-byte status
+ * header and up to 65,536 work items (2 MiB + 256 B).  A schedule needs
+ * ceil(len/128) items per document per query-head pair (per query head when
+ * Hq/Hkv is odd or D == 256); larger schedules return THD_ERR_TOO_LARGE
+ * before anything is enqueued.  No call allocates device or host heap memory
+ * (no cudaMalloc, cudaFree or allocating library routine).
+ *
+ * The first call on a device does the set-up (looks up the scratch's device
+ * address and clears its status header, synchronously): make that first call
+ * before any stream capture.  Every call shares the scratch and it keeps the
+ * last call's contents: the schedule is re-uploaded only when the arguments
+ * change.  Calls that overlap on the GPU (for example on two streams of one
+ * device) race on the scratch; serialise them.
+ */
+int thd_attn_fwd_noalloc(const void* q, const void* k, const void* v,
+                         const int32_t* cu_seqlens, int n_docs,
+                         int Hq, int Hkv, int D, int window, float scale,
+                         const float* sinks_or_null,
+                         void* out, float* lse,
+                         int* device_status_or_null,
+                         void* stream);
 
 /* ABI version of this header: (major << 16) | minor. */
 int thd_attn_abi_version(void);

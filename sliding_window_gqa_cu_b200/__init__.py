@@ -20,15 +20,15 @@ from typing import Optional
 
 import numpy as np
 
-__all__ = ["thd_attn_fwd", "thd_attn_get_error", "thd_attn_plan", "ThdAttnError", "library_path",
-           "load_library", "STATUS"]
+__all__ = ["thd_attn_fwd", "thd_attn_fwd_noalloc", "thd_attn_get_error", "thd_attn_plan",
+           "ThdAttnError", "library_path", "load_library", "STATUS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_NAME = "libthdattn.so"
 _lib = None
 
 STATUS = {0: "THD_OK", -1: "THD_ERR_INVALID_ARG", -2: "THD_ERR_UNSUPPORTED", -3: "THD_ERR_CUDA",
-          -4: "THD_ERR_TIMEOUT", -5: "THD_ERR_NO_MEMORY"}
+          -4: "THD_ERR_TIMEOUT", -5: "THD_ERR_NO_MEMORY", -6: "THD_ERR_TOO_LARGE"}
 
 WORK_ITEM_FIELDS = ("q0", "q1", "doc_start", "head0", "kv_start", "n_kv", "n_heads", "block_n")
 
@@ -71,6 +71,9 @@ def load_library():
                                   ctypes.POINTER(_WorkItem), ctypes.c_int64,
                                   ctypes.POINTER(ctypes.c_int64)]
     lib.thd_attn_plan.restype = c_int
+    lib.thd_attn_fwd_noalloc.argtypes = [vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int,
+                                         ctypes.c_float, vp, vp, vp, vp, vp]
+    lib.thd_attn_fwd_noalloc.restype = c_int
     lib.thd_attn_abi_version.argtypes = []
     lib.thd_attn_abi_version.restype = c_int
     _lib = lib
@@ -170,3 +173,39 @@ def thd_attn_get_error(stream=None) -> int:
     if stream is None:
         stream = torch.cuda.current_stream()
     return int(load_library().thd_attn_get_error(ctypes.c_void_p(stream.cuda_stream)))
+
+
+def thd_attn_fwd_noalloc(q, k, v, cu_seqlens, out, lse=None, window: int = 0,
+                         scale: Optional[float] = None, sinks=None, device_status=None,
+                         stream=None):
+    """Allocation-free forward for callers that may not allocate device memory.
+
+    Same computation as :func:`thd_attn_fwd`, but the caller supplies every
+    buffer (``out`` and, if wanted, ``lse``; optionally a device int32
+    ``device_status`` word) and the library uses only a fixed scratch array
+    compiled into its device image.  This wrapper allocates nothing either.
+    The first call on a device does a one-time synchronous set-up; calls that
+    overlap on the GPU share the scratch and must be serialised.
+    """
+    import torch
+
+    lib = load_library()
+    T, Hq, D = q.shape
+    Hkv = k.shape[1]
+    cu = _cu_array(cu_seqlens)
+    if scale is None:
+        scale = D ** -0.5
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        rc = lib.thd_attn_fwd_noalloc(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(),
+            cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), cu.size - 1,
+            Hq, Hkv, D, int(window), float(scale),
+            sinks.data_ptr() if sinks is not None else None,
+            out.data_ptr(), lse.data_ptr() if lse is not None else None,
+            device_status.data_ptr() if device_status is not None else None,
+            ctypes.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise ThdAttnError(rc, "thd_attn_fwd_noalloc")
+    return out, lse

@@ -14,7 +14,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libthdattn.so")
-SOURCES = [os.path.join(CSRC, "thd_attn_api.cu"), os.path.join(CSRC, "scheduler.cpp")]
+SOURCES = [os.path.join(CSRC, "thd_attn_api.cu"), os.path.join(CSRC, "thd_attn_noalloc.cu"),
+           os.path.join(CSRC, "scheduler.cpp")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("thd_attn_kernel.cuh", "sm100_ptx.cuh", "scheduler.h")] \
     + [os.path.join(ROOT, "include", "thd_attn.h")]
 

@@ -181,6 +181,7 @@ const char* thd_attn_status_string(int status) {
         case THD_ERR_CUDA: return "CUDA call failed";
         case THD_ERR_TIMEOUT: return "kernel wait timed out (pipeline stalled)";
         case THD_ERR_NO_MEMORY: return "out of device memory for the schedule cache";
+        case THD_ERR_TOO_LARGE: return "schedule larger than the allocation-free scratch (65,536 work items)";
         default: return "unknown status";
     }
 }
