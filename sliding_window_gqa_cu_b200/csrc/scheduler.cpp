@@ -9,13 +9,13 @@ bool choose_kernel_shape(int D, int group, KernelShape* out) {
     const bool pair = (group % 2) == 0;  // two heads of one kv group per CTA
     switch (D) {
         case 64:
-            *out = pair ? KernelShape{64, 2, 1, 128, 4} : KernelShape{64, 1, 2, 128, 4};
+            *out = pair ? KernelShape{64, 2, 1, 128, 8} : KernelShape{64, 1, 2, 128, 8};
             return true;
         case 128:
-            *out = pair ? KernelShape{128, 2, 1, 128, 2} : KernelShape{128, 1, 2, 128, 2};
+            *out = pair ? KernelShape{128, 2, 1, 128, 5} : KernelShape{128, 1, 2, 128, 6};
             return true;
         case 256:
-            *out = KernelShape{256, 1, 2, 64, 2};
+            *out = KernelShape{256, 1, 2, 64, 5};
             return true;
         default:
             return false;

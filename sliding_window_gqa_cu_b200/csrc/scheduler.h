@@ -21,7 +21,7 @@ struct KernelShape {
     int nq;       // query heads per work item (1 or 2)
     int nsb;      // S buffers per query tile
     int block_n;  // keys per key tile
-    int nst;      // K/V ring depth
+    int nslot;    // K/V ring slots (one K or V tile each)
 };
 
 // Returns false if the head dim is unsupported.

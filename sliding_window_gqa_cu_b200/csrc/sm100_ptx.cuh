@@ -58,10 +58,16 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 // the limit runs out, or if another role of the CTA has already aborted.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile int* abort_flag, int* status, int code) {
-    if (mbar_try_wait(bar, parity)) return true;
+    // Fast path: plain polling (try_wait itself suspends briefly in hardware).
+#pragma unroll 1
+    for (int spin = 0; spin < 256; ++spin)
+        if (mbar_try_wait(bar, parity)) return true;
+    // Slow path: check the clock and the abort conditions every 64 polls.
     const uint64_t t0 = global_timer_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+#pragma unroll 1
+        for (int spin = 0; spin < 64; ++spin)
+            if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
         if (*reinterpret_cast<volatile int*>(status) != 0) {  // another CTA gave up
             *abort_flag = 1;
@@ -230,7 +236,25 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
            (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Moves registers between warpgroups of a warp-specialised CTA.  Every warp of
+// the warpgroup must execute it; the increases of all warpgroups must fit in
+// what the decreases (and the launch allocation) leave.
+template <uint32_t N>
+__device__ __forceinline__ void regs_increase() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_decrease() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------------- math --
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
 
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;

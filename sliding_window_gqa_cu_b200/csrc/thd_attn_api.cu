@@ -23,11 +23,11 @@ using thd::KernelShape;
 
 // ------------------------------------------------------------ kernel shapes --
 
-using Cfg64x2 = thd::FwdConfig<64, 2, 1, 128, 4>;
-using Cfg64x1 = thd::FwdConfig<64, 1, 2, 128, 4>;
-using Cfg128x2 = thd::FwdConfig<128, 2, 1, 128, 2>;
-using Cfg128x1 = thd::FwdConfig<128, 1, 2, 128, 2>;
-using Cfg256x1 = thd::FwdConfig<256, 1, 2, 64, 2>;
+using Cfg64x2 = thd::FwdConfig<64, 2, 1, 128, 8>;
+using Cfg64x1 = thd::FwdConfig<64, 1, 2, 128, 8>;
+using Cfg128x2 = thd::FwdConfig<128, 2, 1, 128, 5>;
+using Cfg128x1 = thd::FwdConfig<128, 1, 2, 128, 6>;
+using Cfg256x1 = thd::FwdConfig<256, 1, 2, 64, 5>;
 
 constexpr int kNumVariants = 5;
 
@@ -157,6 +157,7 @@ int launch(DeviceState* ds, int vidx, const PlanEntry& plan, const CUtensorMap& 
            cudaStream_t stream) {
     auto kern = thd::thd_attn_fwd_kernel<C>;
     if (!ds->attr_set[vidx]) {
+        if (!thd::launch_registers_ok<C>()) return THD_ERR_UNSUPPORTED;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::SMEM_ALLOC) != cudaSuccess)
             return THD_ERR_CUDA;

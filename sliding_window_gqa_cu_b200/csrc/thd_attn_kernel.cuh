@@ -10,16 +10,15 @@
 // joins the softmax denominator only.
 //
 // Warp roles (warp-specialised, all communication through mbarriers):
-//   warps 0 .. 4*NQ-1  softmax: warpgroup q owns query tile q; thread t owns
-//                      row t (= TMEM lane t).  Reads S from TMEM, masks edge
-//                      tiles, keeps the running max / sum, writes P (bf16)
-//                      back over S in TMEM, rescales O in TMEM when the max
-//                      grows by more than 2^8, and writes O/l and the LSE.
-//   warp 4*NQ          TMA producer: Q tiles once, then K/V tiles through an
-//                      NST-deep shared-memory ring (128-byte swizzle).
-//   warp 4*NQ+1        MMA issuer: S = Q K^T (both operands from shared
-//                      memory, K-major) and O += P V (P from TMEM, V from
-//                      shared memory, MN-major), fp32 accumulators in TMEM.
+//   softmax warpgroups (one per query tile): thread t owns row t (= TMEM
+//     lane t).  Reads S from TMEM, masks edge tiles, keeps the running max
+//     and sum, rescales O in TMEM when the max grows by more than 2^8, and
+//     writes P (bf16) back over S for O += P V.
+//   control warpgroup: warp 0 is the TMA producer (Q tiles once, then K/V
+//     tiles through a ring of 128-byte-swizzled shared-memory slots), warp 1
+//     the MMA issuer: S = Q K^T (both operands from shared memory, K-major)
+//     and O += P V (P from TMEM, V from shared memory, MN-major), fp32
+//     accumulators in TMEM.
 //
 // TMEM columns: S[q][b] at (q*NSB + b)*BN (b < NSB buffers), O[q] after them.
 // With NSB = 1 the MMA order QK(j) PV(j) QK(j+1) keeps S/P of one tile live;
@@ -27,6 +26,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_runtime.h>
 #include <cstdint>
 
 #include "sm100_ptx.cuh"
@@ -38,17 +38,17 @@ struct WorkItem {  // identical layout to thd_work_item in thd_attn.h
     int32_t kv_start, n_kv, n_heads, block_n;
 };
 
-// Error codes recorded in the device status word (THD_ERR_TIMEOUT family).
+// Error code recorded in the device status word when a wait runs out.
 constexpr int kStatusTimeout = -4;
 
-template <int D_, int NQ_, int NSB_, int BN_, int NST_>
+template <int D_, int NQ_, int NSB_, int BN_, int NSLOT_>
 struct FwdConfig {
     static constexpr int D = D_;
-    static constexpr int NQ = NQ_;    // query tiles (heads) per CTA
-    static constexpr int NSB = NSB_;  // S buffers per query tile
-    static constexpr int BN = BN_;    // keys per key tile
-    static constexpr int NST = NST_;  // K/V ring depth
-    static constexpr int BM = 128;    // query rows per tile (= TMEM lanes)
+    static constexpr int NQ = NQ_;        // query tiles (heads) per CTA
+    static constexpr int NSB = NSB_;      // S buffers per query tile
+    static constexpr int BN = BN_;        // keys per key tile
+    static constexpr int NSLOT = NSLOT_;  // K/V ring slots (one K or V tile each)
+    static constexpr int BM = 128;        // query rows per tile (= TMEM lanes)
 
     static constexpr int KCH = D / 64;                 // 128-byte column chunks
     static constexpr int Q_BOX_BYTES = BM * 128;       // one chunk of a Q tile
@@ -62,37 +62,50 @@ struct FwdConfig {
     static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64
                                    : TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
 
+    // Warpgroups: NQ softmax warpgroups, then one control warpgroup whose
+    // warp 0 is the TMA producer and warp 1 the MMA issuer (warps 2-3 idle).
     static constexpr int NUM_SOFTMAX_WARPS = 4 * NQ;
     static constexpr int PRODUCER_WARP = NUM_SOFTMAX_WARPS;
     static constexpr int MMA_WARP = NUM_SOFTMAX_WARPS + 1;
-    static constexpr int NUM_THREADS = (NUM_SOFTMAX_WARPS + 2) * 32;
+    static constexpr int NUM_THREADS = (NUM_SOFTMAX_WARPS + 4) * 32;
+    // With three warpgroups a thread starts with 168 registers (3 warps per
+    // SM sub-partition); the control warpgroup hands most of its share to the
+    // softmax warpgroups: 2*128*208 + 128*88 = 384*168.
+    static constexpr bool REG_SPLIT = NQ == 2;
+    static constexpr int LAUNCH_REGS = 168;
+    static constexpr int SOFTMAX_REGS = 208;
+    static constexpr int CONTROL_REGS = 88;
+    static_assert(!REG_SPLIT || (NQ * 128 * SOFTMAX_REGS + 128 * CONTROL_REGS <=
+                                 NUM_THREADS * LAUNCH_REGS), "register split exceeds the launch");
 
     // mbarrier indices
     static constexpr int B_Q_FULL = 0;
-    static constexpr int B_K_FULL = 1;
-    static constexpr int B_K_EMPTY = B_K_FULL + NST;
-    static constexpr int B_V_FULL = B_K_EMPTY + NST;
-    static constexpr int B_V_EMPTY = B_V_FULL + NST;
-    static constexpr int B_S_FULL = B_V_EMPTY + NST;   // [NQ][NSB]
-    static constexpr int B_P_FULL = B_S_FULL + NQ * NSB;
-    static constexpr int B_O_FULL = B_P_FULL + NQ;
+    static constexpr int B_SLOT_FULL = 1;
+    static constexpr int B_SLOT_EMPTY = B_SLOT_FULL + NSLOT;
+    static constexpr int B_S_FULL = B_SLOT_EMPTY + NSLOT;  // [NQ][NSB]
+    static constexpr int B_P_FULL = B_S_FULL + NQ * NSB;   // P written, O rescaled
+    static constexpr int B_O_FULL = B_P_FULL + NQ;         // PV done
     static constexpr int B_DRAIN = B_O_FULL + NQ;
     static constexpr int NUM_BARS = B_DRAIN + 1;
 
     // shared memory layout (offsets from a 1024-byte aligned base)
     static constexpr int SMEM_Q = 0;
-    static constexpr int SMEM_K = SMEM_Q + NQ * Q_TILE_BYTES;
-    static constexpr int SMEM_V = SMEM_K + NST * KV_TILE_BYTES;
-    static constexpr int SMEM_BAR = SMEM_V + NST * KV_TILE_BYTES;
+    static constexpr int SMEM_SLOTS = SMEM_Q + NQ * Q_TILE_BYTES;
+    static constexpr int SMEM_BAR = SMEM_SLOTS + NSLOT * KV_TILE_BYTES;
     static constexpr int SMEM_TMEM_SLOT = SMEM_BAR + NUM_BARS * 8;
     static constexpr int SMEM_ABORT = SMEM_TMEM_SLOT + 4;
     static constexpr int SMEM_BYTES = SMEM_ABORT + 4;
     static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
 
     static_assert(D % 64 == 0 && D <= 256, "head dim must be 64, 128 or 256");
-    static_assert(BN % 32 == 0 && BN <= 256, "key tile must be a multiple of 32");
+    static_assert(BN % 64 == 0 && BN <= 256, "key tile must be a multiple of 64");
     static_assert(TMEM_USED <= 512, "TMEM budget exceeded");
     static_assert(SMEM_ALLOC <= 232448, "shared memory budget exceeded");
+    // Every wait of the MMA issuer is for a position whose slot was released
+    // by an MMA it has already issued (V(j) is released right after PV(j),
+    // K(j) right after QK(j)), so two slots already cannot deadlock; more
+    // slots only let the producer run further ahead.
+    static_assert(NSLOT >= 2, "K/V ring needs two slots");
 };
 
 struct FwdParams {
@@ -128,6 +141,29 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
     }
 }
 
+// Exponentials of key columns [C0, C0 + 32*NCH) of one row: p = 2^(s*sl2 - m),
+// two elements per packed FMA, summed into acc and written to TMEM as bf16
+// pairs (key k goes to column k/2 of the S/P buffer).
+template <int C0, int NCH, int BN>
+__device__ __forceinline__ void exp_and_store_p(const float (&sv)[BN], float2 sl2x2, float2 negm2,
+                                                uint32_t p_tmem, float2& acc0, float2& acc1) {
+#pragma unroll
+    for (int cc = 0; cc < NCH; ++cc) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const int c = C0 + cc * 32 + 2 * u;
+            const float2 x = __ffma2_rn(make_float2(sv[c], sv[c + 1]), sl2x2, negm2);
+            const float p0 = ex2_approx(x.x);
+            const float p1 = ex2_approx(x.y);
+            if (u & 1) acc1 = __fadd2_rn(acc1, make_float2(p0, p1));
+            else acc0 = __fadd2_rn(acc0, make_float2(p0, p1));
+            pk[u] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(p_tmem + (C0 / 2) + cc * 16, pk);
+    }
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::NUM_THREADS, 1)
 thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
@@ -150,11 +186,9 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
 
     if (threadIdx.x == 0) {
         mbar_init(bar(C::B_Q_FULL), 1);
-        for (int s = 0; s < C::NST; ++s) {
-            mbar_init(bar(C::B_K_FULL + s), 1);
-            mbar_init(bar(C::B_K_EMPTY + s), 1);
-            mbar_init(bar(C::B_V_FULL + s), 1);
-            mbar_init(bar(C::B_V_EMPTY + s), 1);
+        for (int s = 0; s < C::NSLOT; ++s) {
+            mbar_init(bar(C::B_SLOT_FULL + s), 1);
+            mbar_init(bar(C::B_SLOT_EMPTY + s), 1);
         }
         for (int i = 0; i < C::NQ * C::NSB; ++i) mbar_init(bar(C::B_S_FULL + i), 1);
         for (int q = 0; q < C::NQ; ++q) {
@@ -177,7 +211,9 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
     const uint32_t tmem_base = *tmem_slot;
     const bool skip = *abort_flag != 0;
 
-    if (warp == C::PRODUCER_WARP) {
+    if (warp >= C::NUM_SOFTMAX_WARPS) {
+      if constexpr (C::REG_SPLIT) regs_decrease<C::CONTROL_REGS>();
+      if (warp == C::PRODUCER_WARP) {
         // ------------------------------------------------------ TMA producer
         if (lane == 0 && !skip) {
             tma_prefetch_desc(&tmap_q);
@@ -189,115 +225,118 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 for (int c = 0; c < C::KCH; ++c)
                     tma_load_3d(sbase + C::SMEM_Q + q * C::Q_TILE_BYTES + c * C::Q_BOX_BYTES,
                                 &tmap_q, bar(C::B_Q_FULL), c * 64, it.head0 + q, it.q0);
-            int last_k[C::NST], last_v[C::NST];
-            for (int s = 0; s < C::NST; ++s) last_k[s] = last_v[s] = -1;
+            // Ring positions: 2j holds K(j), 2j+1 holds V(j); position p uses
+            // slot p % NSLOT.  A load waits only for the slot's previous tile.
+            int issued = 0;
             bool ok = true;
-            for (int j = 0; j < n && ok; ++j) {
-                const int st = j % C::NST;
-                const uint32_t ph = (j / C::NST) & 1;
-                const int kt = it.kv_start + j * C::BN;
-                ok = mbar_wait(bar(C::B_K_EMPTY + st), ph ^ 1, abort_flag, p.status, kStatusTimeout);
+            for (int pos = 0; pos < 2 * n && ok; ++pos) {
+                const int slot = pos % C::NSLOT;
+                ok = mbar_wait(bar(C::B_SLOT_EMPTY + slot), ((pos / C::NSLOT) & 1) ^ 1, abort_flag,
+                               p.status, kStatusTimeout);
                 if (!ok) break;
-                mbar_arrive_expect_tx(bar(C::B_K_FULL + st), C::KV_TILE_BYTES);
+                const CUtensorMap* map = (pos & 1) ? &tmap_v : &tmap_k;
+                const int kt = it.kv_start + (pos >> 1) * C::BN;
+                mbar_arrive_expect_tx(bar(C::B_SLOT_FULL + slot), C::KV_TILE_BYTES);
                 for (int c = 0; c < C::KCH; ++c)
-                    tma_load_3d(sbase + C::SMEM_K + st * C::KV_TILE_BYTES + c * C::KV_BOX_BYTES,
-                                &tmap_k, bar(C::B_K_FULL + st), c * 64, g, kt);
-                last_k[st] = j;
-                ok = mbar_wait(bar(C::B_V_EMPTY + st), ph ^ 1, abort_flag, p.status, kStatusTimeout);
-                if (!ok) break;
-                mbar_arrive_expect_tx(bar(C::B_V_FULL + st), C::KV_TILE_BYTES);
-                for (int c = 0; c < C::KCH; ++c)
-                    tma_load_3d(sbase + C::SMEM_V + st * C::KV_TILE_BYTES + c * C::KV_BOX_BYTES,
-                                &tmap_v, bar(C::B_V_FULL + st), c * 64, g, kt);
-                last_v[st] = j;
+                    tma_load_3d(sbase + C::SMEM_SLOTS + slot * C::KV_TILE_BYTES + c * C::KV_BOX_BYTES,
+                                map, bar(C::B_SLOT_FULL + slot), c * 64, g, kt);
+                issued = pos + 1;
             }
             if (!ok) {
                 // Unwinding: let the loads already issued land before exit.
+                // Only the last load issued into each slot can still be in
+                // flight (earlier ones were consumed before the slot was reused).
                 drain_wait(bar(C::B_Q_FULL), 0);
-                for (int s = 0; s < C::NST; ++s) {
-                    if (last_k[s] >= 0) drain_wait(bar(C::B_K_FULL + s), (last_k[s] / C::NST) & 1);
-                    if (last_v[s] >= 0) drain_wait(bar(C::B_V_FULL + s), (last_v[s] / C::NST) & 1);
-                }
+                for (int pos = issued - C::NSLOT > 0 ? issued - C::NSLOT : 0; pos < issued; ++pos)
+                    drain_wait(bar(C::B_SLOT_FULL + pos % C::NSLOT), (pos / C::NSLOT) & 1);
             }
         }
         __syncwarp();
-    } else if (warp == C::MMA_WARP) {
+      } else if (warp == C::MMA_WARP) {
         // -------------------------------------------------------- MMA issuer
         if (lane == 0 && !skip) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, C::BN, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::D, true);
-            auto issue_qk = [&](int q, int b, int st) {
+            // Descriptor bases; per instruction only the start address moves
+            // (adding offset >> 4 to the low field cannot carry: shared
+            // memory addresses stay below 2^18).
+            const uint64_t dq0 = smem_desc_sw128(sbase + C::SMEM_Q, 16, 1024);
+            const uint64_t dk0 = smem_desc_sw128(sbase + C::SMEM_SLOTS, 16, 1024);
+            const uint64_t dv0 = smem_desc_sw128(sbase + C::SMEM_SLOTS, C::KV_BOX_BYTES, 1024);
+            auto issue_qk = [&](int q, int b, int slot) {
                 const uint32_t d_tmem = tmem_base + C::TMEM_S + (q * C::NSB + b) * C::BN;
-                const uint32_t qa = sbase + C::SMEM_Q + q * C::Q_TILE_BYTES;
-                const uint32_t ka = sbase + C::SMEM_K + st * C::KV_TILE_BYTES;
+                const uint64_t dq = dq0 + ((q * C::Q_TILE_BYTES) >> 4);
+                const uint64_t dk = dk0 + ((slot * C::KV_TILE_BYTES) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < C::D / 16; ++kk) {
-                    const uint32_t koff = (kk & 3) * 32;  // 16 bf16 = 32 bytes along K
-                    const uint64_t a = smem_desc_sw128(qa + (kk >> 2) * C::Q_BOX_BYTES + koff, 16, 1024);
-                    const uint64_t b_ = smem_desc_sw128(ka + (kk >> 2) * C::KV_BOX_BYTES + koff, 16, 1024);
-                    mma_bf16_ss(d_tmem, a, b_, idesc_qk, kk > 0 ? 1u : 0u);
+                    // 16 bf16 = 32 bytes along K inside a 128-byte chunk
+                    const uint32_t qo = ((kk >> 2) * C::Q_BOX_BYTES + (kk & 3) * 32) >> 4;
+                    const uint32_t ko = ((kk >> 2) * C::KV_BOX_BYTES + (kk & 3) * 32) >> 4;
+                    mma_bf16_ss(d_tmem, dq + qo, dk + ko, idesc_qk, kk > 0 ? 1u : 0u);
                 }
             };
-            auto issue_pv = [&](int q, int b, int st, bool acc) {
+            // O += P V over the BN keys of one tile (K = 16 per instruction).
+            auto issue_pv = [&](int q, int b, int slot, bool acc) {
                 const uint32_t d_tmem = tmem_base + C::TMEM_O + q * C::D;
                 const uint32_t p_tmem = tmem_base + C::TMEM_S + (q * C::NSB + b) * C::BN;
-                const uint32_t va = sbase + C::SMEM_V + st * C::KV_TILE_BYTES;
+                const uint64_t dv = dv0 + ((slot * C::KV_TILE_BYTES) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; ++kk) {
-                    const uint64_t b_ = smem_desc_sw128(va + kk * 16 * 128, C::KV_BOX_BYTES, 1024);
-                    mma_bf16_ts(d_tmem, p_tmem + kk * 8, b_, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+                    mma_bf16_ts(d_tmem, p_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_pv,
+                                (acc || kk > 0) ? 1u : 0u);
                 }
             };
 
+            auto wait_slot = [&](int pos) -> bool {
+                return mbar_wait(bar(C::B_SLOT_FULL + pos % C::NSLOT), (pos / C::NSLOT) & 1,
+                                 abort_flag, p.status, kStatusTimeout);
+            };
             bool ok = mbar_wait(bar(C::B_Q_FULL), 0, abort_flag, p.status, kStatusTimeout);
             for (int jj = 0; ok && jj < C::NSB && jj < n; ++jj) {
-                const int st = jj % C::NST;
-                ok = mbar_wait(bar(C::B_K_FULL + st), (jj / C::NST) & 1, abort_flag, p.status,
-                               kStatusTimeout);
+                ok = wait_slot(2 * jj);
                 if (!ok) break;
                 tc_fence_after();
                 for (int q = 0; q < C::NQ; ++q) {
-                    issue_qk(q, jj % C::NSB, st);
+                    issue_qk(q, jj % C::NSB, (2 * jj) % C::NSLOT);
                     mma_commit(bar(C::B_S_FULL + q * C::NSB + jj % C::NSB));
                 }
-                mma_commit(bar(C::B_K_EMPTY + st));
+                mma_commit(bar(C::B_SLOT_EMPTY + (2 * jj) % C::NSLOT));
             }
             for (int j = 0; ok && j < n; ++j) {
-                const int st = j % C::NST;
-                ok = mbar_wait(bar(C::B_V_FULL + st), (j / C::NST) & 1, abort_flag, p.status,
-                               kStatusTimeout);
+                const int vslot = (2 * j + 1) % C::NSLOT;
+                ok = wait_slot(2 * j + 1);
                 if (!ok) break;
                 const int jn = j + C::NSB;
                 const bool has_next = jn < n;
-                const int stn = jn % C::NST;
+                const int kslot = (2 * jn) % C::NSLOT;
                 for (int q = 0; q < C::NQ && ok; ++q) {
                     ok = mbar_wait(bar(C::B_P_FULL + q), j & 1, abort_flag, p.status, kStatusTimeout);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_pv(q, j % C::NSB, st, j > 0);
+                    issue_pv(q, j % C::NSB, vslot, j > 0);
                     mma_commit(bar(C::B_O_FULL + q));
+                    if (q == C::NQ - 1) mma_commit(bar(C::B_SLOT_EMPTY + vslot));  // V(j) done
                     if (has_next) {
                         if (q == 0) {
-                            ok = mbar_wait(bar(C::B_K_FULL + stn), (jn / C::NST) & 1, abort_flag,
-                                           p.status, kStatusTimeout);
+                            ok = wait_slot(2 * jn);
                             if (!ok) break;
                             tc_fence_after();
                         }
-                        issue_qk(q, jn % C::NSB, stn);
+                        issue_qk(q, jn % C::NSB, kslot);
                         mma_commit(bar(C::B_S_FULL + q * C::NSB + jn % C::NSB));
+                        if (q == C::NQ - 1) mma_commit(bar(C::B_SLOT_EMPTY + kslot));  // K(jn) done
                     }
                 }
-                if (!ok) break;
-                mma_commit(bar(C::B_V_EMPTY + st));
-                if (has_next) mma_commit(bar(C::B_K_EMPTY + stn));
             }
             // Every MMA issued by this thread has completed once this lands.
             mma_commit(bar(C::B_DRAIN));
             drain_wait(bar(C::B_DRAIN), 0);
         }
         __syncwarp();
+      }
     } else {
         // ------------------------------------------------------------ softmax
+        if constexpr (C::REG_SPLIT) regs_increase<C::SOFTMAX_REGS>();
         const int q = warp >> 2;
         const int wq = warp & 3;
         const int row = wq * 32 + lane;
@@ -350,13 +389,11 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 for (int c = 0; c < C::BN; ++c)
                     if (c < c_lo || c > c_hi) sv[c] = -INFINITY;
             }
-            float mx[8];
+            // Row max: 3-input max over pairs, four independent chains.
+            float mx[4] = {sv[0], sv[1], sv[2], sv[3]};
 #pragma unroll
-            for (int u = 0; u < 8; ++u) mx[u] = sv[u];
-#pragma unroll
-            for (int c = 8; c < C::BN; ++c) mx[c & 7] = fmaxf(mx[c & 7], sv[c]);
-            const float smax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            for (int c = 4; c < C::BN; c += 2) mx[(c >> 1) & 3] = max3f(mx[(c >> 1) & 3], sv[c], sv[c + 1]);
+            const float smax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             const float m_tile = smax * sl2;
 
             float alpha = 1.0f;
@@ -374,47 +411,53 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
             l *= alpha;
             const float neg_m = (m_ref == -INFINITY) ? 0.0f : -m_ref;
 
-            float rs[4] = {0.f, 0.f, 0.f, 0.f};
-            uint32_t pk[C::BN / 2];
+            // O must hold PV(j-1) before it is rescaled and before PV(j)
+            // starts.  With one S buffer that is implied by S(j) being ready
+            // (QK(j) was issued after PV(j-1)); with two it is waited for,
+            // once per step: here if O is rescaled, else before P(j) is
+            // published (which also keeps the P barriers from running two
+            // phases ahead of the MMA issuer).
+            const bool warp_rescale = j > 0 && __any_sync(0xffffffffu, rescale_o);
+            bool o_ready = C::NSB == 1 || j == 0;
+            if (warp_rescale) {
+                if (!o_ready) {
+                    ok = warp_wait(bar(C::B_O_FULL + q), (j - 1) & 1, abort_flag, p.status);
+                    if (!ok) break;
+                    tc_fence_after();
+                    o_ready = true;
+                }
+#pragma unroll 1
+                for (int c = 0; c < C::D / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(o_tmem + c * 32, r);
+                    tmem_wait_ld();
+                    reg_fence32(r);
 #pragma unroll
-            for (int c = 0; c < C::BN / 2; ++c) {
-                const float p0 = ex2_approx(fmaf(sv[2 * c], sl2, neg_m));
-                const float p1 = ex2_approx(fmaf(sv[2 * c + 1], sl2, neg_m));
-                rs[c & 3] += p0 + p1;
-                pk[c] = pack_bf16x2(p0, p1);
+                    for (int u = 0; u < 32; u += 2) {
+                        const float2 y = __fmul2_rn(
+                            make_float2(__uint_as_float(r[u]), __uint_as_float(r[u + 1])),
+                            make_float2(alpha, alpha));
+                        r[u] = __float_as_uint(y.x);
+                        r[u + 1] = __float_as_uint(y.y);
+                    }
+                    tmem_st32(o_tmem + c * 32, r);
+                }
+                tmem_wait_st();
             }
-            l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-#pragma unroll
-            for (int c = 0; c < C::BN / 64; ++c)
-                tmem_st32(s_tmem + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[c * 32]));
-            if constexpr ((C::BN / 2) % 32 == 16)
-                tmem_st16(s_tmem + (C::BN / 64) * 32,
-                          *reinterpret_cast<const uint32_t(*)[16]>(&pk[(C::BN / 64) * 32]));
-            tmem_wait_st();
 
-            if (j > 0) {
-                // O must hold PV(j-1) before it is rescaled (and before PV(j)).
+            const float2 sl2x2 = make_float2(sl2, sl2);
+            const float2 negm2 = make_float2(neg_m, neg_m);
+            float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+            exp_and_store_p<0, C::BN / 32, C::BN>(sv, sl2x2, negm2, s_tmem, acc0, acc1);
+            tmem_wait_st();
+            if (!o_ready) {
                 ok = warp_wait(bar(C::B_O_FULL + q), (j - 1) & 1, abort_flag, p.status);
                 if (!ok) break;
-                tc_fence_after();
-                if (__any_sync(0xffffffffu, rescale_o)) {
-#pragma unroll 1
-                    for (int c = 0; c < C::D / 32; ++c) {
-                        uint32_t r[32];
-                        tmem_ld32(o_tmem + c * 32, r);
-                        tmem_wait_ld();
-                        reg_fence32(r);
-#pragma unroll
-                        for (int u = 0; u < 32; ++u)
-                            r[u] = __float_as_uint(__uint_as_float(r[u]) * alpha);
-                        tmem_st32(o_tmem + c * 32, r);
-                    }
-                    tmem_wait_st();
-                }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(C::B_P_FULL + q));
+            l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
         }
 
         if (ok) ok = warp_wait(bar(C::B_O_FULL + q), (n - 1) & 1, abort_flag, p.status);
@@ -451,6 +494,20 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
     if (warp == C::MMA_WARP) {
         tc_fence_after();
         tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// Host check before the first launch of a shape: the register split above
+// assumes the kernel starts with LAUNCH_REGS registers per thread; with fewer,
+// setmaxnreg.inc could never be satisfied.
+template <class C>
+inline bool launch_registers_ok() {
+    if constexpr (!C::REG_SPLIT) {
+        return true;
+    } else {
+        cudaFuncAttributes a{};
+        if (cudaFuncGetAttributes(&a, thd_attn_fwd_kernel<C>) != cudaSuccess) return false;
+        return a.numRegs >= C::LAUNCH_REGS;
     }
 }
 

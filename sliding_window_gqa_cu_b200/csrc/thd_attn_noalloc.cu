@@ -59,11 +59,11 @@ std::mutex g_mu;
 NoAllocDevice g_dev[kMaxDevices];
 thd_work_item g_host_items[kMaxItems];
 
-using NCfg64x2 = thd::FwdConfig<64, 2, 1, 128, 4>;
-using NCfg64x1 = thd::FwdConfig<64, 1, 2, 128, 4>;
-using NCfg128x2 = thd::FwdConfig<128, 2, 1, 128, 2>;
-using NCfg128x1 = thd::FwdConfig<128, 1, 2, 128, 2>;
-using NCfg256x1 = thd::FwdConfig<256, 1, 2, 64, 2>;
+using NCfg64x2 = thd::FwdConfig<64, 2, 1, 128, 8>;
+using NCfg64x1 = thd::FwdConfig<64, 1, 2, 128, 8>;
+using NCfg128x2 = thd::FwdConfig<128, 2, 1, 128, 5>;
+using NCfg128x1 = thd::FwdConfig<128, 1, 2, 128, 6>;
+using NCfg256x1 = thd::FwdConfig<256, 1, 2, 64, 5>;
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -155,6 +155,7 @@ int launch(NoAllocDevice* st, int vidx, int64_t n_items, const CUtensorMap& mq,
            cudaStream_t stream) {
     auto kern = thd::thd_attn_fwd_kernel<C>;
     if (!st->attr_set[vidx]) {
+        if (!thd::launch_registers_ok<C>()) return THD_ERR_UNSUPPORTED;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::SMEM_ALLOC) != cudaSuccess)
             return THD_ERR_CUDA;
