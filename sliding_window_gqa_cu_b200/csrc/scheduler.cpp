@@ -6,16 +6,21 @@
 namespace thd {
 
 bool choose_kernel_shape(int D, int group, KernelShape* out) {
-    const bool pair = (group % 2) == 0;  // two heads of one kv group per CTA
+    // One CTA per item with two heads of one kv group (even group) or one
+    // head; at D = 256 with an even group, the CTA-pair kernel (one head per
+    // CTA, two per item), whose M = 256 instructions keep N = 256 PV and
+    // N = 128 QK at the tensor core's full rate.  (At D = 128 the pair
+    // kernel measured slower than the one-CTA kernel, so it is not used.)
+    const bool two = (group % 2) == 0;
     switch (D) {
         case 64:
-            *out = pair ? KernelShape{64, 2, 1, 128, 8} : KernelShape{64, 1, 2, 128, 8};
+            *out = two ? KernelShape{64, 2, 1, 128, 8, false} : KernelShape{64, 1, 2, 128, 8, false};
             return true;
         case 128:
-            *out = pair ? KernelShape{128, 2, 1, 128, 5} : KernelShape{128, 1, 2, 128, 6};
+            *out = two ? KernelShape{128, 2, 1, 128, 5, false} : KernelShape{128, 1, 2, 128, 6, false};
             return true;
         case 256:
-            *out = KernelShape{256, 1, 2, 64, 5};
+            *out = two ? KernelShape{256, 2, 1, 128, 4, true} : KernelShape{256, 1, 2, 64, 5, false};
             return true;
         default:
             return false;

@@ -22,6 +22,7 @@ struct KernelShape {
     int nsb;      // S buffers per query tile
     int block_n;  // keys per key tile
     int nslot;    // K/V ring slots (one K or V tile each)
+    bool pair;    // CTA-pair kernel (nq heads split over two CTAs)
 };
 
 // Returns false if the head dim is unsupported.

@@ -20,6 +20,25 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
+// One lane of a converged warp (elect.sync): the issuing lane of warp-wide
+// tcgen05 issue loops, whose operands stay warp-uniform.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "elect.sync _|P, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
+// Busy-waits for `ns` nanoseconds of wall clock (used only while unwinding).
+__device__ __forceinline__ void spin_ns(uint64_t ns) {
+    const uint64_t t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < ns) {
+    }
+}
+
 // ---------------------------------------------------------------- mbarrier --
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -87,8 +106,8 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// 3-D tiled load of one box into shared memory; completion is signalled on
-// `bar` as transaction bytes.  No cluster multicast.
+// 3-D tiled load of one box into this CTA's shared memory (one destination);
+// completion is signalled on `bar` as transaction bytes.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int32_t c0, int32_t c1, int32_t c2) {
     asm volatile(
@@ -211,6 +230,121 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+// ------------------------------------------------- CTA pairs (2-CTA MMA) --
+// A cluster of two CTAs shares each MMA: the leader (rank 0) issues
+// tcgen05.mma.cta_group::2 with M = 256; each CTA supplies 128 rows of A and
+// half of B (split along N) from its own shared memory and receives its 128
+// rows of D in its own TMEM.
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+// Arrive on an mbarrier of any CTA of the cluster.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Non-blocking check of a phase (no suspension).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done) : "r"(bar), "r"(parity) : "memory");
+    return done != 0;
+}
+
+// Makes this thread's generic-proxy shared-memory writes visible to the async
+// proxy (TMA, tensor core).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+                 "r"(d) : "memory");
+}
+
+// Waits on barriers that the other CTA of the pair (or the pair's MMA
+// commits) complete.  Scope-wise these are the same waits as mbar_wait; the
+// pair's data (shared memory written by TMA, TMEM written by tcgen05) is
+// ordered by the transaction counts and the tcgen05 fences, not by the
+// barrier's memory scope.
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
+                                                  volatile int* abort_flag, int* status, int code) {
+    return mbar_wait(bar, parity, abort_flag, status, code);
+}
+
+// TMA load into this CTA's shared memory (one destination) whose transaction
+// bytes complete on an mbarrier of either CTA of the pair (`bar` is a
+// shared::cluster address).
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                 int32_t c0, int32_t c1, int32_t c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(dst_smem), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+// M = 256 MMAs over the CTA pair (issued by the leader CTA only).
+__device__ __forceinline__ void mma2_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
+__device__ __forceinline__ void mma2_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
+// Arrive on the mbarrier at address `bar` in both CTAs of the pair once every
+// pair MMA issued so far by this thread has completed.
+__device__ __forceinline__ void mma2_commit_both(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(bar), "h"(static_cast<uint16_t>(3)) : "memory");
+}
+
 // ------------------------------------------------------------- descriptors --
 
 // Shared-memory matrix descriptor (sm_100 format): start address, leading and
@@ -260,6 +394,32 @@ __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x on the FMA pipe for two values at once, so that part of the softmax
+// exponentials bypass the MUFU unit.  Cody-Waite reduction: n = round(x)
+// (adding 1.5*2^23 leaves round(x) in the low mantissa bits), f = x - n in
+// [-1/2, 1/2], 2^f from a degree-3 polynomial, and 2^n added to the exponent
+// field.  The coefficients are a relative-error minimax fit computed by
+// sliding_window_gqa_cu_b200/fit_exp2_poly.py (max relative error 7.5e-5).
+// Inputs are clamped at -125 (below that the result is < 2^-124 instead of
+// smaller; irrelevant next to a softmax sum that is at least one).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f;
+    constexpr float kC2 = 0.2426111251115799f, kC3 = 0.0551716685295105f;
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    x.x = fmaxf(x.x, -125.0f);
+    x.y = fmaxf(x.y, -125.0f);
+    const float2 t = __fadd2_rn(x, make_float2(kMagic, kMagic));
+    const float2 n = __fadd2_rn(t, make_float2(-kMagic, -kMagic));
+    const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);
+    float2 p = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
+    p = __ffma2_rn(p, f, make_float2(kC1, kC1));
+    p = __ffma2_rn(p, f, make_float2(kC0, kC0));
+    // (bits(t) << 23) == n << 23 modulo 2^32: the magic's own bits shift out.
+    const int ex = __float_as_int(t.x) * (1 << 23) + __float_as_int(p.x);
+    const int ey = __float_as_int(t.y) * (1 << 23) + __float_as_int(p.y);
+    return make_float2(__int_as_float(ex), __int_as_float(ey));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -16,6 +16,7 @@
 #include "../../include/thd_attn.h"
 #include "scheduler.h"
 #include "thd_attn_kernel.cuh"
+#include "thd_attn_pair_kernel.cuh"
 
 namespace {
 
@@ -28,10 +29,12 @@ using Cfg64x1 = thd::FwdConfig<64, 1, 2, 128, 8>;
 using Cfg128x2 = thd::FwdConfig<128, 2, 1, 128, 5>;
 using Cfg128x1 = thd::FwdConfig<128, 1, 2, 128, 6>;
 using Cfg256x1 = thd::FwdConfig<256, 1, 2, 64, 5>;
+using PairCfg256 = thd::PairConfig<256, 1, 128, 4>;  // 2 heads per item over a CTA pair
 
-constexpr int kNumVariants = 5;
+constexpr int kNumVariants = 6;
 
 int variant_index(const KernelShape& ks) {
+    if (ks.pair) return 5;
     if (ks.D == 64) return ks.nq == 2 ? 0 : 1;
     if (ks.D == 128) return ks.nq == 2 ? 2 : 3;
     return 4;
@@ -168,6 +171,24 @@ int launch(DeviceState* ds, int vidx, const PlanEntry& plan, const CUtensorMap& 
     return cudaGetLastError() == cudaSuccess ? THD_OK : THD_ERR_CUDA;
 }
 
+// CTA-pair shapes: two CTAs (one cluster) per work item.
+template <class C>
+int launch_pair(DeviceState* ds, int vidx, const PlanEntry& plan, const CUtensorMap& mq,
+                const CUtensorMap& mk, const CUtensorMap& mv, const thd::FwdParams& prm,
+                cudaStream_t stream) {
+    auto kern = thd::thd_attn_fwd_pair_kernel<C>;
+    if (!ds->attr_set[vidx]) {
+        if (!thd::pair_launch_registers_ok<C>()) return THD_ERR_UNSUPPORTED;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_ALLOC) != cudaSuccess)
+            return THD_ERR_CUDA;
+        ds->attr_set[vidx] = true;
+    }
+    kern<<<static_cast<unsigned>(2 * plan.n_items), C::NUM_THREADS, C::SMEM_ALLOC, stream>>>(
+        mq, mk, mv, prm);
+    return cudaGetLastError() == cudaSuccess ? THD_OK : THD_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -231,7 +252,9 @@ int thd_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_
     if (plan->n_items == 0) return THD_OK;
 
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, q, T, Hq, D, 128) || !make_map(&mk, k, T, Hkv, D, ks.block_n) ||
+    // The pair kernel loads half of each K tile (half the keys) per CTA.
+    if (!make_map(&mq, q, T, Hq, D, 128) ||
+        !make_map(&mk, k, T, Hkv, D, ks.pair ? ks.block_n / 2 : ks.block_n) ||
         !make_map(&mv, v, T, Hkv, D, ks.block_n))
         return THD_ERR_CUDA;
 
@@ -251,7 +274,8 @@ int thd_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_
         case 1: return launch<Cfg64x1>(ds, 1, *plan, mq, mk, mv, prm, stream);
         case 2: return launch<Cfg128x2>(ds, 2, *plan, mq, mk, mv, prm, stream);
         case 3: return launch<Cfg128x1>(ds, 3, *plan, mq, mk, mv, prm, stream);
-        default: return launch<Cfg256x1>(ds, 4, *plan, mq, mk, mv, prm, stream);
+        case 4: return launch<Cfg256x1>(ds, 4, *plan, mq, mk, mv, prm, stream);
+        default: return launch_pair<PairCfg256>(ds, 5, *plan, mq, mk, mv, prm, stream);
     }
 }
 

@@ -31,6 +31,10 @@
 
 #include "sm100_ptx.cuh"
 
+#ifndef THD_EXP_EMU
+#define THD_EXP_EMU 1
+#endif
+
 namespace thd {
 
 struct WorkItem {  // identical layout to thd_work_item in thd_attn.h
@@ -49,6 +53,8 @@ struct FwdConfig {
     static constexpr int BN = BN_;        // keys per key tile
     static constexpr int NSLOT = NSLOT_;  // K/V ring slots (one K or V tile each)
     static constexpr int BM = 128;        // query rows per tile (= TMEM lanes)
+    // Element pairs (out of every 4) whose exponential runs on the FMA pipe.
+    static constexpr int EXP_EMU = THD_EXP_EMU;
 
     static constexpr int KCH = D / 64;                 // 128-byte column chunks
     static constexpr int Q_BOX_BYTES = BM * 128;       // one chunk of a Q tile
@@ -144,7 +150,8 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 // Exponentials of key columns [C0, C0 + 32*NCH) of one row: p = 2^(s*sl2 - m),
 // two elements per packed FMA, summed into acc and written to TMEM as bf16
 // pairs (key k goes to column k/2 of the S/P buffer).
-template <int C0, int NCH, int BN>
+// EMU of every 4 element pairs take the FMA-pipe polynomial instead of MUFU.
+template <int C0, int NCH, int BN, int EMU>
 __device__ __forceinline__ void exp_and_store_p(const float (&sv)[BN], float2 sl2x2, float2 negm2,
                                                 uint32_t p_tmem, float2& acc0, float2& acc1) {
 #pragma unroll
@@ -154,8 +161,15 @@ __device__ __forceinline__ void exp_and_store_p(const float (&sv)[BN], float2 sl
         for (int u = 0; u < 16; ++u) {
             const int c = C0 + cc * 32 + 2 * u;
             const float2 x = __ffma2_rn(make_float2(sv[c], sv[c + 1]), sl2x2, negm2);
-            const float p0 = ex2_approx(x.x);
-            const float p1 = ex2_approx(x.y);
+            float p0, p1;
+            if ((u & 3) >= 4 - EMU) {
+                const float2 e = exp2_poly2(x);
+                p0 = e.x;
+                p1 = e.y;
+            } else {
+                p0 = ex2_approx(x.x);
+                p1 = ex2_approx(x.y);
+            }
             if (u & 1) acc1 = __fadd2_rn(acc1, make_float2(p0, p1));
             else acc0 = __fadd2_rn(acc0, make_float2(p0, p1));
             pk[u] = pack_bf16x2(p0, p1);
@@ -448,7 +462,7 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
             const float2 sl2x2 = make_float2(sl2, sl2);
             const float2 negm2 = make_float2(neg_m, neg_m);
             float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-            exp_and_store_p<0, C::BN / 32, C::BN>(sv, sl2x2, negm2, s_tmem, acc0, acc1);
+            exp_and_store_p<0, C::BN / 32, C::BN, C::EXP_EMU>(sv, sl2x2, negm2, s_tmem, acc0, acc1);
             tmem_wait_st();
             if (!o_ready) {
                 ok = warp_wait(bar(C::B_O_FULL + q), (j - 1) & 1, abort_flag, p.status);

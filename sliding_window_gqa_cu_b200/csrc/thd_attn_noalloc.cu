@@ -33,6 +33,7 @@
 #include "../../include/thd_attn.h"
 #include "scheduler.h"
 #include "thd_attn_kernel.cuh"
+#include "thd_attn_pair_kernel.cuh"
 
 namespace {
 
@@ -47,7 +48,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 struct NoAllocDevice {
     bool ready = false;
     unsigned char* scratch = nullptr;  // device address of g_noalloc_scratch
-    bool attr_set[5] = {};
+    bool attr_set[6] = {};
     // arguments of the schedule now in the scratch (valid when have_plan)
     bool have_plan = false;
     int n_docs = 0, Hq = 0, Hkv = 0, D = 0, window = 0;
@@ -64,6 +65,7 @@ using NCfg64x1 = thd::FwdConfig<64, 1, 2, 128, 8>;
 using NCfg128x2 = thd::FwdConfig<128, 2, 1, 128, 5>;
 using NCfg128x1 = thd::FwdConfig<128, 1, 2, 128, 6>;
 using NCfg256x1 = thd::FwdConfig<256, 1, 2, 64, 5>;
+using NPairCfg256 = thd::PairConfig<256, 1, 128, 4>;  // 2 heads per item over a CTA pair
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -166,6 +168,23 @@ int launch(NoAllocDevice* st, int vidx, int64_t n_items, const CUtensorMap& mq,
     return cudaGetLastError() == cudaSuccess ? THD_OK : THD_ERR_CUDA;
 }
 
+template <class C>
+int launch_pair(NoAllocDevice* st, int vidx, int64_t n_items, const CUtensorMap& mq,
+                const CUtensorMap& mk, const CUtensorMap& mv, const thd::FwdParams& prm,
+                cudaStream_t stream) {
+    auto kern = thd::thd_attn_fwd_pair_kernel<C>;
+    if (!st->attr_set[vidx]) {
+        if (!thd::pair_launch_registers_ok<C>()) return THD_ERR_UNSUPPORTED;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_ALLOC) != cudaSuccess)
+            return THD_ERR_CUDA;
+        st->attr_set[vidx] = true;
+    }
+    kern<<<static_cast<unsigned>(2 * n_items), C::NUM_THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv,
+                                                                                      prm);
+    return cudaGetLastError() == cudaSuccess ? THD_OK : THD_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" int thd_attn_fwd_noalloc(const void* q, const void* k, const void* v,
@@ -231,7 +250,8 @@ extern "C" int thd_attn_fwd_noalloc(const void* q, const void* k, const void* v,
     }
 
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, q, T, Hq, D, 128) || !make_map(&mk, k, T, Hkv, D, ks.block_n) ||
+    if (!make_map(&mq, q, T, Hq, D, 128) ||
+        !make_map(&mk, k, T, Hkv, D, ks.pair ? ks.block_n / 2 : ks.block_n) ||
         !make_map(&mv, v, T, Hkv, D, ks.block_n))
         return THD_ERR_CUDA;
 
@@ -246,6 +266,7 @@ extern "C" int thd_attn_fwd_noalloc(const void* q, const void* k, const void* v,
     prm.window = window;
     prm.scale_log2 = scale * 1.4426950408889634f;
 
+    if (ks.pair) return launch_pair<NPairCfg256>(st, 5, n_items, mq, mk, mv, prm, stream);
     if (D == 64) {
         return ks.nq == 2 ? launch<NCfg64x2>(st, 0, n_items, mq, mk, mv, prm, stream)
                           : launch<NCfg64x1>(st, 1, n_items, mq, mk, mv, prm, stream);

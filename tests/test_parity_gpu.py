@@ -78,9 +78,13 @@ CASES = [
     ([390, 5, 128, 1, 200], 8, 2, 128, 129, False),
     ([600], 4, 4, 128, 0, True),                  # MHA, G = 1
     ([333, 64], 6, 2, 128, 50, False),            # G = 3
-    ([520, 3], 16, 1, 256, 0, True),              # MQA, D = 256
+    ([520, 3], 16, 1, 256, 0, True),              # MQA, D = 256 (CTA pair)
     ([520, 3], 4, 2, 256, 65, False),
     ([700, 0, 0], 2, 1, 256, 64, True),
+    ([400, 77], 4, 2, 128, 0, True),              # one CTA, two heads (group 2)
+    ([300, 9], 12, 2, 128, 100, True),            # group 6: one CTA, two heads
+    ([500, 130], 16, 2, 128, 0, True),            # group 8
+    ([300, 45], 3, 1, 256, 0, True),              # odd group at D = 256: one CTA, one head
 ]
 
 

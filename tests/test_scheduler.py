@@ -83,6 +83,7 @@ def test_plan_random_packs():
 
 def test_gqa_heads_adjacent_and_shapes():
     cu = workloads.cu_seqlens_from_lengths([1000, 400])
+    # D = 128: one CTA per item, two heads of one kv group
     plan = swa.thd_attn_plan(cu, 32, 8, 128, 0)
     assert set(plan["n_heads"]) == {2} and set(plan["block_n"]) == {128}
     # consecutive items of one (query tile, kv head) form one run
@@ -93,7 +94,11 @@ def test_gqa_heads_adjacent_and_shapes():
             assert k not in seen, "items of one (tile, kv group) are split apart"
             seen.add(k)
         prev = k
-    assert set(swa.thd_attn_plan(cu, 16, 1, 256, 64)["block_n"]) == {64}
+    # D = 256: CTA-pair items of two heads with 128-key tiles; odd groups fall
+    # back to one head per CTA with 64-key tiles
+    p256 = swa.thd_attn_plan(cu, 16, 1, 256, 64)
+    assert set(p256["block_n"]) == {128} and set(p256["n_heads"]) == {2}
+    assert set(swa.thd_attn_plan(cu, 3, 1, 256, 64)["block_n"]) == {64}
     assert set(swa.thd_attn_plan(cu, 3, 1, 128, 0)["n_heads"]) == {1}
 
 
