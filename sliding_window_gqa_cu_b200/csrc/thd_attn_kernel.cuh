@@ -32,7 +32,7 @@
 #include "sm100_ptx.cuh"
 
 #ifndef THD_EXP_EMU
-#define THD_EXP_EMU 1
+#define THD_EXP_EMU 0
 #endif
 
 namespace thd {
