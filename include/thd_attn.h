@@ -120,7 +120,9 @@ typedef struct thd_work_item {
 
 /*
  * Host-only: build the tile schedule thd_attn_fwd uses for these arguments,
- * ordered longest first (non-increasing n_kv; heads of one kv group adjacent).
+ * ordered by kv head (so the CTAs in flight share one head's K/V in L2) and,
+ * within a kv head, longest first (non-increasing n_kv), the heads of one
+ * (query tile, kv head) adjacent.
  * No CUDA call is made.  `items` may be NULL to query the count.  Writes
  * min(count, capacity) items and sets *n_items = count.  Returns THD_OK or
  * THD_ERR_INVALID_ARG / THD_ERR_UNSUPPORTED for the same argument errors as

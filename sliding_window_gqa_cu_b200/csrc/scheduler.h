@@ -31,8 +31,8 @@ bool choose_kernel_shape(int D, int group, KernelShape* out);
 // Host argument checks shared by every entry point (no CUDA calls).
 int validate_args(const int32_t* cu_seqlens, int n_docs, int Hq, int Hkv, int D, int window);
 
-// Builds the longest-first work list.  cu_seqlens must have passed
-// validate_args.
+// Builds the work list (kv head by kv head, longest first within a head).
+// cu_seqlens must have passed validate_args.
 std::vector<thd_work_item> build_plan(const int32_t* cu_seqlens, int n_docs, int Hq, int Hkv,
                                       int window, const KernelShape& ks);
 

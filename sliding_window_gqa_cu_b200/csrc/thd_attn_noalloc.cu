@@ -103,9 +103,9 @@ int64_t count_items(const int32_t* cu, int n_docs, int Hq, const thd::KernelShap
     return tiles * (Hq / ks.nq);
 }
 
-// Writes the longest-first schedule into g_host_items (same items and order as
-// the cached path's plan: the sort key below is unique and reproduces the
-// generation order among items of equal length).
+// Writes the schedule into g_host_items (same items and order as the cached
+// path's plan: kv group, then longest first; the sort key below is unique
+// and reproduces the generation order among items of equal length).
 void write_plan(const int32_t* cu, int n_docs, int Hq, int Hkv, int window,
                 const thd::KernelShape& ks, int64_t n) {
     const int G = Hq / Hkv, BN = ks.block_n;
@@ -124,7 +124,8 @@ void write_plan(const int32_t* cu, int n_docs, int Hq, int Hkv, int window,
                                                       q1 - n_kv * BN, n_kv, ks.nq, BN};
         }
     }
-    std::sort(g_host_items, g_host_items + n, [](const thd_work_item& a, const thd_work_item& b) {
+    std::sort(g_host_items, g_host_items + n, [G](const thd_work_item& a, const thd_work_item& b) {
+        if (a.head0 / G != b.head0 / G) return a.head0 / G < b.head0 / G;
         if (a.n_kv != b.n_kv) return a.n_kv > b.n_kv;
         if (a.doc_start != b.doc_start) return a.doc_start < b.doc_start;
         if (a.q1 != b.q1) return a.q1 > b.q1;

@@ -1,8 +1,8 @@
 """The host tile schedule covers every visible (query, key, head) triple
 exactly as the kernel needs: each (token, head) row is owned by exactly one
 work item, every visible key of the row lies in the item's key tiles, no key
-tile is fully masked, and items run longest first with the heads of one kv
-group adjacent.  Checked by brute force against the window definition of
+tile is fully masked, and items run one kv group after another, longest first
+within a group, with the heads of one (query tile, kv group) adjacent.  Checked by brute force against the window definition of
 FlintMagiPlan.attention ("flint.magi" page)."""
 import numpy as np
 import pytest
@@ -50,8 +50,11 @@ def check_plan(cu, Hq, Hkv, D, window):
             tile_hit[(lo - ks) // bn:(hi - ks) // bn + 1] = True
         assert tile_hit.all(), "a key tile with no visible pair was scheduled"
     assert (owner >= 0).all(), "some (token, head) row is not covered"
-    nkv = plan["n_kv"]
-    assert (np.diff(nkv) <= 0).all(), "not longest first"
+    # kv groups in order, longest first within each group
+    grp = plan["head0"] // G
+    assert (np.diff(grp) >= 0).all(), "kv groups interleaved"
+    for g in np.unique(grp):
+        assert (np.diff(plan["n_kv"][grp == g]) <= 0).all(), "not longest first within a group"
     return plan
 
 
