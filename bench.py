@@ -38,7 +38,13 @@ METRIC = "THD varlen attention fwd TFLOP/s (valid pairs) and % of B200 BF16 peak
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DATASHEET_BF16_TFLOPS = 2250.0
-KERNEL_NAME = "thd_attn_fwd_kernel"
+
+
+def kernel_name(D: int, group: int) -> str:
+    """The kernel the library launches for this shape (label only): the
+    CTA-pair kernel with the key-split softmax at head dim 256 with an even
+    GQA group, else the one-CTA kernel."""
+    return "thd_attn_fwd_split_kernel" if D == 256 and group % 2 == 0 else "thd_attn_fwd_kernel"
 
 
 def log(*a):
@@ -341,7 +347,7 @@ def run_ours(args, info):
                 else "fallback 1.59 PFLOP/s",
                 "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
                 "frac_of_datasheet_2250": achieved / DATASHEET_BF16_TFLOPS,
-                "kernel": KERNEL_NAME,
+                "kernel": kernel_name(cfg.D, cfg.Hq // cfg.Hkv),
                 "algorithmic_flops_per_launch": flops,
                 "algorithmic_bytes_per_launch": metrics.algorithmic_bytes(T, cfg.Hq, cfg.Hkv, cfg.D)}
 

@@ -7,10 +7,11 @@ namespace thd {
 
 bool choose_kernel_shape(int D, int group, KernelShape* out) {
     // One CTA per item with two heads of one kv group (even group) or one
-    // head; at D = 256 with an even group, the CTA-pair kernel (one head per
-    // CTA, two per item), whose M = 256 instructions keep N = 256 PV and
-    // N = 128 QK at the tensor core's full rate.  (At D = 128 the pair
-    // kernel measured slower than the one-CTA kernel, so it is not used.)
+    // head; at D = 256 with an even group, the CTA-pair kernel with the
+    // key-split softmax (one head per CTA, two per item), whose M = 256
+    // instructions keep N = 256 PV and N = 128 QK at the tensor core's full
+    // rate.  (At D = 128 the pair kernels measured slower than the one-CTA
+    // kernel: there the exponentials take as long as the MMAs per tile.)
     const bool two = (group % 2) == 0;
     switch (D) {
         case 64:
@@ -20,7 +21,7 @@ bool choose_kernel_shape(int D, int group, KernelShape* out) {
             *out = two ? KernelShape{128, 2, 1, 128, 5, false} : KernelShape{128, 1, 2, 128, 6, false};
             return true;
         case 256:
-            *out = two ? KernelShape{256, 2, 1, 128, 4, true} : KernelShape{256, 1, 2, 64, 5, false};
+            *out = two ? KernelShape{256, 2, 2, 128, 4, true} : KernelShape{256, 1, 2, 64, 5, false};
             return true;
         default:
             return false;
@@ -36,6 +37,16 @@ int validate_args(const int32_t* cu_seqlens, int n_docs, int Hq, int Hkv, int D,
         if (cu_seqlens[d + 1] < cu_seqlens[d]) return THD_ERR_INVALID_ARG;
     if (D != 64 && D != 128 && D != 256) return THD_ERR_UNSUPPORTED;
     return THD_OK;
+}
+
+int kv_groups_per_chunk(int64_t T, int D, int Hkv) {
+    // K and V of one kv head over the whole pack, bf16.
+    const int64_t per_group = T * static_cast<int64_t>(D) * 2 * 2;
+    constexpr int64_t kL2Budget = 48ll << 20;  // well inside the 126 MB L2
+    int64_t c = per_group > 0 ? kL2Budget / per_group : Hkv;
+    if (c < 1) c = 1;
+    if (c > Hkv) c = Hkv;
+    return static_cast<int>(c);
 }
 
 std::vector<thd_work_item> build_plan(const int32_t* cu, int n_docs, int Hq, int Hkv, int window,
@@ -67,14 +78,15 @@ std::vector<thd_work_item> build_plan(const int32_t* cu, int n_docs, int Hq, int
                                                   ks.nq, BN});
         }
     }
-    // One kv group after another, longest first within a group.  The CTAs in
-    // flight then read the K/V of one kv head only (at most T * D * 4 bytes,
-    // 33.5 MB for a 64k-token pack at D = 128), which the 126 MB L2 holds,
-    // instead of every group of the longest documents at once.  The stable
-    // sort keeps the items of one (query tile, kv group) next to each other.
-    std::stable_sort(items.begin(), items.end(), [G](const thd_work_item& a, const thd_work_item& b) {
-        const int ga = a.head0 / G, gb = b.head0 / G;
-        if (ga != gb) return ga < gb;
+    // Kv groups in chunks whose K/V fits in L2, longest first within a chunk.
+    // The CTAs in flight then read the K/V of a few kv heads only instead of
+    // every group of the longest documents at once; where the whole pack's
+    // K/V fits, this is plain longest-first (the best load balance).  The
+    // stable sort keeps the items of one (query tile, kv group) adjacent.
+    const int c = kv_groups_per_chunk(cu[n_docs], ks.D, Hkv);
+    std::stable_sort(items.begin(), items.end(), [G, c](const thd_work_item& a, const thd_work_item& b) {
+        const int ca = a.head0 / G / c, cb = b.head0 / G / c;
+        if (ca != cb) return ca < cb;
         return a.n_kv > b.n_kv;
     });
     return items;

@@ -28,6 +28,11 @@ struct KernelShape {
 // Returns false if the head dim is unsupported.
 bool choose_kernel_shape(int D, int group, KernelShape* out);
 
+// Number of consecutive kv groups whose items the plan mixes (longest first
+// among them): as many as keep their K/V (T x D bf16 each for K and V) within
+// 48 MB, at least one.
+int kv_groups_per_chunk(int64_t T, int D, int Hkv);
+
 // Host argument checks shared by every entry point (no CUDA calls).
 int validate_args(const int32_t* cu_seqlens, int n_docs, int Hq, int Hkv, int D, int window);
 

@@ -16,7 +16,7 @@
 #include "../../include/thd_attn.h"
 #include "scheduler.h"
 #include "thd_attn_kernel.cuh"
-#include "thd_attn_pair_kernel.cuh"
+#include "thd_attn_split_kernel.cuh"
 
 namespace {
 
@@ -29,7 +29,7 @@ using Cfg64x1 = thd::FwdConfig<64, 1, 2, 128, 8>;
 using Cfg128x2 = thd::FwdConfig<128, 2, 1, 128, 5>;
 using Cfg128x1 = thd::FwdConfig<128, 1, 2, 128, 6>;
 using Cfg256x1 = thd::FwdConfig<256, 1, 2, 64, 5>;
-using PairCfg256 = thd::PairConfig<256, 1, 128, 4>;  // 2 heads per item over a CTA pair
+using SplitCfg256 = thd::SplitConfig<256, 2, 4>;  // 2 heads per item over a CTA pair
 
 constexpr int kNumVariants = 6;
 
@@ -176,9 +176,8 @@ template <class C>
 int launch_pair(DeviceState* ds, int vidx, const PlanEntry& plan, const CUtensorMap& mq,
                 const CUtensorMap& mk, const CUtensorMap& mv, const thd::FwdParams& prm,
                 cudaStream_t stream) {
-    auto kern = thd::thd_attn_fwd_pair_kernel<C>;
+    auto kern = thd::thd_attn_fwd_split_kernel<C>;
     if (!ds->attr_set[vidx]) {
-        if (!thd::pair_launch_registers_ok<C>()) return THD_ERR_UNSUPPORTED;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::SMEM_ALLOC) != cudaSuccess)
             return THD_ERR_CUDA;
@@ -275,7 +274,7 @@ int thd_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_
         case 2: return launch<Cfg128x2>(ds, 2, *plan, mq, mk, mv, prm, stream);
         case 3: return launch<Cfg128x1>(ds, 3, *plan, mq, mk, mv, prm, stream);
         case 4: return launch<Cfg256x1>(ds, 4, *plan, mq, mk, mv, prm, stream);
-        default: return launch_pair<PairCfg256>(ds, 5, *plan, mq, mk, mv, prm, stream);
+        default: return launch_pair<SplitCfg256>(ds, 5, *plan, mq, mk, mv, prm, stream);
     }
 }
 

@@ -33,7 +33,7 @@
 #include "../../include/thd_attn.h"
 #include "scheduler.h"
 #include "thd_attn_kernel.cuh"
-#include "thd_attn_pair_kernel.cuh"
+#include "thd_attn_split_kernel.cuh"
 
 namespace {
 
@@ -65,7 +65,7 @@ using NCfg64x1 = thd::FwdConfig<64, 1, 2, 128, 8>;
 using NCfg128x2 = thd::FwdConfig<128, 2, 1, 128, 5>;
 using NCfg128x1 = thd::FwdConfig<128, 1, 2, 128, 6>;
 using NCfg256x1 = thd::FwdConfig<256, 1, 2, 64, 5>;
-using NPairCfg256 = thd::PairConfig<256, 1, 128, 4>;  // 2 heads per item over a CTA pair
+using NSplitCfg256 = thd::SplitConfig<256, 2, 4>;  // 2 heads per item over a CTA pair
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -104,7 +104,7 @@ int64_t count_items(const int32_t* cu, int n_docs, int Hq, const thd::KernelShap
 }
 
 // Writes the schedule into g_host_items (same items and order as the cached
-// path's plan: kv group, then longest first; the sort key below is unique
+// path's plan: chunk of kv groups, then longest first; the sort key below is unique
 // and reproduces the generation order among items of equal length).
 void write_plan(const int32_t* cu, int n_docs, int Hq, int Hkv, int window,
                 const thd::KernelShape& ks, int64_t n) {
@@ -124,8 +124,9 @@ void write_plan(const int32_t* cu, int n_docs, int Hq, int Hkv, int window,
                                                       q1 - n_kv * BN, n_kv, ks.nq, BN};
         }
     }
-    std::sort(g_host_items, g_host_items + n, [G](const thd_work_item& a, const thd_work_item& b) {
-        if (a.head0 / G != b.head0 / G) return a.head0 / G < b.head0 / G;
+    const int c = thd::kv_groups_per_chunk(cu[n_docs], ks.D, Hkv);
+    std::sort(g_host_items, g_host_items + n, [G, c](const thd_work_item& a, const thd_work_item& b) {
+        if (a.head0 / G / c != b.head0 / G / c) return a.head0 / G / c < b.head0 / G / c;
         if (a.n_kv != b.n_kv) return a.n_kv > b.n_kv;
         if (a.doc_start != b.doc_start) return a.doc_start < b.doc_start;
         if (a.q1 != b.q1) return a.q1 > b.q1;
@@ -173,9 +174,8 @@ template <class C>
 int launch_pair(NoAllocDevice* st, int vidx, int64_t n_items, const CUtensorMap& mq,
                 const CUtensorMap& mk, const CUtensorMap& mv, const thd::FwdParams& prm,
                 cudaStream_t stream) {
-    auto kern = thd::thd_attn_fwd_pair_kernel<C>;
+    auto kern = thd::thd_attn_fwd_split_kernel<C>;
     if (!st->attr_set[vidx]) {
-        if (!thd::pair_launch_registers_ok<C>()) return THD_ERR_UNSUPPORTED;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::SMEM_ALLOC) != cudaSuccess)
             return THD_ERR_CUDA;
@@ -267,7 +267,7 @@ extern "C" int thd_attn_fwd_noalloc(const void* q, const void* k, const void* v,
     prm.window = window;
     prm.scale_log2 = scale * 1.4426950408889634f;
 
-    if (ks.pair) return launch_pair<NPairCfg256>(st, 5, n_items, mq, mk, mv, prm, stream);
+    if (ks.pair) return launch_pair<NSplitCfg256>(st, 5, n_items, mq, mk, mv, prm, stream);
     if (D == 64) {
         return ks.nq == 2 ? launch<NCfg64x2>(st, 0, n_items, mq, mk, mv, prm, stream)
                           : launch<NCfg64x1>(st, 1, n_items, mq, mk, mv, prm, stream);

@@ -1,8 +1,9 @@
 """The host tile schedule covers every visible (query, key, head) triple
 exactly as the kernel needs: each (token, head) row is owned by exactly one
 work item, every visible key of the row lies in the item's key tiles, no key
-tile is fully masked, and items run one kv group after another, longest first
-within a group, with the heads of one (query tile, kv group) adjacent.  Checked by brute force against the window definition of
+tile is fully masked, and items run in chunks of kv groups whose K/V fits in
+L2, longest first within a chunk, with the heads of one (query tile, kv group)
+adjacent.  Checked by brute force against the window definition of
 FlintMagiPlan.attention ("flint.magi" page)."""
 import numpy as np
 import pytest
@@ -50,12 +51,26 @@ def check_plan(cu, Hq, Hkv, D, window):
             tile_hit[(lo - ks) // bn:(hi - ks) // bn + 1] = True
         assert tile_hit.all(), "a key tile with no visible pair was scheduled"
     assert (owner >= 0).all(), "some (token, head) row is not covered"
-    # kv groups in order, longest first within each group
-    grp = plan["head0"] // G
-    assert (np.diff(grp) >= 0).all(), "kv groups interleaved"
-    for g in np.unique(grp):
-        assert (np.diff(plan["n_kv"][grp == g]) <= 0).all(), "not longest first within a group"
+    # chunks of kv groups in order (as many groups per chunk as keep their
+    # K/V within 48 MB), longest first within each chunk
+    c = int(min(max((48 << 20) // max(T * D * 4, 1), 1), Hkv))
+    chunk = plan["head0"] // G // c
+    assert (np.diff(chunk) >= 0).all(), "kv group chunks interleaved"
+    for g in np.unique(chunk):
+        assert (np.diff(plan["n_kv"][chunk == g]) <= 0).all(), "not longest first within a chunk"
     return plan
+
+
+def test_group_chunks_follow_the_l2_budget():
+    # 64k tokens at D = 128: 32 MiB of K/V per kv head -> one group per chunk
+    cu = workloads.cu_seqlens_from_lengths([30000, 35536])
+    plan = swa.thd_attn_plan(cu, 16, 8, 128, 0)
+    assert (np.diff(plan["head0"] // 2) >= 0).all()
+    # 8k tokens: 4 MiB per kv head -> all 8 groups in one chunk (plain longest first)
+    cu = workloads.cu_seqlens_from_lengths([5000, 3192])
+    plan = swa.thd_attn_plan(cu, 16, 8, 128, 0)
+    assert (np.diff(plan["n_kv"]) <= 0).all()
+    assert len(set(plan["head0"][:8] // 2)) > 1
 
 
 @pytest.mark.parametrize("lens,Hq,Hkv,D,window", [
