@@ -9,6 +9,9 @@ Two independent formulations live here:
 * :func:`attention` / :func:`attention_rows` -- the plain fp64 loop over
   documents, heads and queries in ``thd_attn_oracle.c`` (see that file's
   header for the definition and the page passages it restates);
+* :func:`attention_bwd` / :func:`attention_bwd_q_rows` -- the fp64 gradient
+  of that forward (dq, dk, dv, dsink), the plain derivative written out in the
+  same C file;
 * :func:`dense_attention` -- a dense brute force for tiny packs: it builds the
   boolean ``[query_tokens, key_tokens]`` causal document mask the way
   ``SequenceLayout.allowed`` is described ("mistral_large4.attention" page),
@@ -62,6 +65,12 @@ def _bind(lib):
     lib.oracle_thd_attn_rows.argtypes = [vp, vp, vp, c_int, i32p, c_int, c_int, c_int, c_int,
                                          c_int, c_double, fp, i64p, ctypes.c_int64, dp, dp]
     lib.oracle_thd_attn_rows.restype = c_int
+    lib.oracle_thd_attn_bwd.argtypes = [vp, vp, vp, vp, c_int, i32p, c_int, c_int, c_int, c_int,
+                                        c_int, c_double, fp, dp, dp, dp, dp]
+    lib.oracle_thd_attn_bwd.restype = c_int
+    lib.oracle_thd_attn_bwd_q_rows.argtypes = [vp, vp, vp, vp, c_int, i32p, c_int, c_int, c_int,
+                                               c_int, c_int, c_double, fp, i64p, ctypes.c_int64, dp]
+    lib.oracle_thd_attn_bwd_q_rows.restype = c_int
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = c_int
     return lib
@@ -154,6 +163,60 @@ def attention_rows(q, k, v, cu_seqlens, window: int, scale: float, rows, sinks=N
     if rc != 0:
         raise ValueError("oracle rejected its arguments")
     return out, lse
+
+
+def _dout(dout, dt):
+    da, ddt = _as_input(dout)
+    if ddt != dt:
+        raise ValueError("dout must share the dtype of q, k, v")
+    return da
+
+
+def attention_bwd(q, k, v, dout, cu_seqlens, window: int, scale: float, sinks=None, lib=None):
+    """Full fp64 backward (the derivative of :func:`attention`, see the C
+    source).  Returns (dq [T, Hq, D], dk [T, Hkv, D], dv [T, Hkv, D],
+    dsink [Hq] or None), all float64."""
+    lib = lib or load()
+    qa, ka, va, dt, cu, T, Hq, Hkv, D = _common(q, k, v, cu_seqlens)
+    da = _dout(dout, dt)
+    if da.shape != (T, Hq, D):
+        raise ValueError("dout shape mismatch")
+    s = _sinks(sinks)
+    dq = np.zeros((T, Hq, D))
+    dk = np.zeros((T, Hkv, D))
+    dv = np.zeros((T, Hkv, D))
+    dsink = np.zeros((Hq,)) if s is not None else None
+    dptr = lambda a: a.ctypes.data_as(ctypes.POINTER(ctypes.c_double)) if a is not None else None
+    rc = lib.oracle_thd_attn_bwd(
+        qa.ctypes.data, ka.ctypes.data, va.ctypes.data, da.ctypes.data, dt,
+        cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), len(cu) - 1, Hq, Hkv, D,
+        int(window), float(scale),
+        s.ctypes.data_as(ctypes.POINTER(ctypes.c_float)) if s is not None else None,
+        dptr(dq), dptr(dk), dptr(dv), dptr(dsink))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return dq, dk, dv, dsink
+
+
+def attention_bwd_q_rows(q, k, v, dout, cu_seqlens, window: int, scale: float, rows, sinks=None,
+                         lib=None):
+    """fp64 dq for selected (token, query_head) rows ``rows`` [n, 2]; returns [n, D]."""
+    lib = lib or load()
+    qa, ka, va, dt, cu, T, Hq, Hkv, D = _common(q, k, v, cu_seqlens)
+    da = _dout(dout, dt)
+    s = _sinks(sinks)
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 2))
+    out = np.zeros((r.shape[0], D))
+    rc = lib.oracle_thd_attn_bwd_q_rows(
+        qa.ctypes.data, ka.ctypes.data, va.ctypes.data, da.ctypes.data, dt,
+        cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), len(cu) - 1, Hq, Hkv, D,
+        int(window), float(scale),
+        s.ctypes.data_as(ctypes.POINTER(ctypes.c_float)) if s is not None else None,
+        r.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), r.shape[0],
+        out.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return out
 
 
 def num_threads(lib=None) -> int:

@@ -160,6 +160,185 @@ int oracle_thd_attn_rows(const void *q, const void *k, const void *v, int dtype,
     return 0;
 }
 
+/*
+ * ------------------------------------------------------------------------
+ * Backward.  The pages train through this attention (the Magi plans serve
+ * activation-checkpointed layers, "muse_spark.magi_cp" and "flint.magi"), so
+ * the adjacent step is its gradient.  It is the plain derivative of the
+ * forward above; with P_ij = exp(s_ij - lse_i) (the sink's share is
+ * P_sink,i = exp(sink_h - lse_i)) and dO = dL/d out:
+ *
+ *   D_i      = sum_c dO[i,h,c] * out[i,h,c]
+ *   dP_ij    = sum_c dO[i,h,c] * v[j,g,c]
+ *   dS_ij    = P_ij * (dP_ij - D_i)                (gradient of the score s_ij)
+ *   dq[i,h]  = scale * sum_{j in V(i)} dS_ij * k[j,g]
+ *   dk[j,g]  = scale * sum_{h in g} sum_{i : j in V(i)} dS_ij * q[i,h]
+ *   dv[j,g]  = sum_{h in g} sum_{i : j in V(i)} P_ij * dO[i,h]
+ *   dsink[h] = - sum_i P_sink,i * D_i              (the sink has no value row)
+ *
+ * The key heads collect the gradients of all Hq/Hkv query heads that read
+ * them (the transpose of repeat_kv).
+ * ------------------------------------------------------------------------
+ */
+
+/* Scores, lse and P for row (i, h); keys lo..i.  Returns the key count. */
+static int64_t row_probs(const void *q, const void *k, int dtype, int Hq, int Hkv, int D,
+                         double scale, const float *sinks, int64_t i, int h, int g,
+                         int64_t lo, double *p, double *lse_out, double *psink_out) {
+    const int64_t n = i - lo + 1;
+    double m = -INFINITY;
+    for (int64_t j = lo; j <= i; j++) {
+        double acc = 0.0;
+        for (int c = 0; c < D; c++)
+            acc += load_elem(q, (i * Hq + h) * (int64_t)D + c, dtype) *
+                   load_elem(k, (j * Hkv + g) * (int64_t)D + c, dtype);
+        p[j - lo] = scale * acc;
+        if (p[j - lo] > m) m = p[j - lo];
+    }
+    const double sink = sinks != NULL ? (double)sinks[h] : -INFINITY;
+    if (sink > m) m = sink;
+    double Z = sinks != NULL ? exp(sink - m) : 0.0;
+    for (int64_t j = 0; j < n; j++) Z += exp(p[j] - m);
+    const double lse = m + log(Z);
+    for (int64_t j = 0; j < n; j++) p[j] = exp(p[j] - lse);
+    *lse_out = lse;
+    *psink_out = sinks != NULL ? exp(sink - lse) : 0.0;
+    return n;
+}
+
+/* Lowest visible key of query i in a document starting at s. */
+static int64_t first_key(int64_t i, int64_t s, int window) {
+    const int64_t w_lo = i - window + 1;  /* j > i - W */
+    return (window > 0 && w_lo > s) ? w_lo : s;
+}
+
+/* All gradients of document [s, e) for kv head g; dsink_part[G] collects the
+ * sink gradients of the group's query heads. */
+static void bwd_doc_group(const void *q, const void *k, const void *v, const void *dout,
+                          int dtype, int Hq, int Hkv, int D, int window, double scale,
+                          const float *sinks, int64_t s, int64_t e, int g,
+                          double *dq, double *dk, double *dv, double *dsink_part) {
+    const int G = Hq / Hkv;
+    double *p = (double *)malloc((size_t)(e - s > 0 ? e - s : 1) * sizeof(double));
+    double *o = (double *)malloc((size_t)D * sizeof(double));
+    for (int hh = 0; hh < G; hh++) {
+        const int h = g * G + hh;
+        for (int64_t i = s; i < e; i++) {
+            const int64_t lo = first_key(i, s, window);
+            double lse, psink;
+            const int64_t n = row_probs(q, k, dtype, Hq, Hkv, D, scale, sinks, i, h, g, lo,
+                                        p, &lse, &psink);
+            for (int c = 0; c < D; c++) o[c] = 0.0;
+            for (int64_t j = lo; j <= i; j++)
+                for (int c = 0; c < D; c++)
+                    o[c] += p[j - lo] * load_elem(v, (j * Hkv + g) * (int64_t)D + c, dtype);
+            double Di = 0.0;
+            for (int c = 0; c < D; c++)
+                Di += load_elem(dout, (i * Hq + h) * (int64_t)D + c, dtype) * o[c];
+            dsink_part[hh] -= psink * Di;
+            for (int64_t j = lo; j <= i; j++) {
+                double dP = 0.0;
+                for (int c = 0; c < D; c++)
+                    dP += load_elem(dout, (i * Hq + h) * (int64_t)D + c, dtype) *
+                          load_elem(v, (j * Hkv + g) * (int64_t)D + c, dtype);
+                const double dS = p[j - lo] * (dP - Di);
+                for (int c = 0; c < D; c++) {
+                    dq[(i * Hq + h) * (int64_t)D + c] +=
+                        scale * dS * load_elem(k, (j * Hkv + g) * (int64_t)D + c, dtype);
+                    dk[(j * Hkv + g) * (int64_t)D + c] +=
+                        scale * dS * load_elem(q, (i * Hq + h) * (int64_t)D + c, dtype);
+                    dv[(j * Hkv + g) * (int64_t)D + c] +=
+                        p[j - lo] * load_elem(dout, (i * Hq + h) * (int64_t)D + c, dtype);
+                }
+            }
+            (void)n;
+        }
+    }
+    free(o);
+    free(p);
+}
+
+/*
+ * Full backward in fp64: dq[T, Hq, D], dk/dv[T, Hkv, D], dsink[Hq] (dsink may
+ * be NULL when sinks is NULL).  q/k/v/dout share one dtype (fp64 or bf16
+ * bits).  Parallel over (document, kv head) pairs, whose dk/dv/dq rows are
+ * disjoint.  Returns 0, or -1 on invalid arguments.
+ */
+int oracle_thd_attn_bwd(const void *q, const void *k, const void *v, const void *dout, int dtype,
+                        const int32_t *cu_seqlens, int n_docs, int Hq, int Hkv, int D,
+                        int window, double scale, const float *sinks,
+                        double *dq, double *dk, double *dv, double *dsink) {
+    if (check_args(cu_seqlens, n_docs, Hq, Hkv, D, window)) return -1;
+    const int64_t T = n_docs > 0 ? cu_seqlens[n_docs] : 0;
+    const int G = Hq / Hkv;
+    memset(dq, 0, (size_t)(T * Hq * D) * sizeof(double));
+    memset(dk, 0, (size_t)(T * Hkv * D) * sizeof(double));
+    memset(dv, 0, (size_t)(T * Hkv * D) * sizeof(double));
+    if (dsink) memset(dsink, 0, (size_t)Hq * sizeof(double));
+    const int64_t units = (int64_t)n_docs * Hkv;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t u = 0; u < units; u++) {
+        const int d = (int)(u / Hkv), g = (int)(u % Hkv);
+        double *part = (double *)calloc((size_t)G, sizeof(double));
+        bwd_doc_group(q, k, v, dout, dtype, Hq, Hkv, D, window, scale, sinks,
+                      cu_seqlens[d], cu_seqlens[d + 1], g, dq, dk, dv, part);
+        if (dsink) {
+            for (int hh = 0; hh < G; hh++) {
+#pragma omp atomic
+                dsink[g * G + hh] += part[hh];
+            }
+        }
+        free(part);
+    }
+    return 0;
+}
+
+/*
+ * dq for selected (token, query head) rows only (rows[2r], rows[2r+1]):
+ * each needs just its own row of P.  dq_rows[n_rows, D].
+ */
+int oracle_thd_attn_bwd_q_rows(const void *q, const void *k, const void *v, const void *dout,
+                               int dtype, const int32_t *cu_seqlens, int n_docs, int Hq, int Hkv,
+                               int D, int window, double scale, const float *sinks,
+                               const int64_t *rows, int64_t n_rows, double *dq_rows) {
+    if (check_args(cu_seqlens, n_docs, Hq, Hkv, D, window)) return -1;
+    const int64_t T = n_docs > 0 ? cu_seqlens[n_docs] : 0;
+    for (int64_t r = 0; r < n_rows; r++)
+        if (rows[2 * r] < 0 || rows[2 * r] >= T || rows[2 * r + 1] < 0 || rows[2 * r + 1] >= Hq)
+            return -1;
+    const int G = Hq / Hkv;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n_rows; r++) {
+        const int64_t i = rows[2 * r];
+        const int h = (int)rows[2 * r + 1], g = h / G;
+        const int64_t s = cu_seqlens[find_doc(cu_seqlens, n_docs, i)];
+        const int64_t lo = first_key(i, s, window);
+        double *p = (double *)malloc((size_t)(i - lo + 1) * sizeof(double));
+        double *o = (double *)calloc((size_t)D, sizeof(double));
+        double lse, psink;
+        row_probs(q, k, dtype, Hq, Hkv, D, scale, sinks, i, h, g, lo, p, &lse, &psink);
+        for (int64_t j = lo; j <= i; j++)
+            for (int c = 0; c < D; c++)
+                o[c] += p[j - lo] * load_elem(v, (j * Hkv + g) * (int64_t)D + c, dtype);
+        double Di = 0.0;
+        for (int c = 0; c < D; c++) Di += load_elem(dout, (i * Hq + h) * (int64_t)D + c, dtype) * o[c];
+        double *out = dq_rows + r * D;
+        for (int c = 0; c < D; c++) out[c] = 0.0;
+        for (int64_t j = lo; j <= i; j++) {
+            double dP = 0.0;
+            for (int c = 0; c < D; c++)
+                dP += load_elem(dout, (i * Hq + h) * (int64_t)D + c, dtype) *
+                      load_elem(v, (j * Hkv + g) * (int64_t)D + c, dtype);
+            const double dS = p[j - lo] * (dP - Di);
+            for (int c = 0; c < D; c++)
+                out[c] += scale * dS * load_elem(k, (j * Hkv + g) * (int64_t)D + c, dtype);
+        }
+        free(o);
+        free(p);
+    }
+    return 0;
+}
+
 /* Threads OpenMP would use for the calls above. */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

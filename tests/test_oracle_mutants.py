@@ -68,12 +68,111 @@ def test_unmutated_copy_passes(tmp_path):
     assert _pins_fail(lib) == []
 
 
+# The C source holds the forward first, then the backward after this marker;
+# a forward mutant changes the forward part only, a backward mutant the
+# backward part only.
+BWD_MARKER = " * Backward."
+
+
+def _mutate(old, new, backward):
+    src = open(oracle._SRC).read()
+    cut = src.index(BWD_MARKER)
+    head, tail = src[:cut], src[cut:]
+    part = tail if backward else head
+    assert part.count(old) == 1, f"mutation anchor {old[:40]!r} not unique"
+    return head + tail.replace(old, new) if backward else head.replace(old, new) + tail
+
+
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_mutant_is_caught(name, tmp_path):
     old, new = MUTANTS[name]
-    src = open(oracle._SRC).read()
-    assert src.count(old) == 1, f"mutation anchor for {name} not unique in oracle source"
     path = tmp_path / f"{name}.c"
-    path.write_text(src.replace(old, new))
+    path.write_text(_mutate(old, new, backward=False))
     lib = oracle.load(oracle.build(force=True, src=str(path), out=str(tmp_path / f"{name}.so")))
     assert _pins_fail(lib), f"mutant {name} survived every pin"
+
+
+# ----------------------------------------------------------------- backward --
+# Planted mistakes in the oracle's backward; caught by finite differences of
+# the (unmutated-forward) copy, by PyTorch SDPA autograd, or by the invariants.
+
+BWD_MUTANTS = {
+    "bwd_D_term_dropped": ("const double dS = p[j - lo] * (dP - Di);\n                for (int c = 0; c < D; c++) {",
+                           "const double dS = p[j - lo] * dP;\n                for (int c = 0; c < D; c++) {"),
+    "bwd_dsink_sign": ("dsink_part[hh] -= psink * Di;", "dsink_part[hh] += psink * Di;"),
+    "bwd_dk_uses_key": ("scale * dS * load_elem(q, (i * Hq + h) * (int64_t)D + c, dtype);",
+                        "scale * dS * load_elem(k, (i * Hkv + g) * (int64_t)D + c, dtype);"),
+    "bwd_dv_weighted_by_dS": ("p[j - lo] * load_elem(dout, (i * Hq + h) * (int64_t)D + c, dtype);",
+                              "dS * load_elem(dout, (i * Hq + h) * (int64_t)D + c, dtype);"),
+    "bwd_dq_scale_dropped": ("dq[(i * Hq + h) * (int64_t)D + c] +=\n                        scale * dS",
+                             "dq[(i * Hq + h) * (int64_t)D + c] +=\n                        dS"),
+    "bwd_dk_wrong_group": ("dk[(j * Hkv + g) * (int64_t)D + c] +=", "dk[(j * Hkv + h % Hkv) * (int64_t)D + c] +="),
+}
+
+
+def _bwd_pins_fail(lib) -> list[str]:
+    import torch
+    failures = []
+    # finite differences of the forward on a tiny pack with a sink and a window
+    p = workloads.random_pack(3, [5, 0, 7, 1], 4, 2, 4, 3, 0.5, True)
+    q, k, v = (p[n].double().numpy() for n in "qkv")
+    s = p["sinks"].numpy().astype(np.float32)
+    dout = np.random.default_rng(103).standard_normal(q.shape)
+    cu = p["cu_seqlens"]
+    dq, dk, dv, ds = oracle.attention_bwd(q, k, v, dout, cu, 3, 0.5, s, lib=lib)
+
+    def loss(q_, k_, v_, s_):
+        o, _ = oracle.attention(q_, k_, v_, cu, 3, 0.5, s_)  # the real (pinned) forward
+        return float((o * dout).sum())
+
+    h = 1e-5
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for idx in list(np.ndindex(x.shape))[::3]:
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            a = {"q": q, "k": k, "v": v}
+            a[name] = xp
+            fp = loss(a["q"], a["k"], a["v"], s)
+            a[name] = xm
+            fm = loss(a["q"], a["k"], a["v"], s)
+            if abs((fp - fm) / (2 * h) - g[idx]) > 1e-6 * max(1.0, np.abs(g).max()):
+                failures.append(f"fd_{name}")
+                break
+    for hh in range(4):
+        sp, sm = s.copy(), s.copy()
+        sp[hh] += np.float32(1e-2)
+        sm[hh] -= np.float32(1e-2)
+        fd = (loss(q, k, v, sp) - loss(q, k, v, sm)) / (float(sp[hh]) - float(sm[hh]))
+        if abs(fd - ds[hh]) > 2e-4 * max(1.0, abs(ds[hh])):
+            failures.append("fd_sink")
+            break
+    # SDPA autograd, one document, no sink
+    p = workloads.random_pack(5, [23], 4, 2, 16, 0, 0.25, False)
+    q, k, v = (p[n].double().numpy() for n in "qkv")
+    dout = np.random.default_rng(105).standard_normal(q.shape)
+    dq, dk, dv, _ = oracle.attention_bwd(q, k, v, dout, p["cu_seqlens"], 0, 0.25, lib=lib)
+    qt, kt, vt = (torch.tensor(a).permute(1, 0, 2).requires_grad_() for a in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(
+        qt, kt.repeat_interleave(2, 0), vt.repeat_interleave(2, 0), is_causal=True, scale=0.25)
+    o.backward(torch.tensor(dout).permute(1, 0, 2))
+    for name, t, g in (("q", qt, dq), ("k", kt, dk), ("v", vt, dv)):
+        if not np.allclose(t.grad.permute(1, 0, 2).numpy(), g, atol=1e-10):
+            failures.append(f"sdpa_{name}")
+    return failures
+
+
+def test_unmutated_backward_copy_passes(tmp_path):
+    path = tmp_path / "copy_bwd.c"
+    path.write_text(open(oracle._SRC).read())
+    lib = oracle.load(oracle.build(force=True, src=str(path), out=str(tmp_path / "copy_bwd.so")))
+    assert _bwd_pins_fail(lib) == []
+
+
+@pytest.mark.parametrize("name", sorted(BWD_MUTANTS))
+def test_backward_mutant_is_caught(name, tmp_path):
+    old, new = BWD_MUTANTS[name]
+    path = tmp_path / f"{name}.c"
+    path.write_text(_mutate(old, new, backward=True))
+    lib = oracle.load(oracle.build(force=True, src=str(path), out=str(tmp_path / f"{name}.so")))
+    assert _bwd_pins_fail(lib), f"mutant {name} survived every pin"
