@@ -81,13 +81,18 @@ def measured_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+# Sources that decide the forward kernels' DRAM traffic: the kernels and the
+# schedule (item order).  Host-only entry-point code is not part of it.
+TRAFFIC_SOURCES = ("sm100_ptx.cuh", "thd_attn_kernel.cuh", "thd_attn_split_kernel.cuh",
+                   "scheduler.cpp", "scheduler.h")
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sliding_window_gqa_cu_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".cpp", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in TRAFFIC_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
