@@ -42,6 +42,7 @@
 #ifndef THD_ATTN_H
 #define THD_ATTN_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -120,8 +121,9 @@ typedef struct thd_work_item {
 
 /*
  * Host-only: build the tile schedule thd_attn_fwd uses for these arguments,
- * ordered by kv head (so the CTAs in flight share one head's K/V in L2) and,
- * within a kv head, longest first (non-increasing n_kv), the heads of one
+ * ordered by chunks of consecutive kv heads whose K/V (T x D bf16 each)
+ * fits in 48 MB (so the CTAs in flight share those heads' K/V in L2) and,
+ * within a chunk, longest first (non-increasing n_kv), the heads of one
  * (query tile, kv head) adjacent.
  * No CUDA call is made.  `items` may be NULL to query the count.  Writes
  * min(count, capacity) items and sets *n_items = count.  Returns THD_OK or
@@ -167,6 +169,65 @@ int thd_attn_fwd_noalloc(const void* q, const void* k, const void* v,
                          void* out, float* lse,
                          int* device_status_or_null,
                          void* stream);
+
+/*
+ * ------------------------------------------------------------------ backward
+ * The pages run this attention inside training: the Magi plans are selected
+ * "before entering checkpointed layers" and retained by the forward's
+ * activation-checkpointing graph ("muse_spark.magi_cp" page,
+ * _MuseMagiBatchPlans.select), so the gradient is taken through it.  The
+ * backward is the exact derivative of thd_attn_fwd: with P_ij =
+ * exp(s_ij - lse_i) from the forward's saved log-sum-exp and dO = dL/d out,
+ *   D_i = sum_c dO_ic out_ic,  dS_ij = P_ij (dO_i . v_j - D_i),
+ *   dq_i = scale sum_j dS_ij k_j,
+ *   dk_j = scale sum over the query heads h of j's kv head and queries i of dS_ij q_i,
+ *   dv_j = sum over the same (h, i) of P_ij dO_i,
+ *   dsink_h = -sum_i exp(sink_h - lse_i) D_i.
+ */
+
+/*
+ * One unit of work of the backward's key-side kernel (dk, dv): the 128 keys
+ * [k0, k0 + 128) of the document [doc_start, doc_end) for kv head g, against
+ * n_q query tiles [k0 + 128 t, k0 + 128 t + 128) of every query head of the
+ * group.  Keys or queries at or past doc_end are masked.
+ */
+typedef struct thd_bwd_kv_item {
+    int32_t k0, doc_start, doc_end, g;
+    int32_t n_q, pad0, pad1, pad2;
+} thd_bwd_kv_item;
+
+/* Bytes of device workspace thd_attn_bwd needs for a pack of total_tokens
+ * tokens and Hq query heads (two fp32 values per (token, query head)). */
+size_t thd_attn_bwd_workspace_bytes(int64_t total_tokens, int Hq);
+
+/*
+ * Backward of thd_attn_fwd for head dim 64 or 128 (256: THD_ERR_UNSUPPORTED).
+ *   q, k, v, cu_seqlens, n_docs, Hq, Hkv, D, window, scale, sinks_or_null
+ *              exactly as passed to thd_attn_fwd
+ *   out        bf16 device [T, Hq, D]: the forward's output
+ *   lse        fp32 device [T, Hq]: the forward's log-sum-exp (required)
+ *   dout       bf16 device [T, Hq, D]: gradient of the loss w.r.t. out
+ *   dq         bf16 device [T, Hq, D]    (written; caller-owned)
+ *   dk, dv     bf16 device [T, Hkv, D]   (written; caller-owned)
+ *   dsinks_or_null  fp32 device [Hq]: written with dL/dsink when given
+ *              (zeros when sinks_or_null is NULL)
+ *   workspace  device scratch of at least thd_attn_bwd_workspace_bytes(T, Hq)
+ *              bytes, 16-byte aligned, caller-owned; its contents on entry do
+ *              not matter and are garbage on return
+ *   stream     cudaStream_t to enqueue on
+ * Row-major contiguous tensors, 16-byte aligned bf16 pointers, 4-byte
+ * aligned fp32 pointers.  The result is deterministic (no atomics).  Argument
+ * errors return a negative code before anything is enqueued; kernel stalls
+ * are reported by thd_attn_get_error like the forward's.
+ */
+int thd_attn_bwd(const void* q, const void* k, const void* v,
+                 const void* out, const float* lse, const void* dout,
+                 const int32_t* cu_seqlens, int n_docs,
+                 int Hq, int Hkv, int D, int window, float scale,
+                 const float* sinks_or_null,
+                 void* dq, void* dk, void* dv, float* dsinks_or_null,
+                 void* workspace, size_t workspace_bytes,
+                 void* stream);
 
 /* ABI version of this header: (major << 16) | minor. */
 int thd_attn_abi_version(void);

@@ -74,6 +74,11 @@ def load_library():
     lib.thd_attn_fwd_noalloc.argtypes = [vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int,
                                          ctypes.c_float, vp, vp, vp, vp, vp]
     lib.thd_attn_fwd_noalloc.restype = c_int
+    lib.thd_attn_bwd_workspace_bytes.argtypes = [ctypes.c_int64, c_int]
+    lib.thd_attn_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.thd_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int,
+                                 ctypes.c_float, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.thd_attn_bwd.restype = c_int
     lib.thd_attn_abi_version.argtypes = []
     lib.thd_attn_abi_version.restype = c_int
     _lib = lib
@@ -165,6 +170,69 @@ def thd_attn_fwd(q, k, v, cu_seqlens, window: int = 0, scale: Optional[float] = 
     if rc != 0:
         raise ThdAttnError(rc, "thd_attn_fwd")
     return out, lse
+
+
+def thd_attn_bwd(q, k, v, out, lse, dout, cu_seqlens, window: int = 0,
+                 scale: Optional[float] = None, sinks=None, dq=None, dk=None, dv=None,
+                 workspace=None, stream=None):
+    """Backward of :func:`thd_attn_fwd` (head dim 64 or 128).
+
+    q, k, v, cu_seqlens, window, scale, sinks: as passed to the forward;
+    out, lse: the forward's results; dout: bf16 CUDA [T, Hq, D] gradient of the
+    loss w.r.t. out.  Returns ``(dq, dk, dv, dsinks)`` (``dsinks`` is None
+    without sinks).  ``workspace`` (optional) is a CUDA byte tensor of at least
+    ``thd_attn_bwd_workspace_bytes(T, Hq)`` bytes.
+    """
+    import torch
+
+    lib = load_library()
+    T, Hq, D = q.shape
+    Hkv = k.shape[1]
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    if out.shape != q.shape or dout.shape != q.shape:
+        raise ValueError("out and dout must be [tokens, heads, head_dim] like q")
+    if k.shape != (T, Hkv, D) or v.shape != (T, Hkv, D):
+        raise ValueError("k and v must be [tokens, kv_heads, head_dim] like q")
+    if lse is None or lse.dtype != torch.float32 or not lse.is_contiguous() or lse.shape != (T, Hq):
+        raise ValueError("lse must be the forward's contiguous fp32 [tokens, heads] log-sum-exp")
+    cu = _cu_array(cu_seqlens)
+    if int(cu[-1]) != T:
+        raise ValueError(f"cu_seqlens[-1]={int(cu[-1])} does not match {T} tokens")
+    if scale is None:
+        scale = D ** -0.5
+    dsinks = None
+    if sinks is not None:
+        if sinks.dtype != torch.float32 or not sinks.is_cuda or sinks.numel() != Hq:
+            raise ValueError("sinks must be an fp32 CUDA tensor of Hq values")
+        sinks = sinks.contiguous()
+        dsinks = torch.empty((Hq,), dtype=torch.float32, device=q.device)
+    dq = dq if dq is not None else torch.empty_like(q)
+    dk = dk if dk is not None else torch.empty_like(k)
+    dv = dv if dv is not None else torch.empty_like(v)
+    need = int(lib.thd_attn_bwd_workspace_bytes(T, Hq))
+    if workspace is None:
+        workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        rc = lib.thd_attn_bwd(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+            dout.data_ptr(), cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), cu.size - 1,
+            Hq, Hkv, D, int(window), float(scale),
+            sinks.data_ptr() if sinks is not None else None,
+            dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+            dsinks.data_ptr() if dsinks is not None else None,
+            workspace.data_ptr(), workspace.numel(), ctypes.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise ThdAttnError(rc, "thd_attn_bwd")
+    return dq, dk, dv, dsinks
+
+
+def thd_attn_bwd_workspace_bytes(T: int, Hq: int) -> int:
+    """Workspace bytes :func:`thd_attn_bwd` needs for T tokens and Hq query heads."""
+    return int(load_library().thd_attn_bwd_workspace_bytes(int(T), int(Hq)))
 
 
 def thd_attn_get_error(stream=None) -> int:

@@ -92,4 +92,31 @@ std::vector<thd_work_item> build_plan(const int32_t* cu, int n_docs, int Hq, int
     return items;
 }
 
+std::vector<thd_bwd_kv_item> build_bwd_kv_plan(const int32_t* cu, int n_docs, int Hq, int Hkv,
+                                               int D, int window) {
+    constexpr int BT = 128;
+    std::vector<thd_bwd_kv_item> items;
+    for (int d = 0; d < n_docs; ++d) {
+        const int s = cu[d], e = cu[d + 1];
+        for (int k0 = s; k0 < e; k0 += BT) {
+            // Queries that see a key of [k0, k0 + 128): [k0, q_end), q_end =
+            // the document end, or one past k0 + 127 + (W - 1) with a window.
+            int64_t q_end = e;
+            if (window > 0 && static_cast<int64_t>(k0) + 127 + window < q_end)
+                q_end = static_cast<int64_t>(k0) + 127 + window;
+            const int n_q = static_cast<int>((q_end - k0 + BT - 1) / BT);
+            for (int g = 0; g < Hkv; ++g)
+                items.push_back(thd_bwd_kv_item{k0, s, e, g, n_q, 0, 0, 0});
+        }
+    }
+    const int c = kv_groups_per_chunk(cu[n_docs], D, Hkv);
+    std::stable_sort(items.begin(), items.end(),
+                     [c](const thd_bwd_kv_item& a, const thd_bwd_kv_item& b) {
+                         if (a.g / c != b.g / c) return a.g / c < b.g / c;
+                         return a.n_q > b.n_q;
+                     });
+    (void)Hq;
+    return items;
+}
+
 }  // namespace thd

@@ -41,4 +41,10 @@ int validate_args(const int32_t* cu_seqlens, int n_docs, int Hq, int Hkv, int D,
 std::vector<thd_work_item> build_plan(const int32_t* cu_seqlens, int n_docs, int Hq, int Hkv,
                                       int window, const KernelShape& ks);
 
+// Key-side work list of the backward (dk, dv): one item per (128-key tile of
+// a document, kv head), with the query tiles that see any of its keys; same
+// chunked kv-group order, longest first within a chunk.
+std::vector<thd_bwd_kv_item> build_bwd_kv_plan(const int32_t* cu_seqlens, int n_docs, int Hq,
+                                               int Hkv, int D, int window);
+
 }  // namespace thd

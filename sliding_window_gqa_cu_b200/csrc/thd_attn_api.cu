@@ -18,6 +18,7 @@
 #include "tma_map.h"
 #include "thd_attn_kernel.cuh"
 #include "thd_attn_split_kernel.cuh"
+#include "thd_attn_bwd_kernels.cuh"
 
 namespace {
 
@@ -50,10 +51,25 @@ struct PlanEntry {
     int64_t n_items = 0;
 };
 
+// Backward schedules: the dq kernel's items (one query head each) and the
+// dk/dv kernel's items.
+struct BwdPlanEntry {
+    std::vector<int32_t> cu;
+    int Hq, Hkv, D, window;
+    thd::WorkItem* d_q_items = nullptr;
+    int64_t n_q_items = 0;
+    thd::BwdKVItem* d_kv_items = nullptr;
+    int64_t n_kv_items = 0;
+};
+
+constexpr int kNumBwdVariants = 4;  // {dq, dkdv} x {D = 64, D = 128}
+
 struct DeviceState {
     int* d_status = nullptr;
     bool attr_set[kNumVariants] = {};
-    std::list<PlanEntry> plans;  // most recently used first
+    bool bwd_attr_set[kNumBwdVariants] = {};
+    std::list<PlanEntry> plans;         // most recently used first
+    std::list<BwdPlanEntry> bwd_plans;  // most recently used first
 };
 
 constexpr size_t kMaxPlans = 16;
@@ -160,11 +176,119 @@ int launch_pair(DeviceState* ds, int vidx, const PlanEntry& plan, const CUtensor
     return cudaGetLastError() == cudaSuccess ? THD_OK : THD_ERR_CUDA;
 }
 
+// Uploads `n` items to a new device buffer (synchronously on `stream`).
+template <class T>
+int upload(const std::vector<T>& v, T** out, cudaStream_t stream) {
+    *out = nullptr;
+    if (v.empty()) return THD_OK;
+    const size_t bytes = v.size() * sizeof(T);
+    if (cudaMalloc(out, bytes) != cudaSuccess) {
+        *out = nullptr;
+        return THD_ERR_NO_MEMORY;
+    }
+    if (cudaMemcpyAsync(*out, v.data(), bytes, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess) {
+        cudaFree(*out);
+        *out = nullptr;
+        return THD_ERR_CUDA;
+    }
+    return THD_OK;
+}
+
+// Finds or builds the backward schedules for these arguments.  Caller holds g_mu.
+int get_bwd_plan(DeviceState* ds, const int32_t* cu, int n_docs, int Hq, int Hkv, int D, int window,
+                 cudaStream_t stream, const BwdPlanEntry** out) {
+    for (auto it = ds->bwd_plans.begin(); it != ds->bwd_plans.end(); ++it) {
+        if (it->Hq == Hq && it->Hkv == Hkv && it->D == D && it->window == window &&
+            it->cu.size() == static_cast<size_t>(n_docs) + 1 &&
+            std::memcmp(it->cu.data(), cu, sizeof(int32_t) * (n_docs + 1)) == 0) {
+            ds->bwd_plans.splice(ds->bwd_plans.begin(), ds->bwd_plans, it);
+            *out = &ds->bwd_plans.front();
+            return THD_OK;
+        }
+    }
+    // dq items: the forward's query tiles and key ranges, one query head each.
+    const KernelShape qs{D, 1, 1, 128, 4, false};
+    std::vector<thd_work_item> qi = thd::build_plan(cu, n_docs, Hq, Hkv, window, qs);
+    std::vector<thd_bwd_kv_item> ki = thd::build_bwd_kv_plan(cu, n_docs, Hq, Hkv, D, window);
+    std::vector<thd::WorkItem> qv(qi.size());
+    std::memcpy(qv.data(), qi.data(), qi.size() * sizeof(thd::WorkItem));
+    std::vector<thd::BwdKVItem> kv(ki.size());
+    std::memcpy(kv.data(), ki.data(), ki.size() * sizeof(thd::BwdKVItem));
+    BwdPlanEntry e;
+    e.cu.assign(cu, cu + n_docs + 1);
+    e.Hq = Hq;
+    e.Hkv = Hkv;
+    e.D = D;
+    e.window = window;
+    int rc = upload(qv, &e.d_q_items, stream);
+    if (rc != THD_OK) return rc;
+    rc = upload(kv, &e.d_kv_items, stream);
+    if (rc != THD_OK) {
+        if (e.d_q_items) cudaFree(e.d_q_items);
+        return rc;
+    }
+    e.n_q_items = static_cast<int64_t>(qv.size());
+    e.n_kv_items = static_cast<int64_t>(kv.size());
+    if (ds->bwd_plans.size() >= kMaxPlans) {
+        auto& old = ds->bwd_plans.back();
+        if (old.d_q_items) cudaFree(old.d_q_items);
+        if (old.d_kv_items) cudaFree(old.d_kv_items);
+        ds->bwd_plans.pop_back();
+    }
+    ds->bwd_plans.push_front(std::move(e));
+    *out = &ds->bwd_plans.front();
+    return THD_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+template <int D>
+int launch_bwd(DeviceState* ds, const BwdPlanEntry& plan, const CUtensorMap& mq,
+               const CUtensorMap& mdo, const CUtensorMap& mk, const CUtensorMap& mv,
+               const thd::BwdParams& prm, const void* out, const void* dout, const float* sinks,
+               float* dsinks, float* delta, float* sink_part, cudaStream_t stream) {
+    using Cq = thd::BwdConfig<D, D == 64 ? 8 : 4>;  // one CTA per SM (all 512 TMEM columns)
+    using Ckv = thd::BwdConfig<D, D == 64 ? 4 : 2>;
+    auto kq = thd::thd_attn_bwd_dq_kernel<Cq>;
+    auto kkv = thd::thd_attn_bwd_dkdv_kernel<Ckv>;
+    const int vq = D == 64 ? 0 : 2, vkv = vq + 1;
+    if (!ds->bwd_attr_set[vq]) {
+        if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 thd::DqLayout<Cq>::SMEM_ALLOC) != cudaSuccess)
+            return THD_ERR_CUDA;
+        ds->bwd_attr_set[vq] = true;
+    }
+    if (!ds->bwd_attr_set[vkv]) {
+        if (cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 thd::DkvLayout<Ckv>::SMEM_ALLOC) != cudaSuccess)
+            return THD_ERR_CUDA;
+        ds->bwd_attr_set[vkv] = true;
+    }
+    const int64_t rows = prm.T * prm.Hq;
+    thd::thd_attn_bwd_preprocess_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), prm.lse,
+        sinks, delta, sink_part, rows, prm.Hq);
+    if (dsinks != nullptr) {
+        if (sinks != nullptr)
+            thd::thd_attn_bwd_dsink_kernel<<<prm.Hq, 256, 0, stream>>>(sink_part, prm.T, prm.Hq, dsinks);
+        else if (cudaMemsetAsync(dsinks, 0, sizeof(float) * prm.Hq, stream) != cudaSuccess)
+            return THD_ERR_CUDA;
+    }
+    if (plan.n_q_items > 0)
+        kq<<<static_cast<unsigned>(plan.n_q_items), Cq::NUM_THREADS, thd::DqLayout<Cq>::SMEM_ALLOC,
+             stream>>>(mq, mdo, mk, mv, prm);
+    if (plan.n_kv_items > 0)
+        kkv<<<static_cast<unsigned>(plan.n_kv_items), Ckv::NUM_THREADS,
+              thd::DkvLayout<Ckv>::SMEM_ALLOC, stream>>>(mq, mdo, mk, mv, prm);
+    return cudaGetLastError() == cudaSuccess ? THD_OK : THD_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
 
-int thd_attn_abi_version(void) { return (1 << 16) | 0; }
+int thd_attn_abi_version(void) { return (1 << 16) | 1; }
 
 const char* thd_attn_status_string(int status) {
     switch (status) {
@@ -248,6 +372,76 @@ int thd_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_
         case 4: return launch<Cfg256x1>(ds, 4, *plan, mq, mk, mv, prm, stream);
         default: return launch_pair<SplitCfg256>(ds, 5, *plan, mq, mk, mv, prm, stream);
     }
+}
+
+size_t thd_attn_bwd_workspace_bytes(int64_t total_tokens, int Hq) {
+    if (total_tokens <= 0 || Hq <= 0) return 0;
+    return 2 * align256(static_cast<size_t>(total_tokens) * static_cast<size_t>(Hq) * sizeof(float));
+}
+
+int thd_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                 const void* dout, const int32_t* cu_seqlens, int n_docs, int Hq, int Hkv, int D,
+                 int window, float scale, const float* sinks_or_null, void* dq, void* dk, void* dv,
+                 float* dsinks_or_null, void* workspace, size_t workspace_bytes, void* stream_ptr) {
+    int rc = thd::validate_args(cu_seqlens, n_docs, Hq, Hkv, D, window);
+    if (rc != THD_OK) return rc;
+    if (D != 64 && D != 128) return THD_ERR_UNSUPPORTED;
+    if (!(std::isfinite(scale) && scale > 0.0f)) return THD_ERR_INVALID_ARG;
+    const int64_t T = cu_seqlens[n_docs];
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+    if ((dsinks_or_null && (reinterpret_cast<uintptr_t>(dsinks_or_null) & 3u)) ||
+        (sinks_or_null && (reinterpret_cast<uintptr_t>(sinks_or_null) & 3u)))
+        return THD_ERR_INVALID_ARG;
+    if (T == 0) {
+        if (dsinks_or_null &&
+            cudaMemsetAsync(dsinks_or_null, 0, sizeof(float) * Hq, stream) != cudaSuccess)
+            return THD_ERR_CUDA;
+        return THD_OK;
+    }
+    if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv || !workspace)
+        return THD_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace) ||
+        (reinterpret_cast<uintptr_t>(lse) & 3u))
+        return THD_ERR_INVALID_ARG;
+    if (workspace_bytes < thd_attn_bwd_workspace_bytes(T, Hq)) return THD_ERR_INVALID_ARG;
+
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState* ds = nullptr;
+    rc = device_state(&ds, nullptr);
+    if (rc != THD_OK) return rc;
+    const BwdPlanEntry* plan = nullptr;
+    rc = get_bwd_plan(ds, cu_seqlens, n_docs, Hq, Hkv, D, window, stream, &plan);
+    if (rc != THD_OK) return rc;
+
+    CUtensorMap mq, mdo, mk, mv;
+    if (!make_map(&mq, q, T, Hq, D, 128) || !make_map(&mdo, dout, T, Hq, D, 128) ||
+        !make_map(&mk, k, T, Hkv, D, 128) || !make_map(&mv, v, T, Hkv, D, 128))
+        return THD_ERR_CUDA;
+    float* delta = static_cast<float*>(workspace);
+    float* sink_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                                align256(static_cast<size_t>(T) * Hq * sizeof(float)));
+    thd::BwdParams prm;
+    prm.q_items = plan->d_q_items;
+    prm.kv_items = plan->d_kv_items;
+    prm.lse = lse;
+    prm.delta = delta;
+    prm.dq = static_cast<__nv_bfloat16*>(dq);
+    prm.dk = static_cast<__nv_bfloat16*>(dk);
+    prm.dv = static_cast<__nv_bfloat16*>(dv);
+    prm.status = ds->d_status;
+    prm.T = T;
+    prm.Hq = Hq;
+    prm.Hkv = Hkv;
+    prm.G = Hq / Hkv;
+    prm.window = window;
+    prm.scale = scale;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    if (D == 64)
+        return launch_bwd<64>(ds, *plan, mq, mdo, mk, mv, prm, out, dout, sinks_or_null,
+                              dsinks_or_null, delta, sink_part, stream);
+    return launch_bwd<128>(ds, *plan, mq, mdo, mk, mv, prm, out, dout, sinks_or_null,
+                           dsinks_or_null, delta, sink_part, stream);
 }
 
 int thd_attn_get_error(void* stream_ptr) {

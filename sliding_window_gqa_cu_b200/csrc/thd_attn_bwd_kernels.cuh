@@ -1,0 +1,679 @@
+// Packed-THD sliding-window GQA attention BACKWARD for B200 (sm_100a).
+//
+// The gradient of the forward in thd_attn_kernel.cuh (same document, window
+// and sink readings of the API pages).  With P_ij = exp(s_ij - lse_i), the
+// forward's saved log-sum-exp, and dO the gradient of the output:
+//   D_i   = sum_c dO_ic O_ic                        (preprocess kernel)
+//   dP_ij = dO_i . v_j,  dS_ij = P_ij (dP_ij - D_i)
+//   dq_i  = scale * sum_j dS_ij k_j                  (dq kernel)
+//   dk_j  = scale * sum_{h in group} sum_i dS_ij q_i (dkdv kernel)
+//   dv_j  = sum_{h in group} sum_i P_ij dO_i         (dkdv kernel)
+//   dsink_h = -sum_i exp(sink_h - lse_i) D_i         (preprocess + reduce)
+//
+// Both main kernels recompute S and dP on the tensor core instead of sharing
+// them through memory, so nothing is accumulated with atomics and the result
+// is bitwise reproducible:
+//   * dq kernel: one CTA per (128-row query tile, query head), looping over
+//     the key tiles the tile sees: S = Q K^T, dP = dO V^T (both from shared
+//     memory), dS written as bf16 over S in TMEM, dq += dS K (dS from TMEM,
+//     K from shared memory as an MN-major operand).
+//   * dkdv kernel: one CTA per (128-key tile, kv head), looping over the
+//     query heads of the group and the query tiles that see the keys:
+//     S^T = K Q^T and dP^T = V dO^T (TMEM lane = key), P^T and dS^T written as
+//     bf16 over them, dv += P^T dO and dk += dS^T Q (TMEM operands, dO and Q
+//     as MN-major operands); dk and dv stay in TMEM for the whole group.
+//
+// Warps (both kernels): 0-3 elementwise (thread t owns TMEM lane t), 4 TMA
+// producer, 5 MMA issuer, 6-7 idle.  Every wait is bounded and reports a
+// timeout in the device status word.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+#include "thd_attn_kernel.cuh"
+
+namespace thd {
+
+struct BwdKVItem {  // identical layout to thd_bwd_kv_item in thd_attn.h
+    int32_t k0, doc_start, doc_end, g;
+    int32_t n_q, pad0, pad1, pad2;
+};
+
+struct BwdParams {
+    const WorkItem* q_items;    // dq kernel: one query head per item
+    const BwdKVItem* kv_items;  // dkdv kernel
+    const float* lse;           // [T, Hq] natural log (forward output)
+    const float* delta;         // [T, Hq] rowsum(dO * O)
+    __nv_bfloat16* dq;          // [T, Hq, D]
+    __nv_bfloat16* dk;          // [T, Hkv, D]
+    __nv_bfloat16* dv;          // [T, Hkv, D]
+    int* status;
+    int64_t T;
+    int Hq, Hkv, G, window;
+    float scale;
+    float scale_log2;  // scale * log2(e)
+};
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// -------------------------------------------------------------- preprocess --
+// One warp per (token, head) row: delta = sum_c dO * O in fp32; with sinks
+// also the row's share of the sink gradient, -exp(sink_h - lse) * delta.
+template <int D>
+__global__ void __launch_bounds__(256) thd_attn_bwd_preprocess_kernel(
+    const __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ dout,
+    const float* __restrict__ lse, const float* __restrict__ sinks, float* __restrict__ delta,
+    float* __restrict__ sink_part, int64_t rows, int Hq) {
+    constexpr int PER_LANE = D / 32;  // 2, 4 or 8 bf16 per lane
+    const int lane = threadIdx.x & 31;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (row >= rows) return;
+    const __nv_bfloat16* o = out + row * D + lane * PER_LANE;
+    const __nv_bfloat16* g = dout + row * D + lane * PER_LANE;
+    float acc = 0.0f;
+    if constexpr (PER_LANE == 8) {
+        const uint4 a = *reinterpret_cast<const uint4*>(o);
+        const uint4 b = *reinterpret_cast<const uint4*>(g);
+        const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&av[u]));
+            const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bv[u]));
+            acc = fmaf(x.x, y.x, fmaf(x.y, y.y, acc));
+        }
+    } else if constexpr (PER_LANE == 4) {
+        const uint2 a = *reinterpret_cast<const uint2*>(o);
+        const uint2 b = *reinterpret_cast<const uint2*>(g);
+        const uint32_t av[2] = {a.x, a.y}, bv[2] = {b.x, b.y};
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&av[u]));
+            const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bv[u]));
+            acc = fmaf(x.x, y.x, fmaf(x.y, y.y, acc));
+        }
+    } else {
+        const uint32_t a = *reinterpret_cast<const uint32_t*>(o);
+        const uint32_t b = *reinterpret_cast<const uint32_t*>(g);
+        const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a));
+        const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&b));
+        acc = fmaf(x.x, y.x, x.y * y.y);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) {
+        delta[row] = acc;
+        if (sinks != nullptr) {
+            const int h = static_cast<int>(row % Hq);
+            sink_part[row] = -ex2_approx((sinks[h] - lse[row]) * kLog2e) * acc;
+        }
+    }
+}
+
+// dsink[h] = sum over tokens of sink_part[t, h], one block per head, in a
+// fixed order (strided per-thread sums, then a tree): deterministic.
+__global__ void __launch_bounds__(256) thd_attn_bwd_dsink_kernel(const float* __restrict__ sink_part,
+                                                                 int64_t T, int Hq,
+                                                                 float* __restrict__ dsink) {
+    __shared__ float red[256];
+    const int h = blockIdx.x;
+    float acc = 0.0f;
+    for (int64_t t = threadIdx.x; t < T; t += blockDim.x) acc += sink_part[t * Hq + h];
+    red[threadIdx.x] = acc;
+    __syncthreads();
+    for (int s = blockDim.x / 2; s > 0; s >>= 1) {
+        if (static_cast<int>(threadIdx.x) < s) red[threadIdx.x] += red[threadIdx.x + s];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) dsink[h] = red[0];
+}
+
+// ------------------------------------------------------------ shared shape --
+
+template <int D_, int NSLOT_>
+struct BwdConfig {
+    static constexpr int D = D_;
+    static constexpr int NSLOT = NSLOT_;  // dq: K/V ring slots; dkdv: Q/dO pairs
+    static constexpr int BM = 128;        // TMEM lanes (queries for dq, keys for dkdv)
+    static constexpr int BN = 128;        // columns of S per tile
+    static constexpr int KCH = D / 64;
+    static constexpr int BOX_BYTES = 128 * 128;   // one 64-column chunk of a 128-row tile
+    static constexpr int TILE_BYTES = 128 * D * 2;
+
+    static constexpr int TM_S = 0;        // S (dq) or S^T (dkdv), then P / dS bf16
+    static constexpr int TM_DP = 128;     // dP or dP^T, then dS^T (dkdv)
+    static constexpr int TM_ACC0 = 256;   // dq (dq kernel) or dv (dkdv kernel)
+    static constexpr int TM_ACC1 = 256 + D;  // dk (dkdv kernel)
+    static constexpr int TMEM_COLS = 512;
+
+    static constexpr int PRODUCER_WARP = 4;
+    static constexpr int MMA_WARP = 5;
+    static constexpr int NUM_THREADS = 256;
+
+    static_assert(D == 64 || D == 128, "backward kernels: head dim 64 or 128");
+    static_assert(TM_ACC1 + D <= 512, "TMEM budget exceeded");
+    static_assert(NSLOT >= 2, "ring needs two slots");
+};
+
+// ------------------------------------------------------------------ dq ------
+template <class C>
+struct DqLayout {
+    static constexpr int B_IN_FULL = 0;                       // Q and dO landed
+    static constexpr int B_SLOT_FULL = 1;
+    static constexpr int B_SLOT_EMPTY = B_SLOT_FULL + C::NSLOT;
+    static constexpr int B_S_FULL = B_SLOT_EMPTY + C::NSLOT;  // S and dP done
+    static constexpr int B_DS_FULL = B_S_FULL + 1;            // dS in TMEM (4 warps)
+    static constexpr int B_ACC_FULL = B_DS_FULL + 1;          // dq accumulated
+    static constexpr int B_DRAIN = B_ACC_FULL + 1;
+    static constexpr int NUM_BARS = B_DRAIN + 1;
+    static constexpr int SMEM_Q = 0;
+    static constexpr int SMEM_DO = SMEM_Q + C::TILE_BYTES;
+    static constexpr int SMEM_SLOTS = SMEM_DO + C::TILE_BYTES;
+    static constexpr int SMEM_BAR = SMEM_SLOTS + C::NSLOT * C::TILE_BYTES;
+    static constexpr int SMEM_TMEM_SLOT = SMEM_BAR + NUM_BARS * 8;
+    static constexpr int SMEM_ABORT = SMEM_TMEM_SLOT + 4;
+    static constexpr int SMEM_ALLOC = SMEM_ABORT + 4 + 1024;
+    static_assert(SMEM_ALLOC <= 232448, "shared memory budget exceeded");
+};
+
+template <class C>
+__global__ void __launch_bounds__(C::NUM_THREADS, 1)
+thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                       const __grid_constant__ CUtensorMap tmap_do,
+                       const __grid_constant__ CUtensorMap tmap_k,
+                       const __grid_constant__ CUtensorMap tmap_v, const BwdParams prm) {
+    using L = DqLayout<C>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = smem_addr(smem_raw);
+    uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
+    const uint32_t sbase = smem_addr(smem);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const WorkItem it = prm.q_items[blockIdx.x];
+    const int n = it.n_kv;
+    const int h = it.head0;
+
+    auto bar = [&](int idx) -> uint32_t { return sbase + L::SMEM_BAR + 8u * idx; };
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::SMEM_ABORT);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::SMEM_TMEM_SLOT);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(L::B_IN_FULL), 1);
+        for (int s = 0; s < C::NSLOT; ++s) {
+            mbar_init(bar(L::B_SLOT_FULL + s), 1);
+            mbar_init(bar(L::B_SLOT_EMPTY + s), 1);
+        }
+        mbar_init(bar(L::B_S_FULL), 1);
+        mbar_init(bar(L::B_DS_FULL), 4);
+        mbar_init(bar(L::B_ACC_FULL), 1);
+        mbar_init(bar(L::B_DRAIN), 1);
+        *abort_flag = *reinterpret_cast<volatile int*>(prm.status) != 0 ? 1 : 0;
+        fence_barrier_init();
+    }
+    if (warp == C::MMA_WARP) {
+        tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const bool skip = *abort_flag != 0;
+
+    if (warp == C::PRODUCER_WARP) {
+        if (lane == 0 && !skip) {
+            tma_prefetch_desc(&tmap_q);
+            tma_prefetch_desc(&tmap_do);
+            tma_prefetch_desc(&tmap_k);
+            tma_prefetch_desc(&tmap_v);
+            const int g = h / prm.G;
+            mbar_arrive_expect_tx(bar(L::B_IN_FULL), 2 * C::TILE_BYTES);
+            for (int c = 0; c < C::KCH; ++c) {
+                tma_load_3d(sbase + L::SMEM_Q + c * C::BOX_BYTES, &tmap_q, bar(L::B_IN_FULL), c * 64,
+                            h, it.q0);
+                tma_load_3d(sbase + L::SMEM_DO + c * C::BOX_BYTES, &tmap_do, bar(L::B_IN_FULL),
+                            c * 64, h, it.q0);
+            }
+            // Ring positions: 2j holds K(j), 2j+1 holds V(j).
+            int issued = 0;
+            bool ok = true;
+            for (int pos = 0; pos < 2 * n && ok; ++pos) {
+                const int slot = pos % C::NSLOT;
+                ok = mbar_wait(bar(L::B_SLOT_EMPTY + slot), ((pos / C::NSLOT) & 1) ^ 1, abort_flag,
+                               prm.status, kStatusTimeout);
+                if (!ok) break;
+                const CUtensorMap* map = (pos & 1) ? &tmap_v : &tmap_k;
+                const int kt = it.kv_start + (pos >> 1) * C::BN;
+                mbar_arrive_expect_tx(bar(L::B_SLOT_FULL + slot), C::TILE_BYTES);
+                for (int c = 0; c < C::KCH; ++c)
+                    tma_load_3d(sbase + L::SMEM_SLOTS + slot * C::TILE_BYTES + c * C::BOX_BYTES, map,
+                                bar(L::B_SLOT_FULL + slot), c * 64, g, kt);
+                issued = pos + 1;
+            }
+            if (!ok) {
+                drain_wait(bar(L::B_IN_FULL), 0);
+                for (int pos = issued - C::NSLOT > 0 ? issued - C::NSLOT : 0; pos < issued; ++pos)
+                    drain_wait(bar(L::B_SLOT_FULL + pos % C::NSLOT), (pos / C::NSLOT) & 1);
+            }
+        }
+        __syncwarp();
+    } else if (warp == C::MMA_WARP) {
+        if (lane == 0 && !skip) {
+            constexpr uint32_t idesc_s = idesc_bf16_f32(128, C::BN, false);
+            constexpr uint32_t idesc_acc = idesc_bf16_f32(128, C::D, true);
+            const uint64_t dq0 = smem_desc_sw128(sbase + L::SMEM_Q, 16, 1024);
+            const uint64_t ddo0 = smem_desc_sw128(sbase + L::SMEM_DO, 16, 1024);
+            const uint64_t dkv0 = smem_desc_sw128(sbase + L::SMEM_SLOTS, 16, 1024);
+            const uint64_t dkmn0 = smem_desc_sw128(sbase + L::SMEM_SLOTS, C::BOX_BYTES, 1024);
+            auto wait = [&](int idx, uint32_t parity) -> bool {
+                return mbar_wait(bar(idx), parity, abort_flag, prm.status, kStatusTimeout);
+            };
+            auto wait_slot = [&](int pos) -> bool {
+                return wait(L::B_SLOT_FULL + pos % C::NSLOT, (pos / C::NSLOT) & 1);
+            };
+            bool ok = wait(L::B_IN_FULL, 0);
+            for (int j = 0; ok && j < n; ++j) {
+                const int kslot = (2 * j) % C::NSLOT, vslot = (2 * j + 1) % C::NSLOT;
+                ok = wait_slot(2 * j) && wait_slot(2 * j + 1);
+                if (!ok) break;
+                tc_fence_after();
+                const uint64_t dk = dkv0 + ((kslot * C::TILE_BYTES) >> 4);
+                const uint64_t dv = dkv0 + ((vslot * C::TILE_BYTES) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < C::D / 16; ++kk) {  // S = Q K^T
+                    const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
+                    mma_bf16_ss(tmem_base + C::TM_S, dq0 + o, dk + o, idesc_s, kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < C::D / 16; ++kk) {  // dP = dO V^T
+                    const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
+                    mma_bf16_ss(tmem_base + C::TM_DP, ddo0 + o, dv + o, idesc_s, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bar(L::B_S_FULL));
+                mma_commit(bar(L::B_SLOT_EMPTY + vslot));  // V(j) consumed
+                ok = wait(L::B_DS_FULL, j & 1);
+                if (!ok) break;
+                tc_fence_after();
+                const uint64_t dkmn = dkmn0 + ((kslot * C::TILE_BYTES) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; ++kk)  // dq += dS K
+                    mma_bf16_ts(tmem_base + C::TM_ACC0, tmem_base + C::TM_S + kk * 8,
+                                dkmn + ((kk * 16 * 128) >> 4), idesc_acc, (j > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(bar(L::B_SLOT_EMPTY + kslot));  // K(j) consumed
+            }
+            if (ok) mma_commit(bar(L::B_ACC_FULL));
+            mma_commit(bar(L::B_DRAIN));
+            drain_wait(bar(L::B_DRAIN), 0);
+        }
+        __syncwarp();
+    } else if (warp < 4) {
+        const int row = warp * 32 + lane;
+        const int i = it.q0 + row;
+        const int s_doc = it.doc_start;
+        const int r_lo = it.q0 > s_doc ? it.q0 : s_doc;
+        const int r_hi = it.q1 - 1;
+        const bool row_valid = i >= r_lo && i <= r_hi;
+        const int W = prm.window;
+        // Visible keys of this row: [lo_i, i]; an empty range for rows
+        // outside the document.
+        int lo_i = (W > 0 && i - W + 1 > s_doc) ? i - W + 1 : s_doc;
+        if (!row_valid) lo_i = i + 1;
+        const float lse2 = row_valid ? prm.lse[static_cast<int64_t>(i) * prm.Hq + h] * kLog2e : 0.0f;
+        const float Di = row_valid ? prm.delta[static_cast<int64_t>(i) * prm.Hq + h] : 0.0f;
+        const float sl2 = prm.scale_log2;
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+
+        bool ok = !skip;
+        for (int j = 0; ok && j < n; ++j) {
+            ok = warp_wait(bar(L::B_S_FULL), j & 1, abort_flag, prm.status);
+            if (!ok) break;
+            tc_fence_after();
+            const int kt = it.kv_start + j * C::BN;
+            const bool full = row_valid && kt >= s_doc && kt + C::BN - 1 <= r_lo &&
+                              (W == 0 || kt >= r_hi - W + 1);
+#pragma unroll
+            for (int c = 0; c < C::BN / 32; ++c) {
+                uint32_t sr[32], dr[32];
+                tmem_ld32(lane_base + C::TM_S + c * 32, sr);
+                tmem_ld32(lane_base + C::TM_DP + c * 32, dr);
+                tmem_wait_ld();
+                reg_fence32(sr);
+                reg_fence32(dr);
+                uint32_t pk[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    float ds[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int col = c * 32 + 2 * u + e;
+                        const int key = kt + col;
+                        const bool vis = full || (key >= lo_i && key <= i);
+                        const float p = vis ? ex2_approx(fmaf(__uint_as_float(sr[2 * u + e]), sl2, -lse2))
+                                            : 0.0f;
+                        ds[e] = p * (__uint_as_float(dr[2 * u + e]) - Di);
+                    }
+                    pk[u] = pack_bf16x2(ds[0], ds[1]);
+                }
+                // dS of columns [32c, 32c + 32) goes to TMEM columns
+                // [16c, 16c + 16): S columns already read (chunks <= c).
+                tmem_st16(lane_base + C::TM_S + c * 16, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(L::B_DS_FULL));
+        }
+        if (ok) ok = warp_wait(bar(L::B_ACC_FULL), 0, abort_flag, prm.status);
+        if (ok) {
+            tc_fence_after();
+            __nv_bfloat16* orow = prm.dq + (static_cast<int64_t>(i) * prm.Hq + h) * C::D;
+#pragma unroll 1
+            for (int c = 0; c < C::D / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(lane_base + C::TM_ACC0 + c * 32, r);
+                tmem_wait_ld();
+                reg_fence32(r);
+                uint32_t w[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u)
+                    w[u] = pack_bf16x2(__uint_as_float(r[2 * u]) * prm.scale,
+                                       __uint_as_float(r[2 * u + 1]) * prm.scale);
+                if (row_valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        dst[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == C::MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- dk, dv ----
+template <class C>
+struct DkvLayout {
+    static constexpr int NPAIR = C::NSLOT;                    // Q/dO tile pairs in flight
+    static constexpr int B_KV_FULL = 0;                       // K and V landed
+    static constexpr int B_PAIR_FULL = 1;                     // [NPAIR] Q, dO, lse, delta
+    static constexpr int B_PAIR_EMPTY = B_PAIR_FULL + NPAIR;  // [NPAIR]
+    static constexpr int B_S_FULL = B_PAIR_EMPTY + NPAIR;     // S^T and dP^T done
+    static constexpr int B_PS_FULL = B_S_FULL + 1;            // P^T, dS^T in TMEM (4 warps)
+    static constexpr int B_ACC_FULL = B_PS_FULL + 1;          // dk, dv accumulated
+    static constexpr int B_DRAIN = B_ACC_FULL + 1;
+    static constexpr int NUM_BARS = B_DRAIN + 1;
+    static constexpr int SMEM_K = 0;
+    static constexpr int SMEM_V = SMEM_K + C::TILE_BYTES;
+    static constexpr int SMEM_PAIRS = SMEM_V + C::TILE_BYTES;  // [NPAIR][Q tile, dO tile]
+    static constexpr int PAIR_BYTES = 2 * C::TILE_BYTES;
+    static constexpr int SMEM_SIDE = SMEM_PAIRS + NPAIR * PAIR_BYTES;  // [NPAIR][lse2 128, delta 128]
+    static constexpr int SIDE_BYTES = 2 * 128 * 4;
+    static constexpr int SMEM_BAR = SMEM_SIDE + NPAIR * SIDE_BYTES;
+    static constexpr int SMEM_TMEM_SLOT = SMEM_BAR + NUM_BARS * 8;
+    static constexpr int SMEM_ABORT = SMEM_TMEM_SLOT + 4;
+    static constexpr int SMEM_ALLOC = SMEM_ABORT + 4 + 1024;
+    static_assert(SMEM_ALLOC <= 232448, "shared memory budget exceeded");
+};
+
+template <class C>
+__global__ void __launch_bounds__(C::NUM_THREADS, 1)
+thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                         const __grid_constant__ CUtensorMap tmap_do,
+                         const __grid_constant__ CUtensorMap tmap_k,
+                         const __grid_constant__ CUtensorMap tmap_v, const BwdParams prm) {
+    using L = DkvLayout<C>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = smem_addr(smem_raw);
+    uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
+    const uint32_t sbase = smem_addr(smem);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const BwdKVItem it = prm.kv_items[blockIdx.x];
+    const int G = prm.G;
+    const int n_steps = G * it.n_q;  // (query head, query tile) steps
+
+    auto bar = [&](int idx) -> uint32_t { return sbase + L::SMEM_BAR + 8u * idx; };
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::SMEM_ABORT);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::SMEM_TMEM_SLOT);
+    float* side = reinterpret_cast<float*>(smem + L::SMEM_SIDE);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(L::B_KV_FULL), 1);
+        for (int s = 0; s < L::NPAIR; ++s) {
+            mbar_init(bar(L::B_PAIR_FULL + s), 2);  // TMA bytes + the side values
+            mbar_init(bar(L::B_PAIR_EMPTY + s), 1);
+        }
+        mbar_init(bar(L::B_S_FULL), 1);
+        mbar_init(bar(L::B_PS_FULL), 4);
+        mbar_init(bar(L::B_ACC_FULL), 1);
+        mbar_init(bar(L::B_DRAIN), 1);
+        *abort_flag = *reinterpret_cast<volatile int*>(prm.status) != 0 ? 1 : 0;
+        fence_barrier_init();
+    }
+    if (warp == C::MMA_WARP) {
+        tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const bool skip = *abort_flag != 0;
+
+    if (warp == C::PRODUCER_WARP) {
+        // All 32 lanes stage the per-query lse / delta values; lane 0 issues
+        // the copies.
+        bool ok = !skip;
+        int issued = 0;  // steps whose copies were issued
+        if (ok && lane == 0) {
+            tma_prefetch_desc(&tmap_q);
+            tma_prefetch_desc(&tmap_do);
+            tma_prefetch_desc(&tmap_k);
+            tma_prefetch_desc(&tmap_v);
+            mbar_arrive_expect_tx(bar(L::B_KV_FULL), 2 * C::TILE_BYTES);
+            for (int c = 0; c < C::KCH; ++c) {
+                tma_load_3d(sbase + L::SMEM_K + c * C::BOX_BYTES, &tmap_k, bar(L::B_KV_FULL), c * 64,
+                            it.g, it.k0);
+                tma_load_3d(sbase + L::SMEM_V + c * C::BOX_BYTES, &tmap_v, bar(L::B_KV_FULL), c * 64,
+                            it.g, it.k0);
+            }
+        }
+        for (int s = 0; ok && s < n_steps; ++s) {
+            const int pr = s % L::NPAIR;
+            ok = warp_wait(bar(L::B_PAIR_EMPTY + pr), ((s / L::NPAIR) & 1) ^ 1, abort_flag, prm.status);
+            if (!ok) break;
+            const int h = it.g * G + s / it.n_q;
+            const int i0 = it.k0 + (s % it.n_q) * 128;
+            if (lane == 0) {
+                const uint32_t full = bar(L::B_PAIR_FULL + pr);
+                const uint32_t dst = sbase + L::SMEM_PAIRS + pr * L::PAIR_BYTES;
+                mbar_arrive_expect_tx(full, 2 * C::TILE_BYTES);
+                for (int c = 0; c < C::KCH; ++c) {
+                    tma_load_3d(dst + c * C::BOX_BYTES, &tmap_q, full, c * 64, h, i0);
+                    tma_load_3d(dst + C::TILE_BYTES + c * C::BOX_BYTES, &tmap_do, full, c * 64, h, i0);
+                }
+            }
+            float* sd = side + pr * 256;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int col = lane * 4 + u;
+                const int64_t i = static_cast<int64_t>(i0) + col;
+                const bool in = i < prm.T;
+                sd[col] = in ? prm.lse[i * prm.Hq + h] * kLog2e : 0.0f;
+                sd[128 + col] = in ? prm.delta[i * prm.Hq + h] : 0.0f;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(L::B_PAIR_FULL + pr));
+            issued = s + 1;
+        }
+        if (!ok && !skip && lane == 0) {
+            // Unwinding: let the copies already issued land before exit.
+            drain_wait(bar(L::B_KV_FULL), 0);
+            for (int s = issued - L::NPAIR > 0 ? issued - L::NPAIR : 0; s < issued; ++s)
+                drain_wait(bar(L::B_PAIR_FULL + s % L::NPAIR), (s / L::NPAIR) & 1);
+        }
+        __syncwarp();
+    } else if (warp == C::MMA_WARP) {
+        if (lane == 0 && !skip) {
+            constexpr uint32_t idesc_s = idesc_bf16_f32(128, C::BN, false);
+            constexpr uint32_t idesc_acc = idesc_bf16_f32(128, C::D, true);
+            const uint64_t dk0 = smem_desc_sw128(sbase + L::SMEM_K, 16, 1024);
+            const uint64_t dv0 = smem_desc_sw128(sbase + L::SMEM_V, 16, 1024);
+            const uint64_t dpair0 = smem_desc_sw128(sbase + L::SMEM_PAIRS, 16, 1024);
+            const uint64_t dpairmn0 = smem_desc_sw128(sbase + L::SMEM_PAIRS, C::BOX_BYTES, 1024);
+            auto wait = [&](int idx, uint32_t parity) -> bool {
+                return mbar_wait(bar(idx), parity, abort_flag, prm.status, kStatusTimeout);
+            };
+            bool ok = wait(L::B_KV_FULL, 0);
+            for (int s = 0; ok && s < n_steps; ++s) {
+                const int pr = s % L::NPAIR;
+                ok = wait(L::B_PAIR_FULL + pr, (s / L::NPAIR) & 1);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t qoff = (pr * L::PAIR_BYTES) >> 4;
+                const uint32_t dooff = (pr * L::PAIR_BYTES + C::TILE_BYTES) >> 4;
+#pragma unroll
+                for (int kk = 0; kk < C::D / 16; ++kk) {  // S^T = K Q^T
+                    const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
+                    mma_bf16_ss(tmem_base + C::TM_S, dk0 + o, dpair0 + qoff + o, idesc_s,
+                                kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < C::D / 16; ++kk) {  // dP^T = V dO^T
+                    const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
+                    mma_bf16_ss(tmem_base + C::TM_DP, dv0 + o, dpair0 + dooff + o, idesc_s,
+                                kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bar(L::B_S_FULL));
+                ok = wait(L::B_PS_FULL, s & 1);
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; ++kk) {
+                    const uint32_t o = (kk * 16 * 128) >> 4;  // 16 query rows
+                    // dv += P^T dO
+                    mma_bf16_ts(tmem_base + C::TM_ACC0, tmem_base + C::TM_S + kk * 8,
+                                dpairmn0 + dooff + o, idesc_acc, (s > 0 || kk > 0) ? 1u : 0u);
+                    // dk += dS^T Q
+                    mma_bf16_ts(tmem_base + C::TM_ACC1, tmem_base + C::TM_DP + kk * 8,
+                                dpairmn0 + qoff + o, idesc_acc, (s > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(bar(L::B_PAIR_EMPTY + pr));
+            }
+            if (ok) mma_commit(bar(L::B_ACC_FULL));
+            mma_commit(bar(L::B_DRAIN));
+            drain_wait(bar(L::B_DRAIN), 0);
+        }
+        __syncwarp();
+    } else if (warp < 4) {
+        const int row = warp * 32 + lane;
+        const int j = it.k0 + row;  // key of this TMEM lane
+        const int e_doc = it.doc_end;
+        const bool row_valid = j < e_doc;
+        const int W = prm.window;
+        const float sl2 = prm.scale_log2;
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+        const int k_last = it.k0 + 127 < e_doc - 1 ? it.k0 + 127 : e_doc - 1;
+
+        bool ok = !skip;
+        for (int s = 0; ok && s < n_steps; ++s) {
+            const int pr = s % L::NPAIR;
+            const int i0 = it.k0 + (s % it.n_q) * 128;
+            // The side values of this step were stored before PAIR_FULL.
+            ok = warp_wait(bar(L::B_PAIR_FULL + pr), (s / L::NPAIR) & 1, abort_flag, prm.status) &&
+                 warp_wait(bar(L::B_S_FULL), s & 1, abort_flag, prm.status);
+            if (!ok) break;
+            tc_fence_after();
+            const float* lse2 = side + pr * 256;
+            const float* dlt = lse2 + 128;
+            // Every (key, query) of the tile visible: all queries after every
+            // key, inside the document and inside every key's window.
+            const bool full = i0 >= k_last && i0 + 127 < e_doc && it.k0 + 127 < e_doc &&
+                              (W == 0 || i0 + 127 - it.k0 < W);
+#pragma unroll
+            for (int c = 0; c < C::BN / 32; ++c) {
+                uint32_t sr[32], dr[32];
+                tmem_ld32(lane_base + C::TM_S + c * 32, sr);
+                tmem_ld32(lane_base + C::TM_DP + c * 32, dr);
+                tmem_wait_ld();
+                reg_fence32(sr);
+                reg_fence32(dr);
+                uint32_t pp[16], pd[16];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c * 32 + 4 * u);
+                    const float4 d4 = *reinterpret_cast<const float4*>(dlt + c * 32 + 4 * u);
+                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                    const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+                    float pv[4], dsv[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int col = c * 32 + 4 * u + e;
+                        const int i = i0 + col;
+                        const bool vis = full || (row_valid && i >= j && i < e_doc &&
+                                                  (W == 0 || i - j < W));
+                        const float p = vis ? ex2_approx(fmaf(__uint_as_float(sr[4 * u + e]), sl2, -lv[e]))
+                                            : 0.0f;
+                        pv[e] = p;
+                        dsv[e] = p * (__uint_as_float(dr[4 * u + e]) - dv4[e]);
+                    }
+                    pp[2 * u] = pack_bf16x2(pv[0], pv[1]);
+                    pp[2 * u + 1] = pack_bf16x2(pv[2], pv[3]);
+                    pd[2 * u] = pack_bf16x2(dsv[0], dsv[1]);
+                    pd[2 * u + 1] = pack_bf16x2(dsv[2], dsv[3]);
+                }
+                tmem_st16(lane_base + C::TM_S + c * 16, pp);   // P^T over read S^T columns
+                tmem_st16(lane_base + C::TM_DP + c * 16, pd);  // dS^T over read dP^T columns
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(L::B_PS_FULL));
+        }
+        if (ok) ok = warp_wait(bar(L::B_ACC_FULL), 0, abort_flag, prm.status);
+        if (ok) {
+            tc_fence_after();
+            const int64_t base = (static_cast<int64_t>(j) * prm.Hkv + it.g) * C::D;
+#pragma unroll 1
+            for (int a = 0; a < 2; ++a) {
+                __nv_bfloat16* dst_row = (a == 0 ? prm.dv : prm.dk) + base;
+                const float f = a == 0 ? 1.0f : prm.scale;
+                const uint32_t acc = lane_base + (a == 0 ? C::TM_ACC0 : C::TM_ACC1);
+#pragma unroll 1
+                for (int c = 0; c < C::D / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(acc + c * 32, r);
+                    tmem_wait_ld();
+                    reg_fence32(r);
+                    uint32_t w[16];
+#pragma unroll
+                    for (int u = 0; u < 16; ++u)
+                        w[u] = pack_bf16x2(__uint_as_float(r[2 * u]) * f, __uint_as_float(r[2 * u + 1]) * f);
+                    if (row_valid) {
+                        uint4* dst = reinterpret_cast<uint4*>(dst_row + c * 32);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            dst[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == C::MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+}  // namespace thd

@@ -30,7 +30,7 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for want in ("thd_attn_fwd", "thd_attn_get_error", "thd_attn_status_string", "thd_attn_plan",
-                 "thd_attn_abi_version"):
+                 "thd_attn_abi_version", "thd_attn_bwd", "thd_attn_bwd_workspace_bytes"):
         assert want in names
 
 
@@ -99,3 +99,37 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(swa, "_PKG", str(tmp_path))
     with pytest.raises(ImportError):
         swa.load_library()
+
+
+# --------------------------------------------------------------- backward ---
+
+def _bwd(lib, cu, Hq=4, Hkv=2, D=64, window=0, scale=0.125, ptr=0x10000, lse=0x10000,
+         ws=0x10000, ws_bytes=1 << 30, dq=0x10000):
+    cu = np.asarray(cu, dtype=np.int32)
+    lib.thd_attn_bwd.argtypes = [ctypes.c_void_p] * 6 + [ctypes.POINTER(ctypes.c_int32)] + \
+        [ctypes.c_int] * 5 + [ctypes.c_float] + [ctypes.c_void_p] * 6 + [ctypes.c_size_t, ctypes.c_void_p]
+    return lib.thd_attn_bwd(ptr, ptr, ptr, ptr, lse, ptr,
+                            cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), cu.size - 1,
+                            Hq, Hkv, D, window, scale, None, dq, ptr, ptr, None, ws, ws_bytes, None)
+
+
+def test_bwd_workspace_size(lib):
+    lib.thd_attn_bwd_workspace_bytes.argtypes = [ctypes.c_int64, ctypes.c_int]
+    lib.thd_attn_bwd_workspace_bytes.restype = ctypes.c_size_t
+    assert lib.thd_attn_bwd_workspace_bytes(1000, 6) == 2 * 24064  # 2 x 24000 rounded up to 256
+    assert lib.thd_attn_bwd_workspace_bytes(0, 6) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(cu=[0, 5, 3]), -1),                 # decreasing boundaries
+    (dict(cu=[0, 5], D=256), -2),             # the backward covers D = 64 and 128
+    (dict(cu=[0, 5], D=48), -2),
+    (dict(cu=[0, 5], scale=0.0), -1),
+    (dict(cu=[0, 5], lse=None), -1),          # the forward's lse is required
+    (dict(cu=[0, 5], lse=0x10002), -1),       # misaligned fp32 pointer
+    (dict(cu=[0, 5], dq=0x10008), -1),        # misaligned bf16 pointer
+    (dict(cu=[0, 5], ws=None), -1),
+    (dict(cu=[0, 5], ws_bytes=100), -1),      # workspace smaller than needed
+])
+def test_bwd_rejects_bad_arguments_before_any_launch(lib, kw, code):
+    assert _bwd(lib, **kw) == code
