@@ -23,9 +23,13 @@
 //     bf16 over them, dv += P^T dO and dk += dS^T Q (TMEM operands, dO and Q
 //     as MN-major operands); dk and dv stay in TMEM for the whole group.
 //
-// Warps (both kernels): 0-3 elementwise (thread t owns TMEM lane t), 4 TMA
-// producer, 5 MMA issuer, 6-7 idle.  Every wait is bounded and reports a
-// timeout in the device status word.
+// Warps (both kernels): 0-7 elementwise, 8 TMA producer, 9 MMA issuer, 10-11
+// idle.  Elementwise warp w owns TMEM lanes [32 (w % 4), 32 (w % 4) + 32)
+// and the 64 columns [64 h, 64 h + 64) of S and dP, h = w / 4: no row-wide
+// reduction is needed (the log-sum-exp is known), so the two warps on a
+// sub-partition work on independent halves of every tile.  Half h writes
+// its 64 bf16 results (P, dS) over its own columns [64 h, 64 h + 32).  Every
+// wait is bounded and reports a timeout in the device status word.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -58,6 +62,13 @@ struct BwdParams {
 };
 
 constexpr float kLog2e = 1.4426950408889634f;
+
+// TMEM column (relative to S or dP) of the bf16 operand for K-step kk of an
+// MMA over 128 columns: half kk / 4 is packed into [64 (kk / 4), +32), eight
+// columns (16 values) per step.
+__device__ __forceinline__ constexpr uint32_t pcol(int kk) {
+    return static_cast<uint32_t>(64 * (kk >> 2) + 8 * (kk & 3));
+}
 
 // -------------------------------------------------------------- preprocess --
 // One warp per (token, head) row: delta = sum_c dO * O in fp32; with sinks
@@ -148,9 +159,9 @@ struct BwdConfig {
     static constexpr int TM_ACC1 = 256 + D;  // dk (dkdv kernel)
     static constexpr int TMEM_COLS = 512;
 
-    static constexpr int PRODUCER_WARP = 4;
-    static constexpr int MMA_WARP = 5;
-    static constexpr int NUM_THREADS = 256;
+    static constexpr int PRODUCER_WARP = 8;
+    static constexpr int MMA_WARP = 9;
+    static constexpr int NUM_THREADS = 384;
 
     static_assert(D == 64 || D == 128, "backward kernels: head dim 64 or 128");
     static_assert(TM_ACC1 + D <= 512, "TMEM budget exceeded");
@@ -164,7 +175,7 @@ struct DqLayout {
     static constexpr int B_SLOT_FULL = 1;
     static constexpr int B_SLOT_EMPTY = B_SLOT_FULL + C::NSLOT;
     static constexpr int B_S_FULL = B_SLOT_EMPTY + C::NSLOT;  // S and dP done
-    static constexpr int B_DS_FULL = B_S_FULL + 1;            // dS in TMEM (4 warps)
+    static constexpr int B_DS_FULL = B_S_FULL + 1;            // dS in TMEM (8 warps)
     static constexpr int B_ACC_FULL = B_DS_FULL + 1;          // dq accumulated
     static constexpr int B_DRAIN = B_ACC_FULL + 1;
     static constexpr int NUM_BARS = B_DRAIN + 1;
@@ -206,7 +217,7 @@ thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
             mbar_init(bar(L::B_SLOT_EMPTY + s), 1);
         }
         mbar_init(bar(L::B_S_FULL), 1);
-        mbar_init(bar(L::B_DS_FULL), 4);
+        mbar_init(bar(L::B_DS_FULL), 8);
         mbar_init(bar(L::B_ACC_FULL), 1);
         mbar_init(bar(L::B_DRAIN), 1);
         *abort_flag = *reinterpret_cast<volatile int*>(prm.status) != 0 ? 1 : 0;
@@ -299,7 +310,7 @@ thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 const uint64_t dkmn = dkmn0 + ((kslot * C::TILE_BYTES) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; ++kk)  // dq += dS K
-                    mma_bf16_ts(tmem_base + C::TM_ACC0, tmem_base + C::TM_S + kk * 8,
+                    mma_bf16_ts(tmem_base + C::TM_ACC0, tmem_base + C::TM_S + pcol(kk),
                                 dkmn + ((kk * 16 * 128) >> 4), idesc_acc, (j > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(bar(L::B_SLOT_EMPTY + kslot));  // K(j) consumed
             }
@@ -308,36 +319,40 @@ thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
             drain_wait(bar(L::B_DRAIN), 0);
         }
         __syncwarp();
-    } else if (warp < 4) {
-        const int row = warp * 32 + lane;
+    } else if (warp < 8) {
+        const int h = warp >> 2;  // column half
+        const int wq = warp & 3;
+        const int row = wq * 32 + lane;
         const int i = it.q0 + row;
         const int s_doc = it.doc_start;
         const int r_lo = it.q0 > s_doc ? it.q0 : s_doc;
         const int r_hi = it.q1 - 1;
         const bool row_valid = i >= r_lo && i <= r_hi;
         const int W = prm.window;
-        // Visible keys of this row: [lo_i, i]; an empty range for rows
-        // outside the document.
+        // Visible keys of this row: [lo_i, i]; none for rows outside the
+        // document.
         int lo_i = (W > 0 && i - W + 1 > s_doc) ? i - W + 1 : s_doc;
         if (!row_valid) lo_i = i + 1;
-        const float lse2 = row_valid ? prm.lse[static_cast<int64_t>(i) * prm.Hq + h] * kLog2e : 0.0f;
-        const float Di = row_valid ? prm.delta[static_cast<int64_t>(i) * prm.Hq + h] : 0.0f;
+        const int hq = it.head0;
+        const float lse2 = row_valid ? prm.lse[static_cast<int64_t>(i) * prm.Hq + hq] * kLog2e : 0.0f;
+        const float Di = row_valid ? prm.delta[static_cast<int64_t>(i) * prm.Hq + hq] : 0.0f;
         const float sl2 = prm.scale_log2;
-        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(wq * 32) << 16);
 
         bool ok = !skip;
         for (int j = 0; ok && j < n; ++j) {
             ok = warp_wait(bar(L::B_S_FULL), j & 1, abort_flag, prm.status);
             if (!ok) break;
             tc_fence_after();
-            const int kt = it.kv_start + j * C::BN;
-            const bool full = row_valid && kt >= s_doc && kt + C::BN - 1 <= r_lo &&
-                              (W == 0 || kt >= r_hi - W + 1);
+            const int kh = it.kv_start + j * C::BN + 64 * h;  // first key of this half
+            const bool full = row_valid && kh >= s_doc && kh + 63 <= r_lo &&
+                              (W == 0 || kh >= r_hi - W + 1);
+            const int c_lo = lo_i - kh, c_hi = i - kh;  // visible columns of the half
 #pragma unroll
-            for (int c = 0; c < C::BN / 32; ++c) {
+            for (int cc = 0; cc < 2; ++cc) {
                 uint32_t sr[32], dr[32];
-                tmem_ld32(lane_base + C::TM_S + c * 32, sr);
-                tmem_ld32(lane_base + C::TM_DP + c * 32, dr);
+                tmem_ld32(lane_base + C::TM_S + 64 * h + 32 * cc, sr);
+                tmem_ld32(lane_base + C::TM_DP + 64 * h + 32 * cc, dr);
                 tmem_wait_ld();
                 reg_fence32(sr);
                 reg_fence32(dr);
@@ -347,18 +362,16 @@ thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     float ds[2];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int col = c * 32 + 2 * u + e;
-                        const int key = kt + col;
-                        const bool vis = full || (key >= lo_i && key <= i);
-                        const float p = vis ? ex2_approx(fmaf(__uint_as_float(sr[2 * u + e]), sl2, -lse2))
-                                            : 0.0f;
-                        ds[e] = p * (__uint_as_float(dr[2 * u + e]) - Di);
+                        const int col = 32 * cc + 2 * u + e;
+                        float pv = ex2_approx(fmaf(__uint_as_float(sr[2 * u + e]), sl2, -lse2));
+                        if (!full) pv = (col >= c_lo && col <= c_hi) ? pv : 0.0f;
+                        ds[e] = pv * (__uint_as_float(dr[2 * u + e]) - Di);
                     }
                     pk[u] = pack_bf16x2(ds[0], ds[1]);
                 }
-                // dS of columns [32c, 32c + 32) goes to TMEM columns
-                // [16c, 16c + 16): S columns already read (chunks <= c).
-                tmem_st16(lane_base + C::TM_S + c * 16, pk);
+                // dS of this half's columns [32 cc, 32 cc + 32) goes to TMEM
+                // columns 64 h + [16 cc, 16 cc + 16): S of this half, read.
+                tmem_st16(lane_base + C::TM_S + 64 * h + 16 * cc, pk);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -368,11 +381,13 @@ thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
         if (ok) ok = warp_wait(bar(L::B_ACC_FULL), 0, abort_flag, prm.status);
         if (ok) {
             tc_fence_after();
-            __nv_bfloat16* orow = prm.dq + (static_cast<int64_t>(i) * prm.Hq + h) * C::D;
+            // Half h stores dq columns [h D / 2, (h + 1) D / 2).
+            constexpr int HC = C::D / 2;
+            __nv_bfloat16* orow = prm.dq + (static_cast<int64_t>(i) * prm.Hq + hq) * C::D + h * HC;
 #pragma unroll 1
-            for (int c = 0; c < C::D / 32; ++c) {
+            for (int c = 0; c < HC / 32; ++c) {
                 uint32_t r[32];
-                tmem_ld32(lane_base + C::TM_ACC0 + c * 32, r);
+                tmem_ld32(lane_base + C::TM_ACC0 + h * HC + c * 32, r);
                 tmem_wait_ld();
                 reg_fence32(r);
                 uint32_t w[16];
@@ -406,7 +421,7 @@ struct DkvLayout {
     static constexpr int B_PAIR_FULL = 1;                     // [NPAIR] Q, dO, lse, delta
     static constexpr int B_PAIR_EMPTY = B_PAIR_FULL + NPAIR;  // [NPAIR]
     static constexpr int B_S_FULL = B_PAIR_EMPTY + NPAIR;     // S^T and dP^T done
-    static constexpr int B_PS_FULL = B_S_FULL + 1;            // P^T, dS^T in TMEM (4 warps)
+    static constexpr int B_PS_FULL = B_S_FULL + 1;            // P^T, dS^T in TMEM (8 warps)
     static constexpr int B_ACC_FULL = B_PS_FULL + 1;          // dk, dv accumulated
     static constexpr int B_DRAIN = B_ACC_FULL + 1;
     static constexpr int NUM_BARS = B_DRAIN + 1;
@@ -452,7 +467,7 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
             mbar_init(bar(L::B_PAIR_EMPTY + s), 1);
         }
         mbar_init(bar(L::B_S_FULL), 1);
-        mbar_init(bar(L::B_PS_FULL), 4);
+        mbar_init(bar(L::B_PS_FULL), 8);
         mbar_init(bar(L::B_ACC_FULL), 1);
         mbar_init(bar(L::B_DRAIN), 1);
         *abort_flag = *reinterpret_cast<volatile int*>(prm.status) != 0 ? 1 : 0;
@@ -560,10 +575,10 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 for (int kk = 0; kk < C::BN / 16; ++kk) {
                     const uint32_t o = (kk * 16 * 128) >> 4;  // 16 query rows
                     // dv += P^T dO
-                    mma_bf16_ts(tmem_base + C::TM_ACC0, tmem_base + C::TM_S + kk * 8,
+                    mma_bf16_ts(tmem_base + C::TM_ACC0, tmem_base + C::TM_S + pcol(kk),
                                 dpairmn0 + dooff + o, idesc_acc, (s > 0 || kk > 0) ? 1u : 0u);
                     // dk += dS^T Q
-                    mma_bf16_ts(tmem_base + C::TM_ACC1, tmem_base + C::TM_DP + kk * 8,
+                    mma_bf16_ts(tmem_base + C::TM_ACC1, tmem_base + C::TM_DP + pcol(kk),
                                 dpairmn0 + qoff + o, idesc_acc, (s > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(bar(L::B_PAIR_EMPTY + pr));
@@ -573,55 +588,59 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
             drain_wait(bar(L::B_DRAIN), 0);
         }
         __syncwarp();
-    } else if (warp < 4) {
-        const int row = warp * 32 + lane;
+    } else if (warp < 8) {
+        const int h = warp >> 2;  // column half
+        const int wq = warp & 3;
+        const int row = wq * 32 + lane;
         const int j = it.k0 + row;  // key of this TMEM lane
         const int e_doc = it.doc_end;
         const bool row_valid = j < e_doc;
         const int W = prm.window;
         const float sl2 = prm.scale_log2;
-        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(wq * 32) << 16);
         const int k_last = it.k0 + 127 < e_doc - 1 ? it.k0 + 127 : e_doc - 1;
+        // Queries that see key j: [j, i_hi]; none for keys past the document.
+        int i_hi = e_doc - 1;
+        if (W > 0 && j + W - 1 < i_hi) i_hi = j + W - 1;
+        if (!row_valid) i_hi = j - 1;
 
         bool ok = !skip;
         for (int s = 0; ok && s < n_steps; ++s) {
             const int pr = s % L::NPAIR;
-            const int i0 = it.k0 + (s % it.n_q) * 128;
+            const int ih = it.k0 + (s % it.n_q) * 128 + 64 * h;  // first query of this half
             // The side values of this step were stored before PAIR_FULL.
             ok = warp_wait(bar(L::B_PAIR_FULL + pr), (s / L::NPAIR) & 1, abort_flag, prm.status) &&
                  warp_wait(bar(L::B_S_FULL), s & 1, abort_flag, prm.status);
             if (!ok) break;
             tc_fence_after();
-            const float* lse2 = side + pr * 256;
-            const float* dlt = lse2 + 128;
-            // Every (key, query) of the tile visible: all queries after every
+            const float* lse2 = side + pr * 256 + 64 * h;
+            const float* dlt = side + pr * 256 + 128 + 64 * h;
+            // Every (key, query) of this half visible: its queries after every
             // key, inside the document and inside every key's window.
-            const bool full = i0 >= k_last && i0 + 127 < e_doc && it.k0 + 127 < e_doc &&
-                              (W == 0 || i0 + 127 - it.k0 < W);
+            const bool full = ih >= k_last && ih + 63 < e_doc && it.k0 + 127 < e_doc &&
+                              (W == 0 || ih + 63 - it.k0 < W);
+            const int c_lo = j - ih, c_hi = i_hi - ih;  // visible columns of the half
 #pragma unroll
-            for (int c = 0; c < C::BN / 32; ++c) {
+            for (int cc = 0; cc < 2; ++cc) {
                 uint32_t sr[32], dr[32];
-                tmem_ld32(lane_base + C::TM_S + c * 32, sr);
-                tmem_ld32(lane_base + C::TM_DP + c * 32, dr);
+                tmem_ld32(lane_base + C::TM_S + 64 * h + 32 * cc, sr);
+                tmem_ld32(lane_base + C::TM_DP + 64 * h + 32 * cc, dr);
                 tmem_wait_ld();
                 reg_fence32(sr);
                 reg_fence32(dr);
                 uint32_t pp[16], pd[16];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c * 32 + 4 * u);
-                    const float4 d4 = *reinterpret_cast<const float4*>(dlt + c * 32 + 4 * u);
+                    const float4 l4 = *reinterpret_cast<const float4*>(lse2 + 32 * cc + 4 * u);
+                    const float4 d4 = *reinterpret_cast<const float4*>(dlt + 32 * cc + 4 * u);
                     const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
                     const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
                     float pv[4], dsv[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int col = c * 32 + 4 * u + e;
-                        const int i = i0 + col;
-                        const bool vis = full || (row_valid && i >= j && i < e_doc &&
-                                                  (W == 0 || i - j < W));
-                        const float p = vis ? ex2_approx(fmaf(__uint_as_float(sr[4 * u + e]), sl2, -lv[e]))
-                                            : 0.0f;
+                        const int col = 32 * cc + 4 * u + e;
+                        float p = ex2_approx(fmaf(__uint_as_float(sr[4 * u + e]), sl2, -lv[e]));
+                        if (!full) p = (col >= c_lo && col <= c_hi) ? p : 0.0f;
                         pv[e] = p;
                         dsv[e] = p * (__uint_as_float(dr[4 * u + e]) - dv4[e]);
                     }
@@ -630,8 +649,10 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     pd[2 * u] = pack_bf16x2(dsv[0], dsv[1]);
                     pd[2 * u + 1] = pack_bf16x2(dsv[2], dsv[3]);
                 }
-                tmem_st16(lane_base + C::TM_S + c * 16, pp);   // P^T over read S^T columns
-                tmem_st16(lane_base + C::TM_DP + c * 16, pd);  // dS^T over read dP^T columns
+                // P^T and dS^T of this half's columns [32 cc, 32 cc + 32) go to
+                // columns 64 h + [16 cc, 16 cc + 16) of S^T and dP^T (read).
+                tmem_st16(lane_base + C::TM_S + 64 * h + 16 * cc, pp);
+                tmem_st16(lane_base + C::TM_DP + 64 * h + 16 * cc, pd);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -641,28 +662,26 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
         if (ok) ok = warp_wait(bar(L::B_ACC_FULL), 0, abort_flag, prm.status);
         if (ok) {
             tc_fence_after();
-            const int64_t base = (static_cast<int64_t>(j) * prm.Hkv + it.g) * C::D;
+            // Half 0 stores dv, half 1 stores dk (times the score scale).
+            __nv_bfloat16* dst_row = (h == 0 ? prm.dv : prm.dk) +
+                                     (static_cast<int64_t>(j) * prm.Hkv + it.g) * C::D;
+            const float f = h == 0 ? 1.0f : prm.scale;
+            const uint32_t acc = lane_base + (h == 0 ? C::TM_ACC0 : C::TM_ACC1);
 #pragma unroll 1
-            for (int a = 0; a < 2; ++a) {
-                __nv_bfloat16* dst_row = (a == 0 ? prm.dv : prm.dk) + base;
-                const float f = a == 0 ? 1.0f : prm.scale;
-                const uint32_t acc = lane_base + (a == 0 ? C::TM_ACC0 : C::TM_ACC1);
-#pragma unroll 1
-                for (int c = 0; c < C::D / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(acc + c * 32, r);
-                    tmem_wait_ld();
-                    reg_fence32(r);
-                    uint32_t w[16];
+            for (int c = 0; c < C::D / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(acc + c * 32, r);
+                tmem_wait_ld();
+                reg_fence32(r);
+                uint32_t w[16];
 #pragma unroll
-                    for (int u = 0; u < 16; ++u)
-                        w[u] = pack_bf16x2(__uint_as_float(r[2 * u]) * f, __uint_as_float(r[2 * u + 1]) * f);
-                    if (row_valid) {
-                        uint4* dst = reinterpret_cast<uint4*>(dst_row + c * 32);
+                for (int u = 0; u < 16; ++u)
+                    w[u] = pack_bf16x2(__uint_as_float(r[2 * u]) * f, __uint_as_float(r[2 * u + 1]) * f);
+                if (row_valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(dst_row + c * 32);
 #pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            dst[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
-                    }
+                    for (int u = 0; u < 4; ++u)
+                        dst[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
                 }
             }
         }
