@@ -14,9 +14,9 @@
 // them through memory, so nothing is accumulated with atomics and the result
 // is bitwise reproducible:
 //   * dq kernel: one CTA per (128-row query tile, query head), looping over
-//     the key tiles the tile sees: S = Q K^T, dP = dO V^T (both from shared
-//     memory), dS written as bf16 over S in TMEM, dq += dS K (dS from TMEM,
-//     K from shared memory as an MN-major operand).
+//     the key tiles the tile sees: S = Q K^T, dP = dO V^T, dS written as bf16
+//     over S in TMEM, dq += dS K (dS from TMEM, K from shared memory as an
+//     MN-major operand).
 //   * dkdv kernel: one CTA per (128-key tile, kv head), looping over the
 //     query heads of the group and the query tiles that see the keys:
 //     S^T = K Q^T and dP^T = V dO^T (TMEM lane = key), P^T and dS^T written as
@@ -174,8 +174,9 @@ struct DqLayout {
     static constexpr int B_IN_FULL = 0;                       // Q and dO landed
     static constexpr int B_SLOT_FULL = 1;
     static constexpr int B_SLOT_EMPTY = B_SLOT_FULL + C::NSLOT;
-    static constexpr int B_S_FULL = B_SLOT_EMPTY + C::NSLOT;  // S and dP done
-    static constexpr int B_DS_FULL = B_S_FULL + 1;            // dS in TMEM (8 warps)
+    static constexpr int B_S_FULL = B_SLOT_EMPTY + C::NSLOT;  // S done
+    static constexpr int B_DP_FULL = B_S_FULL + 1;            // dP done
+    static constexpr int B_DS_FULL = B_DP_FULL + 1;           // dS in TMEM (8 warps)
     static constexpr int B_ACC_FULL = B_DS_FULL + 1;          // dq accumulated
     static constexpr int B_DRAIN = B_ACC_FULL + 1;
     static constexpr int NUM_BARS = B_DRAIN + 1;
@@ -217,6 +218,7 @@ thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
             mbar_init(bar(L::B_SLOT_EMPTY + s), 1);
         }
         mbar_init(bar(L::B_S_FULL), 1);
+        mbar_init(bar(L::B_DP_FULL), 1);
         mbar_init(bar(L::B_DS_FULL), 8);
         mbar_init(bar(L::B_ACC_FULL), 1);
         mbar_init(bar(L::B_DRAIN), 1);
@@ -297,12 +299,13 @@ thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
                     mma_bf16_ss(tmem_base + C::TM_S, dq0 + o, dk + o, idesc_s, kk > 0 ? 1u : 0u);
                 }
+                mma_commit(bar(L::B_S_FULL));  // the exponentials start under dP
 #pragma unroll
                 for (int kk = 0; kk < C::D / 16; ++kk) {  // dP = dO V^T
                     const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
                     mma_bf16_ss(tmem_base + C::TM_DP, ddo0 + o, dv + o, idesc_s, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(bar(L::B_S_FULL));
+                mma_commit(bar(L::B_DP_FULL));
                 mma_commit(bar(L::B_SLOT_EMPTY + vslot));  // V(j) consumed
                 ok = wait(L::B_DS_FULL, j & 1);
                 if (!ok) break;
@@ -348,29 +351,37 @@ thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
             const bool full = row_valid && kh >= s_doc && kh + 63 <= r_lo &&
                               (W == 0 || kh >= r_hi - W + 1);
             const int c_lo = lo_i - kh, c_hi = i - kh;  // visible columns of the half
+            // P of this half (64 values) while the tensor core computes dP.
+            float pv[64];
+            {
+                uint32_t sr[64];
+                tmem_ld32(lane_base + C::TM_S + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                tmem_ld32(lane_base + C::TM_S + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                tmem_wait_ld();
+                reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+#pragma unroll
+                for (int c = 0; c < 64; ++c) {
+                    const float x = ex2_approx(fmaf(__uint_as_float(sr[c]), sl2, -lse2));
+                    pv[c] = (full || (c >= c_lo && c <= c_hi)) ? x : 0.0f;
+                }
+            }
+            ok = warp_wait(bar(L::B_DP_FULL), j & 1, abort_flag, prm.status);
+            if (!ok) break;
+            tc_fence_after();
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
-                uint32_t sr[32], dr[32];
-                tmem_ld32(lane_base + C::TM_S + 64 * h + 32 * cc, sr);
+                uint32_t dr[32];
                 tmem_ld32(lane_base + C::TM_DP + 64 * h + 32 * cc, dr);
                 tmem_wait_ld();
-                reg_fence32(sr);
                 reg_fence32(dr);
                 uint32_t pk[16];
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    float ds[2];
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int col = 32 * cc + 2 * u + e;
-                        float pv = ex2_approx(fmaf(__uint_as_float(sr[2 * u + e]), sl2, -lse2));
-                        if (!full) pv = (col >= c_lo && col <= c_hi) ? pv : 0.0f;
-                        ds[e] = pv * (__uint_as_float(dr[2 * u + e]) - Di);
-                    }
-                    pk[u] = pack_bf16x2(ds[0], ds[1]);
-                }
+                for (int u = 0; u < 16; ++u)
+                    pk[u] = pack_bf16x2(pv[32 * cc + 2 * u] * (__uint_as_float(dr[2 * u]) - Di),
+                                        pv[32 * cc + 2 * u + 1] * (__uint_as_float(dr[2 * u + 1]) - Di));
                 // dS of this half's columns [32 cc, 32 cc + 32) goes to TMEM
-                // columns 64 h + [16 cc, 16 cc + 16): S of this half, read.
+                // columns 64 h + [16 cc, 16 cc + 16) (S of this half, read).
                 tmem_st16(lane_base + C::TM_S + 64 * h + 16 * cc, pk);
             }
             tmem_wait_st();
@@ -420,9 +431,11 @@ struct DkvLayout {
     static constexpr int B_KV_FULL = 0;                       // K and V landed
     static constexpr int B_PAIR_FULL = 1;                     // [NPAIR] Q, dO, lse, delta
     static constexpr int B_PAIR_EMPTY = B_PAIR_FULL + NPAIR;  // [NPAIR]
-    static constexpr int B_S_FULL = B_PAIR_EMPTY + NPAIR;     // S^T and dP^T done
-    static constexpr int B_PS_FULL = B_S_FULL + 1;            // P^T, dS^T in TMEM (8 warps)
-    static constexpr int B_ACC_FULL = B_PS_FULL + 1;          // dk, dv accumulated
+    static constexpr int B_S_FULL = B_PAIR_EMPTY + NPAIR;     // S^T done
+    static constexpr int B_DP_FULL = B_S_FULL + 1;            // dP^T done
+    static constexpr int B_P_READY = B_DP_FULL + 1;           // P^T in TMEM (8 warps)
+    static constexpr int B_DS_READY = B_P_READY + 1;          // dS^T in TMEM (8 warps)
+    static constexpr int B_ACC_FULL = B_DS_READY + 1;         // dk, dv accumulated
     static constexpr int B_DRAIN = B_ACC_FULL + 1;
     static constexpr int NUM_BARS = B_DRAIN + 1;
     static constexpr int SMEM_K = 0;
@@ -467,7 +480,9 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
             mbar_init(bar(L::B_PAIR_EMPTY + s), 1);
         }
         mbar_init(bar(L::B_S_FULL), 1);
-        mbar_init(bar(L::B_PS_FULL), 8);
+        mbar_init(bar(L::B_DP_FULL), 1);
+        mbar_init(bar(L::B_P_READY), 8);
+        mbar_init(bar(L::B_DS_READY), 8);
         mbar_init(bar(L::B_ACC_FULL), 1);
         mbar_init(bar(L::B_DRAIN), 1);
         *abort_flag = *reinterpret_cast<volatile int*>(prm.status) != 0 ? 1 : 0;
@@ -561,26 +576,30 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     mma_bf16_ss(tmem_base + C::TM_S, dk0 + o, dpair0 + qoff + o, idesc_s,
                                 kk > 0 ? 1u : 0u);
                 }
+                mma_commit(bar(L::B_S_FULL));  // the exponentials start under dP^T
 #pragma unroll
                 for (int kk = 0; kk < C::D / 16; ++kk) {  // dP^T = V dO^T
                     const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
                     mma_bf16_ss(tmem_base + C::TM_DP, dv0 + o, dpair0 + dooff + o, idesc_s,
                                 kk > 0 ? 1u : 0u);
                 }
-                mma_commit(bar(L::B_S_FULL));
-                ok = wait(L::B_PS_FULL, s & 1);
+                mma_commit(bar(L::B_DP_FULL));
+                ok = wait(L::B_P_READY, s & 1);
                 if (!ok) break;
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < C::BN / 16; ++kk) {
-                    const uint32_t o = (kk * 16 * 128) >> 4;  // 16 query rows
-                    // dv += P^T dO
+                for (int kk = 0; kk < C::BN / 16; ++kk)  // dv += P^T dO (16 query rows a step)
                     mma_bf16_ts(tmem_base + C::TM_ACC0, tmem_base + C::TM_S + pcol(kk),
-                                dpairmn0 + dooff + o, idesc_acc, (s > 0 || kk > 0) ? 1u : 0u);
-                    // dk += dS^T Q
+                                dpairmn0 + dooff + ((kk * 16 * 128) >> 4), idesc_acc,
+                                (s > 0 || kk > 0) ? 1u : 0u);
+                ok = wait(L::B_DS_READY, s & 1);  // dS^T is computed under dv
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; ++kk)  // dk += dS^T Q
                     mma_bf16_ts(tmem_base + C::TM_ACC1, tmem_base + C::TM_DP + pcol(kk),
-                                dpairmn0 + qoff + o, idesc_acc, (s > 0 || kk > 0) ? 1u : 0u);
-                }
+                                dpairmn0 + qoff + ((kk * 16 * 128) >> 4), idesc_acc,
+                                (s > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(bar(L::B_PAIR_EMPTY + pr));
             }
             if (ok) mma_commit(bar(L::B_ACC_FULL));
@@ -620,44 +639,66 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
             const bool full = ih >= k_last && ih + 63 < e_doc && it.k0 + 127 < e_doc &&
                               (W == 0 || ih + 63 - it.k0 < W);
             const int c_lo = j - ih, c_hi = i_hi - ih;  // visible columns of the half
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                uint32_t sr[32], dr[32];
-                tmem_ld32(lane_base + C::TM_S + 64 * h + 32 * cc, sr);
-                tmem_ld32(lane_base + C::TM_DP + 64 * h + 32 * cc, dr);
+            // P^T of this half (while the tensor core computes dP^T) ...
+            float pv[64];
+            {
+                uint32_t sr[64];
+                tmem_ld32(lane_base + C::TM_S + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                tmem_ld32(lane_base + C::TM_S + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
                 tmem_wait_ld();
-                reg_fence32(sr);
-                reg_fence32(dr);
-                uint32_t pp[16], pd[16];
+                reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const float4 l4 = *reinterpret_cast<const float4*>(lse2 + 32 * cc + 4 * u);
-                    const float4 d4 = *reinterpret_cast<const float4*>(dlt + 32 * cc + 4 * u);
+                for (int u = 0; u < 16; ++u) {
+                    const float4 l4 = *reinterpret_cast<const float4*>(lse2 + 4 * u);
                     const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-                    const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
-                    float pv[4], dsv[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int col = 32 * cc + 4 * u + e;
-                        float p = ex2_approx(fmaf(__uint_as_float(sr[4 * u + e]), sl2, -lv[e]));
-                        if (!full) p = (col >= c_lo && col <= c_hi) ? p : 0.0f;
-                        pv[e] = p;
-                        dsv[e] = p * (__uint_as_float(dr[4 * u + e]) - dv4[e]);
+                        const int c = 4 * u + e;
+                        const float x = ex2_approx(fmaf(__uint_as_float(sr[c]), sl2, -lv[e]));
+                        pv[c] = (full || (c >= c_lo && c <= c_hi)) ? x : 0.0f;
                     }
-                    pp[2 * u] = pack_bf16x2(pv[0], pv[1]);
-                    pp[2 * u + 1] = pack_bf16x2(pv[2], pv[3]);
+                }
+                uint32_t pp[32];
+#pragma unroll
+                for (int u = 0; u < 32; ++u) pp[u] = pack_bf16x2(pv[2 * u], pv[2 * u + 1]);
+                // Over this half's own S^T columns [64 h, 64 h + 32), all read.
+                tmem_st16(lane_base + C::TM_S + 64 * h, *reinterpret_cast<uint32_t(*)[16]>(&pp[0]));
+                tmem_st16(lane_base + C::TM_S + 64 * h + 16, *reinterpret_cast<uint32_t(*)[16]>(&pp[16]));
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(L::B_P_READY));
+            // ... then dS^T = P^T (dP^T - delta) while it computes dv.
+            ok = warp_wait(bar(L::B_DP_FULL), s & 1, abort_flag, prm.status);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                uint32_t dr[32];
+                tmem_ld32(lane_base + C::TM_DP + 64 * h + 32 * cc, dr);
+                tmem_wait_ld();
+                reg_fence32(dr);
+                uint32_t pd[16];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const float4 d4 = *reinterpret_cast<const float4*>(dlt + 32 * cc + 4 * u);
+                    const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+                    float dsv[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dsv[e] = pv[32 * cc + 4 * u + e] * (__uint_as_float(dr[4 * u + e]) - dv4[e]);
                     pd[2 * u] = pack_bf16x2(dsv[0], dsv[1]);
                     pd[2 * u + 1] = pack_bf16x2(dsv[2], dsv[3]);
                 }
-                // P^T and dS^T of this half's columns [32 cc, 32 cc + 32) go to
-                // columns 64 h + [16 cc, 16 cc + 16) of S^T and dP^T (read).
-                tmem_st16(lane_base + C::TM_S + 64 * h + 16 * cc, pp);
+                // Over dP^T columns 64 h + [16 cc, 16 cc + 16), already read.
                 tmem_st16(lane_base + C::TM_DP + 64 * h + 16 * cc, pd);
             }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(L::B_PS_FULL));
+            if (lane == 0) mbar_arrive(bar(L::B_DS_READY));
         }
         if (ok) ok = warp_wait(bar(L::B_ACC_FULL), 0, abort_flag, prm.status);
         if (ok) {
