@@ -12,6 +12,8 @@ Two independent formulations live here:
 * :func:`attention_bwd` / :func:`attention_bwd_q_rows` -- the fp64 gradient
   of that forward (dq, dk, dv, dsink), the plain derivative written out in the
   same C file;
+* :mod:`oracle.prologue` -- the Q/K prologue (scaleless RMSNorm, then
+  split-half RoPE at per-document positions) in plain fp64 numpy;
 * :func:`dense_attention` -- a dense brute force for tiny packs: it builds the
   boolean ``[query_tokens, key_tokens]`` causal document mask the way
   ``SequenceLayout.allowed`` is described ("mistral_large4.attention" page),
