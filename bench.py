@@ -8,6 +8,12 @@ TFLOP/s over valid (unmasked) query-key pairs, FLOP = 4 * pairs * D * Hq.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
+``--pass bwd`` times the backward (thd_attn_bwd: dq, dk, dv, dsink) on the
+same pack instead, FLOP = 2.5x the forward's (the usual count of a backward
+that recomputes P); ``--pass prologue`` times the in-place Q/K prologue
+(thd_qk_norm_rope), bytes = Q and K read and written once.  Both print one
+JSON line of the same shape with their own metric.
+
 Prints one JSON line on stdout (rank 0).  Multi-GPU runs are launched with
 torchrun, one process per GPU; every rank runs its own pack of the same shape
 (no data-path collective), the timed region is bracketed by a barrier and a
@@ -66,6 +72,8 @@ def parse_args(argv=None):
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd", "prologue"], default="fwd",
+                    help="what one step runs (default: the forward, the headline)")
     return ap.parse_args(argv)
 
 
@@ -385,11 +393,105 @@ def run_ours(args, info):
     return 0
 
 
+# ------------------------------------------------- backward and prologue --
+
+def run_other_pass(args, info):
+    """--pass bwd / prologue: device-timed steps of thd_attn_bwd or
+    thd_qk_norm_rope on the same synthetic pack (inputs resident in HBM)."""
+    import sliding_window_gqa_cu_b200 as swa
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the CUDA path has no CPU fallback)")
+    multirank.init("nccl")
+    device = torch.device("cuda", info.local_rank)
+    torch.cuda.set_device(device)
+    swa.load_library()
+    cfg = workloads.CONFIGS[args.workload]
+    pack = workloads.make_pack(cfg, args.seed, tensor_seed=multirank.tensor_seed(args.seed, info.rank),
+                               T_override=args.tokens)
+    cu = pack["cu_seqlens"]
+    T = pack["T"]
+    pairs = metrics.valid_pairs(cu, cfg.window)
+    q, k, v = (pack[n].to(device) for n in "qkv")
+    sinks = pack["sinks"].to(device) if pack["sinks"] is not None else None
+    stream = torch.cuda.current_stream(device)
+    peaks, peak_src = measured_peaks()
+    if args.pass_ == "bwd":
+        out, lse = swa.thd_attn_fwd(q, k, v, cu, cfg.window, cfg.scale, sinks, stream=stream)
+        g = torch.Generator(device="cpu").manual_seed(7)
+        dout = torch.randn((T, cfg.Hq, cfg.D), generator=g).to(torch.bfloat16).to(device)
+        ws = torch.empty((max(16, swa.thd_attn_bwd_workspace_bytes(T, cfg.Hq)),), dtype=torch.uint8,
+                         device=device)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        work = 2.5 * 4 * pairs * cfg.D * cfg.Hq
+        launches = 4 if sinks is not None else 3
+
+        def step():
+            swa.thd_attn_bwd(q, k, v, out, lse, dout, cu, cfg.window, cfg.scale, sinks, dq=dq, dk=dk,
+                             dv=dv, workspace=ws, stream=stream)
+        metric, unit = "THD varlen attention bwd TFLOP/s (valid pairs, 2.5x forward FLOP)", "TFLOP/s"
+        peak = float(peaks["bf16_tflops"])
+        bound, kern = "tensor", "thd_attn_bwd_dq_kernel + thd_attn_bwd_dkdv_kernel"
+    else:
+        work = 2 * T * (cfg.Hq + cfg.Hkv) * cfg.D * 2  # bytes: Q and K read and written once
+        launches = 1
+
+        def step():
+            swa.thd_qk_norm_rope(q, k, cu, stream=stream)
+        metric, unit = "Q/K prologue (scaleless RMSNorm + split-half RoPE) GB/s", "GB/s"
+        peak = float(peaks["hbm_gbs"])
+        bound, kern = "hbm", "thd_qk_norm_rope_kernel"
+    step()
+    torch.cuda.synchronize(device)
+    if swa.thd_attn_get_error(stream) != 0:
+        raise RuntimeError("kernel reported an error status")
+    clocks = ClockSampler(device)
+    for _ in range(args.warmup):
+        step()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    multirank.barrier(device)
+    torch.cuda.synchronize(device)
+    h0 = time.time()
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    h1 = time.time()
+    multirank.barrier(device)
+    clocks.stop()
+    ms = multirank.max_over_ranks(start.elapsed_time(end), device)
+    scale = 1e12 if unit == "TFLOP/s" else 1e9
+    value = multirank.aggregate_rate(work * args.steps, info.world, ms / 1e3) / scale
+    achieved = work / (ms / args.steps / 1e3) / scale
+    csum = clocks.summary(h0, h1)
+    if info.is_root:
+        line = {
+            "metric": metric, "value": value, "unit": unit, "n_gpus": info.world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "pass": args.pass_,
+            "config": workload_config(cfg, cu, pairs, {"parallelism": f"pack-parallel x{info.world}"}),
+            "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                         "frac": achieved / peak, "traffic": None, "kernel": kern,
+                         "peak_source": f"{peak_src} (MEASURED_PEAKS.json)"},
+            "cpu_baseline": None, "e2e": None, "gpu_launches": launches * args.steps,
+            "clocks": {k: csum[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+        }
+        log(f"[bench] {cfg.name} {args.pass_}: {ms / args.steps:.3f} ms/step, {value:.1f} {unit} "
+            f"({100 * achieved / peak:.1f}% of measured {peak:.0f}), clocks {csum}")
+        print(json.dumps(line), flush=True)
+    multirank.shutdown()
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     info = multirank.rank_info()
     if args.impl == "reference":
         return run_reference(args, info)
+    if args.pass_ != "fwd":
+        return run_other_pass(args, info)
     return run_ours(args, info)
 
 

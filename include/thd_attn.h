@@ -229,6 +229,31 @@ int thd_attn_bwd(const void* q, const void* k, const void* v,
                  void* workspace, size_t workspace_bytes,
                  void* stream);
 
+/*
+ * ------------------------------------------------------------------ prologue
+ * Q/K prologue of the attention, in place: every query and key head vector
+ * is normalised by the parameter-free RMSNorm ("muse_glimmer.model" page,
+ * MuseGlimmerScalelessRMSNorm: y = x / sqrt(mean(x^2) + eps), eps default
+ * 1e-5) and then, when apply_rope != 0, turned by the split-half rotary
+ * embedding (MuseGlimmerRotaryEmbedding, theta default 500000, and
+ * apply_rotary_emb): for k < D/2 with a = position * theta^(-2k/D),
+ *   out[k] = y[k] cos a - y[k + D/2] sin a,  out[k + D/2] = y[k + D/2] cos a + y[k] sin a.
+ *   q          bf16 device [T, Hq, D], overwritten
+ *   k          bf16 device [T, Hkv, D], overwritten (may be NULL if Hkv == 0)
+ *   cu_seqlens, n_docs  HOST int32 document boundaries as for thd_attn_fwd
+ *   positions_or_null   device int32 [T] positions; NULL = each token's
+ *              offset inside its document (the position resets at every
+ *              document start of the pack)
+ *   D          64, 128 or 256;  eps > 0;  theta > 1 (ignored without RoPE)
+ * 16-byte aligned tensors.  fp32 arithmetic with the angle reduced in double
+ * precision, one bf16 rounding.  With default positions the library keeps a
+ * device copy of the last cu_seqlens per device (updated synchronously when
+ * it changes).  Returns THD_OK or a negative code before anything is enqueued.
+ */
+int thd_qk_norm_rope(void* q, void* k, const int32_t* cu_seqlens, int n_docs,
+                     const int32_t* positions_or_null, int Hq, int Hkv, int D,
+                     float eps, float theta, int apply_rope, void* stream);
+
 /* ABI version of this header: (major << 16) | minor. */
 int thd_attn_abi_version(void);
 

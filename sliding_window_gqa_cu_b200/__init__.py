@@ -79,6 +79,9 @@ def load_library():
     lib.thd_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int,
                                  ctypes.c_float, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.thd_attn_bwd.restype = c_int
+    lib.thd_qk_norm_rope.argtypes = [vp, vp, i32p, c_int, vp, c_int, c_int, c_int, ctypes.c_float,
+                                     ctypes.c_float, c_int, vp]
+    lib.thd_qk_norm_rope.restype = c_int
     lib.thd_attn_abi_version.argtypes = []
     lib.thd_attn_abi_version.restype = c_int
     _lib = lib
@@ -233,6 +236,45 @@ def thd_attn_bwd(q, k, v, out, lse, dout, cu_seqlens, window: int = 0,
 def thd_attn_bwd_workspace_bytes(T: int, Hq: int) -> int:
     """Workspace bytes :func:`thd_attn_bwd` needs for T tokens and Hq query heads."""
     return int(load_library().thd_attn_bwd_workspace_bytes(int(T), int(Hq)))
+
+
+def thd_qk_norm_rope(q, k, cu_seqlens, eps: float = 1e-5, theta: float = 500000.0,
+                     apply_rope: bool = True, positions=None, stream=None):
+    """In-place Q/K prologue: scaleless RMSNorm of every head vector, then
+    split-half RoPE at per-document positions (or ``positions``, an int32 CUDA
+    tensor [T]).  q: bf16 CUDA [T, Hq, D]; k: bf16 CUDA [T, Hkv, D] or None.
+    Returns (q, k)."""
+    import torch
+
+    lib = load_library()
+    T, Hq, D = q.shape
+    for name, t in (("q", q), ("k", k)):
+        if t is None:
+            continue
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 3:
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor [tokens, heads, head_dim]")
+        if t.shape[0] != T or t.shape[2] != D:
+            raise ValueError("q and k must share tokens and head_dim")
+    Hkv = k.shape[1] if k is not None else 0
+    cu = _cu_array(cu_seqlens)
+    if int(cu[-1]) != T:
+        raise ValueError(f"cu_seqlens[-1]={int(cu[-1])} does not match {T} tokens")
+    if positions is not None:
+        if positions.dtype != torch.int32 or not positions.is_cuda or positions.numel() != T:
+            raise ValueError("positions must be an int32 CUDA tensor [tokens]")
+        positions = positions.contiguous()
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        rc = lib.thd_qk_norm_rope(
+            q.data_ptr(), k.data_ptr() if k is not None else None,
+            cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), cu.size - 1,
+            positions.data_ptr() if positions is not None else None,
+            Hq, Hkv, D, float(eps), float(theta), int(bool(apply_rope)),
+            ctypes.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise ThdAttnError(rc, "thd_qk_norm_rope")
+    return q, k
 
 
 def thd_attn_get_error(stream=None) -> int:

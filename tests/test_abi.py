@@ -30,7 +30,8 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for want in ("thd_attn_fwd", "thd_attn_get_error", "thd_attn_status_string", "thd_attn_plan",
-                 "thd_attn_abi_version", "thd_attn_bwd", "thd_attn_bwd_workspace_bytes"):
+                 "thd_attn_abi_version", "thd_attn_bwd", "thd_attn_bwd_workspace_bytes",
+                 "thd_qk_norm_rope"):
         assert want in names
 
 
@@ -133,3 +134,31 @@ def test_bwd_workspace_size(lib):
 ])
 def test_bwd_rejects_bad_arguments_before_any_launch(lib, kw, code):
     assert _bwd(lib, **kw) == code
+
+
+# --------------------------------------------------------------- prologue ---
+
+def _pro(lib, cu, Hq=4, Hkv=2, D=128, eps=1e-5, theta=500000.0, rope=1, ptr=0x10000, kptr=0x10000,
+         pos=None):
+    cu = np.asarray(cu, dtype=np.int32)
+    lib.thd_qk_norm_rope.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32),
+                                     ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                     ctypes.c_int, ctypes.c_float, ctypes.c_float, ctypes.c_int,
+                                     ctypes.c_void_p]
+    return lib.thd_qk_norm_rope(ptr, kptr, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                cu.size - 1, pos, Hq, Hkv, D, eps, theta, rope, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(cu=[0, 5, 3]), -1),
+    (dict(cu=[2, 5]), -1),
+    (dict(cu=[0, 5], D=96), -2),
+    (dict(cu=[0, 5], eps=0.0), -1),
+    (dict(cu=[0, 5], theta=0.5), -1),
+    (dict(cu=[0, 5], ptr=0x10008), -1),       # misaligned q
+    (dict(cu=[0, 5], pos=0x10002), -1),       # misaligned positions
+    (dict(cu=[0, 5], kptr=None), -1),         # k missing with Hkv > 0
+    (dict(cu=[0, 0]), 0),                     # empty pack: nothing to do
+])
+def test_prologue_rejects_bad_arguments_before_any_launch(lib, kw, code):
+    assert _pro(lib, **kw) == code
