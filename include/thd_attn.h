@@ -134,6 +134,36 @@ int thd_attn_plan(const int32_t* cu_seqlens, int n_docs, int Hq, int Hkv, int D,
                   thd_work_item* items, int64_t capacity, int64_t* n_items);
 
 /*
+ * Local step of a context-parallel forward: the query rows [q_begin, q_end)
+ * of the pack against keys and values of the WHOLE pack.  The Magi plans
+ * shard the packed tokens over the context-parallel ranks and gather K/V
+ * ("muse_spark.magi_cp" page: one plan per microbatch over the rank's local
+ * tokens, keys exchanged by the attention engine); a rank that owns rows
+ * [q_begin, q_end) and holds the gathered K/V computes exactly those rows of
+ * thd_attn_fwd's result.
+ *   q          bf16 device [q_end - q_begin, Hq, D]: the rows it owns
+ *   k, v       bf16 device [T, Hkv, D]: the whole pack (e.g. all-gathered)
+ *   out, lse   [q_end - q_begin, Hq, D] bf16 and [q_end - q_begin, Hq] fp32
+ *   other arguments as thd_attn_fwd (cu_seqlens covers the whole pack)
+ * 0 <= q_begin <= q_end <= T, else THD_ERR_INVALID_ARG.  thd_attn_fwd is
+ * the range [0, T).
+ */
+int thd_attn_fwd_range(const void* q, const void* k, const void* v,
+                       const int32_t* cu_seqlens, int n_docs,
+                       int64_t q_begin, int64_t q_end,
+                       int Hq, int Hkv, int D, int window, float scale,
+                       const float* sinks_or_null,
+                       void* out, float* lse,
+                       void* stream);
+
+/* Host-only: the schedule thd_attn_fwd_range uses (q0 of a tile that would
+ * reach before q_begin > 0 is raised to q_begin).  Same conventions as
+ * thd_attn_plan. */
+int thd_attn_plan_range(const int32_t* cu_seqlens, int n_docs, int64_t q_begin, int64_t q_end,
+                        int Hq, int Hkv, int D, int window,
+                        thd_work_item* items, int64_t capacity, int64_t* n_items);
+
+/*
  * Allocation-free variant of thd_attn_fwd.  The pages have no counterpart of
  * this entry point: it exists for callers that may not allocate device
  * memory -- runtimes that reserve all device memory up front and hand out

@@ -79,6 +79,13 @@ def load_library():
     lib.thd_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int,
                                  ctypes.c_float, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.thd_attn_bwd.restype = c_int
+    lib.thd_attn_fwd_range.argtypes = [vp, vp, vp, i32p, c_int, ctypes.c_int64, ctypes.c_int64,
+                                       c_int, c_int, c_int, c_int, ctypes.c_float, vp, vp, vp, vp]
+    lib.thd_attn_fwd_range.restype = c_int
+    lib.thd_attn_plan_range.argtypes = [i32p, c_int, ctypes.c_int64, ctypes.c_int64, c_int, c_int,
+                                        c_int, c_int, vp, ctypes.c_int64,
+                                        ctypes.POINTER(ctypes.c_int64)]
+    lib.thd_attn_plan_range.restype = c_int
     lib.thd_qk_norm_rope.argtypes = [vp, vp, i32p, c_int, vp, c_int, c_int, c_int, ctypes.c_float,
                                      ctypes.c_float, c_int, vp]
     lib.thd_qk_norm_rope.restype = c_int
@@ -275,6 +282,77 @@ def thd_qk_norm_rope(q, k, cu_seqlens, eps: float = 1e-5, theta: float = 500000.
     if rc != 0:
         raise ThdAttnError(rc, "thd_qk_norm_rope")
     return q, k
+
+
+def thd_attn_fwd_range(q, k, v, cu_seqlens, q_begin: int, q_end: int, window: int = 0,
+                       scale: Optional[float] = None, sinks=None, out=None, lse=None,
+                       return_lse: bool = True, stream=None):
+    """Forward of the query rows [q_begin, q_end) of the pack against K/V of
+    the whole pack (the local step of a context-parallel forward).
+
+    q: bf16 CUDA [q_end - q_begin, Hq, D]; k, v: bf16 CUDA [T, Hkv, D];
+    cu_seqlens: host boundaries of the whole pack.  Returns ``(out, lse)`` for
+    those rows.
+    """
+    import torch
+
+    lib = load_library()
+    Tq, Hq, D = q.shape
+    T, Hkv = k.shape[0], k.shape[1]
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 3:
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    if v.shape != k.shape or k.shape[2] != D:
+        raise ValueError("k and v must be [tokens, kv_heads, head_dim] with q's head_dim")
+    cu = _cu_array(cu_seqlens)
+    if int(cu[-1]) != T:
+        raise ValueError(f"cu_seqlens[-1]={int(cu[-1])} does not match {T} key tokens")
+    if not (0 <= q_begin <= q_end <= T) or q_end - q_begin != Tq:
+        raise ValueError("q must hold exactly the rows [q_begin, q_end) of the pack")
+    if scale is None:
+        scale = D ** -0.5
+    if sinks is not None:
+        if sinks.dtype != torch.float32 or not sinks.is_cuda or sinks.numel() != Hq:
+            raise ValueError("sinks must be an fp32 CUDA tensor of Hq values")
+        sinks = sinks.contiguous()
+    if out is None:
+        out = torch.empty((Tq, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty((Tq, Hq), dtype=torch.float32, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        rc = lib.thd_attn_fwd_range(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(),
+            cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), cu.size - 1,
+            int(q_begin), int(q_end), Hq, Hkv, D, int(window), float(scale),
+            sinks.data_ptr() if sinks is not None else None,
+            out.data_ptr(), lse.data_ptr() if lse is not None else None,
+            ctypes.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise ThdAttnError(rc, "thd_attn_fwd_range")
+    return out, lse
+
+
+def thd_attn_plan_range(cu_seqlens, q_begin: int, q_end: int, Hq: int, Hkv: int, D: int,
+                        window: int) -> np.ndarray:
+    """Host-only: the work list of :func:`thd_attn_fwd_range` (structured array)."""
+    lib = load_library()
+    cu = _cu_array(cu_seqlens)
+    n = ctypes.c_int64(0)
+    rc = lib.thd_attn_plan_range(cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), cu.size - 1,
+                                 int(q_begin), int(q_end), Hq, Hkv, D, int(window), None, 0,
+                                 ctypes.byref(n))
+    if rc != 0:
+        raise ThdAttnError(rc, "thd_attn_plan_range")
+    dt = np.dtype([(f, np.int32) for f in WORK_ITEM_FIELDS])
+    items = np.zeros(max(1, n.value), dtype=dt)
+    rc = lib.thd_attn_plan_range(cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), cu.size - 1,
+                                 int(q_begin), int(q_end), Hq, Hkv, D, int(window),
+                                 items.ctypes.data, n.value, ctypes.byref(n))
+    if rc != 0:
+        raise ThdAttnError(rc, "thd_attn_plan_range")
+    return items[:n.value].copy()
 
 
 def thd_attn_get_error(stream=None) -> int:

@@ -51,20 +51,32 @@ int kv_groups_per_chunk(int64_t T, int D, int Hkv) {
 
 std::vector<thd_work_item> build_plan(const int32_t* cu, int n_docs, int Hq, int Hkv, int window,
                                       const KernelShape& ks) {
+    return build_plan_range(cu, n_docs, 0, cu[n_docs], Hq, Hkv, window, ks);
+}
+
+std::vector<thd_work_item> build_plan_range(const int32_t* cu, int n_docs, int64_t q_begin,
+                                            int64_t q_end, int Hq, int Hkv, int window,
+                                            const KernelShape& ks) {
     constexpr int BM = 128;
     const int G = Hq / Hkv;
     const int BN = ks.block_n;
     std::vector<thd_work_item> items;
     size_t n_tiles = 0;
-    for (int d = 0; d < n_docs; ++d) n_tiles += (cu[d + 1] - cu[d] + BM - 1) / BM;
+    for (int d = 0; d < n_docs; ++d) n_tiles += (cu[d + 1] - cu[d] + BM - 1) / BM + 1;
     items.reserve(n_tiles * static_cast<size_t>(Hq / ks.nq));
 
     for (int d = 0; d < n_docs; ++d) {
         const int s = cu[d], e = cu[d + 1];
-        // Query tiles are aligned to the document END, so a ragged tile is the
-        // document's first (shortest key range) rather than its last.
-        for (int q1 = e; q1 > s; q1 -= BM) {
-            const int q0 = q1 - BM;
+        // The document's rows inside the range: [a, b).
+        const int a = static_cast<int>(s > q_begin ? s : q_begin);
+        const int b = static_cast<int>(e < q_end ? e : q_end);
+        // Query tiles are aligned to the END of those rows, so a ragged tile
+        // is the first (shortest key range) rather than the last; a tile that
+        // would reach before a range start q_begin > 0 starts at q_begin
+        // (fewer than 128 rows) so that no row outside the range is loaded.
+        for (int q1 = b; q1 > a; q1 -= BM) {
+            int q0 = q1 - BM;
+            if (q_begin > 0 && q0 < q_begin) q0 = static_cast<int>(q_begin);
             const int r_lo = q0 > s ? q0 : s;
             int k_lo = s;  // lowest key any row of the tile can see
             if (window > 0 && r_lo - window + 1 > k_lo) k_lo = r_lo - window + 1;

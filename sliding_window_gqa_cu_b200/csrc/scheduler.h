@@ -41,6 +41,13 @@ int validate_args(const int32_t* cu_seqlens, int n_docs, int Hq, int Hkv, int D,
 std::vector<thd_work_item> build_plan(const int32_t* cu_seqlens, int n_docs, int Hq, int Hkv,
                                       int window, const KernelShape& ks);
 
+// The same for the query rows [q_begin, q_end) of the pack only (keys from
+// the whole pack): the local step of a context-parallel forward whose rank
+// owns those rows.  build_plan is the range [0, T).
+std::vector<thd_work_item> build_plan_range(const int32_t* cu_seqlens, int n_docs, int64_t q_begin,
+                                            int64_t q_end, int Hq, int Hkv, int window,
+                                            const KernelShape& ks);
+
 // Key-side work list of the backward (dk, dv): one item per (128-key tile of
 // a document, kv head), with the query tiles that see any of its keys; same
 // chunked kv-group order, longest first within a chunk.

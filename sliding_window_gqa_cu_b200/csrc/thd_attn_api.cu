@@ -47,6 +47,7 @@ int variant_index(const KernelShape& ks) {
 struct PlanEntry {
     std::vector<int32_t> cu;
     int Hq, Hkv, D, window;
+    int64_t q_begin, q_end;  // query rows of the pack the plan covers
     thd::WorkItem* d_items = nullptr;
     int64_t n_items = 0;
 };
@@ -103,10 +104,12 @@ int device_state(DeviceState** out, int* dev_out) {
 }
 
 // Finds or builds (and uploads) the plan for these arguments.  Caller holds g_mu.
-int get_plan(DeviceState* ds, const int32_t* cu, int n_docs, int Hq, int Hkv, int D, int window,
-             const KernelShape& ks, cudaStream_t stream, const PlanEntry** out) {
+int get_plan(DeviceState* ds, const int32_t* cu, int n_docs, int64_t q_begin, int64_t q_end, int Hq,
+             int Hkv, int D, int window, const KernelShape& ks, cudaStream_t stream,
+             const PlanEntry** out) {
     for (auto it = ds->plans.begin(); it != ds->plans.end(); ++it) {
         if (it->Hq == Hq && it->Hkv == Hkv && it->D == D && it->window == window &&
+            it->q_begin == q_begin && it->q_end == q_end &&
             it->cu.size() == static_cast<size_t>(n_docs) + 1 &&
             std::memcmp(it->cu.data(), cu, sizeof(int32_t) * (n_docs + 1)) == 0) {
             ds->plans.splice(ds->plans.begin(), ds->plans, it);
@@ -114,9 +117,12 @@ int get_plan(DeviceState* ds, const int32_t* cu, int n_docs, int Hq, int Hkv, in
             return THD_OK;
         }
     }
-    std::vector<thd_work_item> items = thd::build_plan(cu, n_docs, Hq, Hkv, window, ks);
+    std::vector<thd_work_item> items =
+        thd::build_plan_range(cu, n_docs, q_begin, q_end, Hq, Hkv, window, ks);
     PlanEntry e;
     e.cu.assign(cu, cu + n_docs + 1);
+    e.q_begin = q_begin;
+    e.q_end = q_end;
     e.Hq = Hq;
     e.Hkv = Hkv;
     e.D = D;
@@ -305,12 +311,22 @@ const char* thd_attn_status_string(int status) {
 
 int thd_attn_plan(const int32_t* cu_seqlens, int n_docs, int Hq, int Hkv, int D, int window,
                   thd_work_item* items, int64_t capacity, int64_t* n_items) {
+    if (n_docs < 0 || cu_seqlens == nullptr) return THD_ERR_INVALID_ARG;
+    return thd_attn_plan_range(cu_seqlens, n_docs, 0, cu_seqlens[n_docs], Hq, Hkv, D, window,
+                               items, capacity, n_items);
+}
+
+int thd_attn_plan_range(const int32_t* cu_seqlens, int n_docs, int64_t q_begin, int64_t q_end,
+                        int Hq, int Hkv, int D, int window, thd_work_item* items,
+                        int64_t capacity, int64_t* n_items) {
     if (n_items == nullptr || capacity < 0) return THD_ERR_INVALID_ARG;
     int rc = thd::validate_args(cu_seqlens, n_docs, Hq, Hkv, D, window);
     if (rc != THD_OK) return rc;
+    if (q_begin < 0 || q_end < q_begin || q_end > cu_seqlens[n_docs]) return THD_ERR_INVALID_ARG;
     KernelShape ks;
     if (!thd::choose_kernel_shape(D, Hq / Hkv, &ks)) return THD_ERR_UNSUPPORTED;
-    std::vector<thd_work_item> v = thd::build_plan(cu_seqlens, n_docs, Hq, Hkv, window, ks);
+    std::vector<thd_work_item> v =
+        thd::build_plan_range(cu_seqlens, n_docs, q_begin, q_end, Hq, Hkv, window, ks);
     *n_items = static_cast<int64_t>(v.size());
     if (items != nullptr) {
         const int64_t n = std::min<int64_t>(capacity, static_cast<int64_t>(v.size()));
@@ -319,14 +335,16 @@ int thd_attn_plan(const int32_t* cu_seqlens, int n_docs, int Hq, int Hkv, int D,
     return THD_OK;
 }
 
-int thd_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
-                 int n_docs, int Hq, int Hkv, int D, int window, float scale,
-                 const float* sinks_or_null, void* out, float* lse, void* stream_ptr) {
+int thd_attn_fwd_range(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                       int n_docs, int64_t q_begin, int64_t q_end, int Hq, int Hkv, int D,
+                       int window, float scale, const float* sinks_or_null, void* out, float* lse,
+                       void* stream_ptr) {
     int rc = thd::validate_args(cu_seqlens, n_docs, Hq, Hkv, D, window);
     if (rc != THD_OK) return rc;
     if (!(std::isfinite(scale) && scale > 0.0f)) return THD_ERR_INVALID_ARG;
     const int64_t T = cu_seqlens[n_docs];
-    if (T == 0) return THD_OK;
+    if (q_begin < 0 || q_end < q_begin || q_end > T) return THD_ERR_INVALID_ARG;
+    if (T == 0 || q_end == q_begin) return THD_OK;
     if (!q || !k || !v || !out) return THD_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
         return THD_ERR_INVALID_ARG;
@@ -342,13 +360,13 @@ int thd_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_
     rc = device_state(&ds, nullptr);
     if (rc != THD_OK) return rc;
     const PlanEntry* plan = nullptr;
-    rc = get_plan(ds, cu_seqlens, n_docs, Hq, Hkv, D, window, ks, stream, &plan);
+    rc = get_plan(ds, cu_seqlens, n_docs, q_begin, q_end, Hq, Hkv, D, window, ks, stream, &plan);
     if (rc != THD_OK) return rc;
     if (plan->n_items == 0) return THD_OK;
 
     CUtensorMap mq, mk, mv;
     // The pair kernel loads half of each K tile (half the keys) per CTA.
-    if (!make_map(&mq, q, T, Hq, D, 128) ||
+    if (!make_map(&mq, q, q_end - q_begin, Hq, D, 128) ||
         !make_map(&mk, k, T, Hkv, D, ks.pair ? ks.block_n / 2 : ks.block_n) ||
         !make_map(&mv, v, T, Hkv, D, ks.block_n))
         return THD_ERR_CUDA;
@@ -363,6 +381,7 @@ int thd_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_
     prm.G = Hq / Hkv;
     prm.window = window;
     prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.q_offset = static_cast<int>(q_begin);
 
     switch (variant_index(ks)) {
         case 0: return launch<Cfg64x2>(ds, 0, *plan, mq, mk, mv, prm, stream);
@@ -372,6 +391,14 @@ int thd_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_
         case 4: return launch<Cfg256x1>(ds, 4, *plan, mq, mk, mv, prm, stream);
         default: return launch_pair<SplitCfg256>(ds, 5, *plan, mq, mk, mv, prm, stream);
     }
+}
+
+int thd_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                 int n_docs, int Hq, int Hkv, int D, int window, float scale,
+                 const float* sinks_or_null, void* out, float* lse, void* stream_ptr) {
+    if (n_docs < 0 || cu_seqlens == nullptr) return THD_ERR_INVALID_ARG;
+    return thd_attn_fwd_range(q, k, v, cu_seqlens, n_docs, 0, cu_seqlens[n_docs], Hq, Hkv, D,
+                              window, scale, sinks_or_null, out, lse, stream_ptr);
 }
 
 size_t thd_attn_bwd_workspace_bytes(int64_t total_tokens, int Hq) {

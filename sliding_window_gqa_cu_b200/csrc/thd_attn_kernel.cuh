@@ -124,6 +124,7 @@ struct FwdParams {
     int G;               // Hq / Hkv
     int window;
     float scale_log2;    // scale * log2(e)
+    int q_offset;        // pack row of row 0 of q / out / lse (0 unless a token range)
 };
 
 // Wait by lane 0 of the calling warp; the result is broadcast to the warp so
@@ -238,7 +239,7 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
             for (int q = 0; q < C::NQ; ++q)
                 for (int c = 0; c < C::KCH; ++c)
                     tma_load_3d(sbase + C::SMEM_Q + q * C::Q_TILE_BYTES + c * C::Q_BOX_BYTES,
-                                &tmap_q, bar(C::B_Q_FULL), c * 64, it.head0 + q, it.q0);
+                                &tmap_q, bar(C::B_Q_FULL), c * 64, it.head0 + q, it.q0 - p.q_offset);
             // Ring positions: 2j holds K(j), 2j+1 holds V(j); position p uses
             // slot p % NSLOT.  A load waits only for the slot's previous tile.
             int issued = 0;
@@ -478,7 +479,7 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         if (ok) {
             tc_fence_after();
             const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
-            __nv_bfloat16* orow = p.out + (static_cast<int64_t>(i) * p.Hq + h) * C::D;
+            __nv_bfloat16* orow = p.out + (static_cast<int64_t>(i - p.q_offset) * p.Hq + h) * C::D;
 #pragma unroll 1
             for (int c = 0; c < C::D / 32; ++c) {
                 uint32_t r[32];
@@ -498,7 +499,7 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 }
             }
             if (row_valid && p.lse != nullptr)
-                p.lse[static_cast<int64_t>(i) * p.Hq + h] =
+                p.lse[static_cast<int64_t>(i - p.q_offset) * p.Hq + h] =
                     l > 0.0f ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
         }
     }

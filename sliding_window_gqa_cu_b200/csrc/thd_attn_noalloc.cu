@@ -241,6 +241,7 @@ extern "C" int thd_attn_fwd_noalloc(const void* q, const void* k, const void* v,
     prm.G = Hq / Hkv;
     prm.window = window;
     prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.q_offset = 0;
 
     if (ks.pair) return launch_pair<NSplitCfg256>(st, 5, n_items, mq, mk, mv, prm, stream);
     if (D == 64) {

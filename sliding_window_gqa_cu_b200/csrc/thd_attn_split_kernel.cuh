@@ -170,7 +170,7 @@ thd_attn_fwd_split_kernel(const __grid_constant__ CUtensorMap tmap_q,
             if (leader) mbar_arrive_expect_tx(bar(C::B_Q_FULL), 2 * C::Q_TILE_BYTES);
             for (int c = 0; c < C::KCH; ++c)
                 tma_load_3d_pair(sbase + C::SMEM_Q + c * C::Q_BOX_BYTES, &tmap_q,
-                                 lead_bar(C::B_Q_FULL), c * 64, head, it.q0);
+                                 lead_bar(C::B_Q_FULL), c * 64, head, it.q0 - p.q_offset);
             // Ring positions: 2j holds K(j), 2j+1 holds V(j).  This CTA loads
             // keys [rank*BN/2, (rank+1)*BN/2) of K(j) and head-dim columns
             // [rank*D/2, (rank+1)*D/2) of V(j).
@@ -422,7 +422,7 @@ thd_attn_fwd_split_kernel(const __grid_constant__ CUtensorMap tmap_q,
             tc_fence_after();
             const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
             __nv_bfloat16* orow =
-                p.out + (static_cast<int64_t>(i) * p.Hq + head) * C::D + h * O_COLS;
+                p.out + (static_cast<int64_t>(i - p.q_offset) * p.Hq + head) * C::D + h * O_COLS;
 #pragma unroll 1
             for (int c = 0; c < O_COLS / 32; ++c) {
                 uint32_t r[32];
@@ -442,7 +442,7 @@ thd_attn_fwd_split_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 }
             }
             if (h == 0 && row_valid && p.lse != nullptr)
-                p.lse[static_cast<int64_t>(i) * p.Hq + head] =
+                p.lse[static_cast<int64_t>(i - p.q_offset) * p.Hq + head] =
                     l > 0.0f ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
         }
     }

@@ -6,10 +6,11 @@
 // place on the packed THD q [T, Hq, D] and k [T, Hkv, D].  Positions are the
 // caller's, or each token's offset inside its own document.
 //
-// One CTA per token: its D/2 (cos, sin) pairs are computed once into shared
-// memory and shared by all Hq + Hkv heads of the token; one warp per head
-// vector (a lane holds D/32 consecutive elements, so the split-half partner
-// of lane l is lane l ^ 16).  Memory bound: each element is read and written
+// One warp per token: a lane holds D/32 consecutive elements of a head
+// vector (so the split-half partner of lane l is lane l ^ 16) and computes
+// the cos / sin of its own D/32 frequencies once, for all Hq + Hkv head
+// vectors of the token; the warp loads four head vectors before it
+// transforms any of them, to keep enough loads in flight.  Memory bound: each element is read and written
 // once (16-bit loads and stores vectorised to 4, 8 or 16 bytes per lane).
 // The angle is reduced modulo 2 pi in double precision before the fp32
 // sine / cosine, so positions up to 2^31 keep full fp32 accuracy; everything
@@ -45,92 +46,100 @@ struct PrologueParams {
 template <int D>
 __global__ void __launch_bounds__(256) thd_qk_norm_rope_kernel(const PrologueParams p) {
     constexpr int E = D / 32;  // elements per lane
-    __shared__ float cs[D / 2], sn[D / 2];
-    __shared__ int s_pos;
-    const int64_t t = blockIdx.x;
+    constexpr int R = 4;       // head vectors loaded per warp before any is transformed
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
+    if (t >= p.T) return;
+    // cos / sin of this lane's E frequencies k = E (lane % 16) + e, shared by
+    // all head vectors of the token (lane l and l ^ 16 hold a split-half pair).
+    float cs[E], sn[E];
     if (p.rope) {
-        if (threadIdx.x == 0) {
-            int pos;
-            if (p.positions != nullptr) {
-                pos = p.positions[t];
-            } else {  // last document starting at or before t
-                int lo = 0, hi = p.n_docs - 1;
-                while (lo < hi) {
-                    const int mid = (lo + hi + 1) >> 1;
-                    if (p.cu[mid] <= t) lo = mid; else hi = mid - 1;
-                }
-                pos = static_cast<int>(t - p.cu[lo]);
+        int pos;
+        if (p.positions != nullptr) {
+            pos = p.positions[t];
+        } else {  // last document starting at or before t
+            int lo = 0, hi = p.n_docs - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (p.cu[mid] <= t) lo = mid; else hi = mid - 1;
             }
-            s_pos = pos;
+            pos = static_cast<int>(t - p.cu[lo]);
         }
-        __syncthreads();
-        for (int kk = threadIdx.x; kk < D / 2; kk += blockDim.x) {
+        const int k0 = E * (lane & 15);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
             constexpr double kTwoPi = 6.283185307179586476925286766559;
-            double a = static_cast<double>(s_pos) * p.inv_freq[kk];
+            double a = static_cast<double>(pos) * p.inv_freq[k0 + e];
             a -= kTwoPi * rint(a * (1.0 / kTwoPi));
-            float sv, cv;
-            sincosf(static_cast<float>(a), &sv, &cv);
-            cs[kk] = cv;
-            sn[kk] = sv;
+            sincosf(static_cast<float>(a), &sn[e], &cs[e]);
         }
-        __syncthreads();
     }
+    const bool second = lane >= 16;
     const int rows = p.Hq + p.Hkv;
-    for (int r = warp; r < rows; r += blockDim.x >> 5) {
-        __nv_bfloat16* row = r < p.Hq ? p.q + (t * p.Hq + r) * D : p.k + (t * p.Hkv + (r - p.Hq)) * D;
-        __nv_bfloat16* mine = row + lane * E;
-        uint32_t w[E / 2];
-        if constexpr (E == 8) {
-            const uint4 x = *reinterpret_cast<const uint4*>(mine);
-            w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
-        } else if constexpr (E == 4) {
-            const uint2 x = *reinterpret_cast<const uint2*>(mine);
-            w[0] = x.x; w[1] = x.y;
-        } else {
-            w[0] = *reinterpret_cast<const uint32_t*>(mine);
-        }
-        float v[E];
+    for (int r0 = 0; r0 < rows; r0 += R) {
+        uint32_t w[R][E / 2];
+        __nv_bfloat16* mine[R];
 #pragma unroll
-        for (int u = 0; u < E / 2; ++u) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[u]));
-            v[2 * u] = f.x;
-            v[2 * u + 1] = f.y;
-        }
-        float ss = 0.0f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) ss = fmaf(v[e], v[e], ss);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-        const float inv = 1.0f / sqrtf(ss * (1.0f / D) + p.eps);
-#pragma unroll
-        for (int e = 0; e < E; ++e) v[e] *= inv;
-        if (p.rope) {
-            // Lane l < 16 holds elements of the first half, lane l + 16 their
-            // partners k + D/2 (E * 16 = D / 2).
-            const int k0 = E * (lane & 15);
-            const bool second = lane >= 16;
-            float o[E];
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-                const float partner = __shfl_xor_sync(0xffffffffu, v[e], 16);
-                const float c = cs[k0 + e], s = sn[k0 + e];
-                o[e] = second ? fmaf(v[e], c, partner * s) : fmaf(v[e], c, -partner * s);
+        for (int i = 0; i < R; ++i) {
+            const int r = r0 + i;
+            mine[i] = nullptr;
+            if (r < rows) {
+                __nv_bfloat16* row = r < p.Hq ? p.q + (t * p.Hq + r) * D
+                                              : p.k + (t * p.Hkv + (r - p.Hq)) * D;
+                mine[i] = row + lane * E;
+                if constexpr (E == 8) {
+                    const uint4 x = *reinterpret_cast<const uint4*>(mine[i]);
+                    w[i][0] = x.x; w[i][1] = x.y; w[i][2] = x.z; w[i][3] = x.w;
+                } else if constexpr (E == 4) {
+                    const uint2 x = *reinterpret_cast<const uint2*>(mine[i]);
+                    w[i][0] = x.x; w[i][1] = x.y;
+                } else {
+                    w[i][0] = *reinterpret_cast<const uint32_t*>(mine[i]);
+                }
             }
-#pragma unroll
-            for (int e = 0; e < E; ++e) v[e] = o[e];
         }
 #pragma unroll
-        for (int u = 0; u < E / 2; ++u) {
-            const __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * u], v[2 * u + 1]);
-            w[u] = *reinterpret_cast<const uint32_t*>(&b);
-        }
-        if constexpr (E == 8) {
-            *reinterpret_cast<uint4*>(mine) = make_uint4(w[0], w[1], w[2], w[3]);
-        } else if constexpr (E == 4) {
-            *reinterpret_cast<uint2*>(mine) = make_uint2(w[0], w[1]);
-        } else {
-            *reinterpret_cast<uint32_t*>(mine) = w[0];
+        for (int i = 0; i < R; ++i) {
+            if (r0 + i >= rows) break;  // warp-uniform
+            float v[E];
+#pragma unroll
+            for (int u = 0; u < E / 2; ++u) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i][u]));
+                v[2 * u] = f.x;
+                v[2 * u + 1] = f.y;
+            }
+            float ss = 0.0f;
+#pragma unroll
+            for (int e = 0; e < E; ++e) ss = fmaf(v[e], v[e], ss);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+            const float inv = 1.0f / sqrtf(ss * (1.0f / D) + p.eps);
+#pragma unroll
+            for (int e = 0; e < E; ++e) v[e] *= inv;
+            if (p.rope) {
+                float o[E];
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const float partner = __shfl_xor_sync(0xffffffffu, v[e], 16);
+                    o[e] = second ? fmaf(v[e], cs[e], partner * sn[e])
+                                  : fmaf(v[e], cs[e], -partner * sn[e]);
+                }
+#pragma unroll
+                for (int e = 0; e < E; ++e) v[e] = o[e];
+            }
+            uint32_t ow[E / 2];
+#pragma unroll
+            for (int u = 0; u < E / 2; ++u) {
+                const __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * u], v[2 * u + 1]);
+                ow[u] = *reinterpret_cast<const uint32_t*>(&b);
+            }
+            if constexpr (E == 8) {
+                *reinterpret_cast<uint4*>(mine[i]) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+            } else if constexpr (E == 4) {
+                *reinterpret_cast<uint2*>(mine[i]) = make_uint2(ow[0], ow[1]);
+            } else {
+                *reinterpret_cast<uint32_t*>(mine[i]) = ow[0];
+            }
         }
     }
 }
@@ -212,7 +221,7 @@ extern "C" int thd_qk_norm_rope(void* q, void* k, const int32_t* cu_seqlens, int
         int rc = device_cu(cu_seqlens, n_docs, stream, &p.cu);
         if (rc != THD_OK) return rc;
     }
-    const unsigned grid = static_cast<unsigned>(T);
+    const unsigned grid = static_cast<unsigned>((T + 7) / 8);  // 8 warps (tokens) per CTA
     switch (D) {
         case 64: thd_qk_norm_rope_kernel<64><<<grid, 256, 0, stream>>>(p); break;
         case 128: thd_qk_norm_rope_kernel<128><<<grid, 256, 0, stream>>>(p); break;

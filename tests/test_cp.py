@@ -1,0 +1,103 @@
+"""Context-parallel forward, host side (CPU): the token shards, the K/V
+all-gather over a world-size-2 gloo group, and the range schedule of each
+rank's local step (every row of the shard owned exactly once, no row outside
+it, every visible key in its items' key tiles), checked by brute force
+against the window definition of FlintMagiPlan.attention ("flint.magi"
+page)."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import sliding_window_gqa_cu_b200 as swa
+from sliding_window_gqa_cu_b200 import build, cp, multirank, workloads
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    swa.load_library()
+
+
+@pytest.mark.parametrize("T,world", [(10, 3), (2, 4), (65536, 8), (1, 1), (129, 2)])
+def test_shard_bounds_partition_the_pack(T, world):
+    b = cp.shard_bounds(T, world)
+    assert len(b) == world and b[0][0] == 0 and b[-1][1] == T
+    assert all(b[r][1] == b[r + 1][0] for r in range(world - 1))
+    assert all(0 <= e - s <= -(-T // world) for s, e in b)
+
+
+def check_range_plan(cu, qb, qe, Hq, Hkv, D, window):
+    plan = swa.thd_attn_plan_range(cu, qb, qe, Hq, Hkv, D, window)
+    cu = np.asarray(cu)
+    T, G = int(cu[-1]), Hq // Hkv
+    owner = np.full((T, Hq), -1)
+    for idx, it in enumerate(plan):
+        q0, q1, s, h0 = int(it["q0"]), int(it["q1"]), int(it["doc_start"]), int(it["head0"])
+        ks, nkv, nh, bn = int(it["kv_start"]), int(it["n_kv"]), int(it["n_heads"]), int(it["block_n"])
+        assert 0 < q1 - q0 <= 128 and q1 <= qe and (q0 >= qb or qb == 0)
+        assert ks + nkv * bn == q1
+        d = int(np.searchsorted(cu, s, side="right") - 1)
+        while cu[d + 1] == cu[d]:
+            d += 1
+        e = int(cu[d + 1])
+        rows = range(max(q0, s, qb), q1)
+        for h in range(h0, h0 + nh):
+            for i in rows:
+                assert owner[i, h] == -1
+                owner[i, h] = idx
+        for i in rows:
+            lo = s if window == 0 else max(s, i - window + 1)
+            assert ks <= lo and i < ks + nkv * bn and i < e
+    assert (owner[qb:qe] >= 0).all(), "a row of the shard is not covered"
+    assert (owner[:qb] < 0).all() and (owner[qe:] < 0).all(), "a row outside the shard is covered"
+
+
+@pytest.mark.parametrize("lens,Hq,Hkv,D,window,world", [
+    ([300, 1, 0, 129, 77], 4, 2, 128, 0, 2),
+    ([300, 1, 0, 129, 77], 4, 2, 128, 100, 3),
+    ([700, 256, 3], 6, 2, 128, 128, 4),
+    ([1000, 33], 16, 1, 256, 129, 3),
+    ([513], 2, 2, 64, 1, 5),
+])
+def test_range_plans_cover_each_shard_exactly(lens, Hq, Hkv, D, window, world):
+    cu = workloads.cu_seqlens_from_lengths(lens)
+    for qb, qe in cp.shard_bounds(int(cu[-1]), world):
+        check_range_plan(cu, qb, qe, Hq, Hkv, D, window)
+
+
+def test_full_range_plan_is_the_forward_plan():
+    cu = workloads.cu_seqlens_from_lengths([300, 1, 0, 129, 77])
+    a = swa.thd_attn_plan(cu, 8, 2, 128, 0)
+    b = swa.thd_attn_plan_range(cu, 0, int(cu[-1]), 8, 2, 128, 0)
+    assert np.array_equal(a, b)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, result_dir):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    multirank.init("gloo", timeout_s=60)
+    p = workloads.random_pack(5, [300, 1, 0, 129, 78], 4, 2, 64, 0, 0.125, False)
+    T = int(p["T"])
+    b, e = cp.shard_bounds(T, world)[rank]
+    k, v = p["k"].float(), p["v"].float()
+    kf, vf = cp.gather_kv(k[b:e].contiguous(), v[b:e].contiguous(), T)
+    ok = torch.equal(kf, k) and torch.equal(vf, v)
+    with open(os.path.join(result_dir, f"r{rank}.txt"), "w") as f:
+        f.write("ok" if ok else "mismatch")
+    multirank.shutdown()
+
+
+def test_two_rank_gloo_kv_all_gather(tmp_path):
+    port = _free_port()
+    mp.spawn(_worker, args=(2, port, str(tmp_path)), nprocs=2, join=True)
+    assert [open(tmp_path / f"r{r}.txt").read() for r in range(2)] == ["ok", "ok"]
