@@ -14,6 +14,8 @@ Two independent formulations live here:
   same C file;
 * :mod:`oracle.prologue` -- the Q/K prologue (scaleless RMSNorm, then
   split-half RoPE at per-document positions) in plain fp64 numpy;
+* :mod:`oracle.sparse_mla` -- sparse MLA over gathered latent KV with the
+  absorbed value projection, fp64 numpy;
 * :func:`dense_attention` -- a dense brute force for tiny packs: it builds the
   boolean ``[query_tokens, key_tokens]`` causal document mask the way
   ``SequenceLayout.allowed`` is described ("mistral_large4.attention" page),
