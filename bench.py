@@ -11,8 +11,11 @@ TFLOP/s over valid (unmasked) query-key pairs, FLOP = 4 * pairs * D * Hq.
 ``--pass bwd`` times the backward (thd_attn_bwd: dq, dk, dv, dsink) on the
 same pack instead, FLOP = 2.5x the forward's (the usual count of a backward
 that recomputes P); ``--pass prologue`` times the in-place Q/K prologue
-(thd_qk_norm_rope), bytes = Q and K read and written once.  Both print one
-JSON line of the same shape with their own metric.
+(thd_qk_norm_rope), bytes = Q and K read and written once; ``--pass
+sparse_mla`` times sparse MLA (thd_sparse_mla_fwd) on its own synthetic
+workload (4,096 tokens, 128 heads, up to 2,048 selected keys, value dim
+128), FLOP = valid slots x heads x 2 x (576 + 512) + the value projection.
+Each prints one JSON line of the same shape with its own metric.
 
 Prints one JSON line on stdout (rank 0).  Multi-GPU runs are launched with
 torchrun, one process per GPU; every rank runs its own pack of the same shape
@@ -72,8 +75,8 @@ def parse_args(argv=None):
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd", "prologue"], default="fwd",
-                    help="what one step runs (default: the forward, the headline)")
+    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd", "prologue", "sparse_mla"],
+                    default="fwd", help="what one step runs (default: the forward, the headline)")
     return ap.parse_args(argv)
 
 
@@ -406,6 +409,8 @@ def run_other_pass(args, info):
     device = torch.device("cuda", info.local_rank)
     torch.cuda.set_device(device)
     swa.load_library()
+    if args.pass_ == "sparse_mla":
+        return run_sparse_mla(args, info, device)
     cfg = workloads.CONFIGS[args.workload]
     pack = workloads.make_pack(cfg, args.seed, tensor_seed=multirank.tensor_seed(args.seed, info.rank),
                                T_override=args.tokens)
@@ -479,6 +484,73 @@ def run_other_pass(args, info):
             "clocks": {k: csum[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
         }
         log(f"[bench] {cfg.name} {args.pass_}: {ms / args.steps:.3f} ms/step, {value:.1f} {unit} "
+            f"({100 * achieved / peak:.1f}% of measured {peak:.0f}), clocks {csum}")
+        print(json.dumps(line), flush=True)
+    multirank.shutdown()
+    return 0
+
+
+SPARSE_MLA_WORKLOAD = dict(name="sparse_mla_t4096_h128_k2048_v128", lens=[4096], H=128, K=2048, vd=128)
+
+
+def run_sparse_mla(args, info, device):
+    """--pass sparse_mla: device-timed thd_sparse_mla_fwd (attention + value
+    projection, two launches) on a synthetic one-document workload."""
+    import sliding_window_gqa_cu_b200 as swa
+
+    w = SPARSE_MLA_WORKLOAD
+    c = workloads.sparse_mla_case(args.seed + 7919 * info.rank, w["lens"], w["H"], w["K"], w["vd"])
+    q, kv, idx, wt = (c[n].to(device) for n in ("q", "kv", "indices", "value_weight"))
+    T, H, vd = c["T"], w["H"], w["vd"]
+    valid = int((c["indices"] >= 0).sum())
+    flop = valid * H * 2 * (576 + 512) + T * H * 512 * vd * 2
+    out = torch.empty((T, H, vd), dtype=torch.bfloat16, device=device)
+    ws = torch.empty((swa.thd_sparse_mla_workspace_bytes(T, H),), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        swa.thd_sparse_mla_fwd(q, kv, idx, wt, c["scale"], out=out, workspace=ws, stream=stream)
+    step()
+    if swa.thd_sparse_mla_get_error(stream) != 0:
+        raise RuntimeError("kernel reported an error status")
+    clocks = ClockSampler(device)
+    for _ in range(args.warmup):
+        step()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    multirank.barrier(device)
+    torch.cuda.synchronize(device)
+    h0 = time.time()
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    h1 = time.time()
+    multirank.barrier(device)
+    clocks.stop()
+    ms = multirank.max_over_ranks(start.elapsed_time(end), device)
+    value = multirank.aggregate_rate(flop * args.steps, info.world, ms / 1e3) / 1e12
+    achieved = flop / (ms / args.steps / 1e3) / 1e12
+    peaks, peak_src = measured_peaks()
+    peak = float(peaks["bf16_tflops"])
+    csum = clocks.summary(h0, h1)
+    if info.is_root:
+        line = {
+            "metric": "sparse MLA fwd TFLOP/s (valid slots, incl. value projection)", "value": value,
+            "unit": "TFLOP/s", "n_gpus": info.world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "pass": "sparse_mla",
+            "config": {"workload": w["name"], "tokens": T, "heads": H, "selected_keys": w["K"],
+                       "value_dim": vd, "valid_slots": valid,
+                       "l2": "inputs larger than L2 (q = %.2f GB), no flush" % (T * H * 576 * 2 / 1e9)},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "kernel": "thd_sparse_mla_attn_kernel + thd_sparse_mla_proj_kernel",
+                         "peak_source": f"{peak_src} (MEASURED_PEAKS.json)"},
+            "cpu_baseline": None, "e2e": None, "gpu_launches": 2 * args.steps,
+            "clocks": {k: csum[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+        }
+        log(f"[bench] {w['name']}: {ms / args.steps:.3f} ms/step, {value:.1f} TFLOP/s "
             f"({100 * achieved / peak:.1f}% of measured {peak:.0f}), clocks {csum}")
         print(json.dumps(line), flush=True)
     multirank.shutdown()

@@ -284,6 +284,35 @@ int thd_qk_norm_rope(void* q, void* k, const int32_t* cu_seqlens, int n_docs,
                      const int32_t* positions_or_null, int Hq, int Hkv, int D,
                      float eps, float theta, int apply_rope, void* stream);
 
+/*
+ * ---------------------------------------------------------------- sparse MLA
+ * Sparse MLA forward ("mistral_large4.attention" page, sparse_mla): for
+ * token t and head h, with the valid slots j (0 <= indices[t, j] < Tg; -1 or
+ * anything out of range is an invalid slot, ignored),
+ *   s_j = scale * <q[t, h, :], kv[indices[t, j], :]>   (576-wide),
+ *   latent = sum_j softmax(s)_j kv[indices[t, j], :512],
+ *   out[t, h, :] = value_weight[h] @ latent;  a row with no valid slot is zero.
+ *   q             bf16 device [T, H, 576] (absorbed queries, last 64 rotary)
+ *   kv            bf16 device [Tg, 576] (latent 512 + rotary 64 per key)
+ *   indices       int32 device [T, K] (the caller applies document / causal
+ *                 boundaries; each valid slot counts once, as given)
+ *   value_weight  bf16 device [H, value_dim, 512]
+ *   out           bf16 device [T, H, value_dim], written
+ *   workspace     device scratch >= thd_sparse_mla_workspace_bytes(T, H)
+ *                 (the bf16 latent [T, H, 512]), 16-byte aligned
+ * Supported: H a multiple of 128, K a multiple of 64 (pad with -1),
+ * value_dim 64, 128 or 256 (else THD_ERR_UNSUPPORTED).  Argument errors
+ * return before anything is enqueued; kernel stalls are reported by
+ * thd_sparse_mla_get_error.
+ */
+size_t thd_sparse_mla_workspace_bytes(int64_t T, int H);
+int thd_sparse_mla_fwd(const void* q, const void* kv, const int32_t* indices,
+                       const void* value_weight, int64_t T, int64_t Tg, int H, int K,
+                       int value_dim, float scale, void* out,
+                       void* workspace, size_t workspace_bytes, void* stream);
+/* Synchronises the stream; returns and clears the sparse-MLA status word. */
+int thd_sparse_mla_get_error(void* stream);
+
 /* ABI version of this header: (major << 16) | minor. */
 int thd_attn_abi_version(void);
 

@@ -86,6 +86,13 @@ def load_library():
                                         c_int, c_int, vp, ctypes.c_int64,
                                         ctypes.POINTER(ctypes.c_int64)]
     lib.thd_attn_plan_range.restype = c_int
+    lib.thd_sparse_mla_workspace_bytes.argtypes = [ctypes.c_int64, c_int]
+    lib.thd_sparse_mla_workspace_bytes.restype = ctypes.c_size_t
+    lib.thd_sparse_mla_fwd.argtypes = [vp, vp, vp, vp, ctypes.c_int64, ctypes.c_int64, c_int, c_int,
+                                       c_int, ctypes.c_float, vp, vp, ctypes.c_size_t, vp]
+    lib.thd_sparse_mla_fwd.restype = c_int
+    lib.thd_sparse_mla_get_error.argtypes = [vp]
+    lib.thd_sparse_mla_get_error.restype = c_int
     lib.thd_qk_norm_rope.argtypes = [vp, vp, i32p, c_int, vp, c_int, c_int, c_int, ctypes.c_float,
                                      ctypes.c_float, c_int, vp]
     lib.thd_qk_norm_rope.restype = c_int
@@ -353,6 +360,54 @@ def thd_attn_plan_range(cu_seqlens, q_begin: int, q_end: int, Hq: int, Hkv: int,
     if rc != 0:
         raise ThdAttnError(rc, "thd_attn_plan_range")
     return items[:n.value].copy()
+
+
+def thd_sparse_mla_fwd(q, kv, indices, value_weight, scale: float, out=None, workspace=None,
+                       stream=None):
+    """Sparse MLA forward.  q: bf16 CUDA [T, H, 576]; kv: bf16 CUDA [Tg, 576];
+    indices: int32 CUDA [T, K] (-1 = invalid slot); value_weight: bf16 CUDA
+    [H, value_dim, 512].  Returns out: bf16 [T, H, value_dim]."""
+    import torch
+
+    lib = load_library()
+    T, H, dq = q.shape
+    Tg = kv.shape[0]
+    K = indices.shape[1] if indices.dim() == 2 else 0
+    vd = value_weight.shape[1]
+    for name, t, dt in (("q", q, torch.bfloat16), ("kv", kv, torch.bfloat16),
+                        ("indices", indices, torch.int32), ("value_weight", value_weight, torch.bfloat16)):
+        if t.dtype != dt or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous {dt} CUDA tensor")
+    if dq != 576 or kv.shape[1] != 576 or indices.shape[0] != T or value_weight.shape != (H, vd, 512):
+        raise ValueError("shapes: q [T, H, 576], kv [Tg, 576], indices [T, K], value_weight [H, vd, 512]")
+    if out is None:
+        out = torch.empty((T, H, vd), dtype=torch.bfloat16, device=q.device)
+    need = int(lib.thd_sparse_mla_workspace_bytes(T, H))
+    if workspace is None:
+        workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        rc = lib.thd_sparse_mla_fwd(q.data_ptr(), kv.data_ptr(), indices.data_ptr(),
+                                    value_weight.data_ptr(), T, Tg, H, K, vd, float(scale),
+                                    out.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                    ctypes.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise ThdAttnError(rc, "thd_sparse_mla_fwd")
+    return out
+
+
+def thd_sparse_mla_workspace_bytes(T: int, H: int) -> int:
+    """Workspace bytes :func:`thd_sparse_mla_fwd` needs (the bf16 latent [T, H, 512])."""
+    return int(load_library().thd_sparse_mla_workspace_bytes(int(T), int(H)))
+
+
+def thd_sparse_mla_get_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the sparse-MLA status word."""
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(load_library().thd_sparse_mla_get_error(ctypes.c_void_p(stream.cuda_stream)))
 
 
 def thd_attn_get_error(stream=None) -> int:

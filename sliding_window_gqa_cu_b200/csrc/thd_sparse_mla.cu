@@ -1,0 +1,562 @@
+// Sparse MLA forward ("mistral_large4.attention" page, sparse_mla) on B200.
+//
+// For token t and head h: s_j = scale * <q[t, h, :576], kv[idx[t, j], :576]>
+// over the valid index slots j (idx >= 0), p = softmax(s), latent =
+// sum_j p_j kv[idx[t, j], :512], out[t, h, :] = value_weight[h] @ latent.
+// A row without a valid slot is zero.  Two kernels:
+//
+// 1. Attention (thd_sparse_mla_attn_kernel): one CTA per (token, group of
+//    128 heads, quarter of the 512 latent columns).  The 128 query rows of
+//    the token (128 x 576 bf16) sit in TMEM as the A operand; the selected
+//    kv rows are gathered 64 at a time by a producer warpgroup (16-byte
+//    cp.async copies into the 128-byte-swizzled layout the tensor core
+//    reads), so one shared-memory tile serves S = Q kv^T (K-major operand)
+//    and latent += P kv[:, quarter] (MN-major operand).  TMEM: Q 288
+//    columns + S / P 64 + the latent quarter 128 = 480 of 512, which is why
+//    the latent is split over four CTAs (each recomputes S: QK^T runs four
+//    times per token; see the design notes).  Online softmax as in the
+//    attention forward (exp2 domain, lazy rescale).  Writes the normalised
+//    latent (bf16) to a workspace [T, H, 512].
+// 2. Projection (thd_sparse_mla_proj_kernel): per head a GEMM
+//    out[:, h, :] = latent[:, h, :] @ value_weight[h]^T, one CTA per
+//    (128-token tile, head), TMA-fed tcgen05 MMAs with K = 512.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "../../include/thd_attn.h"
+#include "sm100_ptx.cuh"
+#include "thd_attn_kernel.cuh"
+#include "tma_map.h"
+
+namespace {
+
+using thd::kStatusTimeout;
+
+// --------------------------------------------------------- cp.async gather --
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+struct SmlaParams {
+    const __nv_bfloat16* q;    // [T, H, 576]
+    const __nv_bfloat16* kv;   // [Tg, 576]
+    const int32_t* idx;        // [T, K]
+    __nv_bfloat16* latent;     // [T, H, 512] (workspace)
+    int* status;
+    int64_t T, Tg;
+    int H, K;
+    float scale_log2;
+};
+
+constexpr int kQDim = 576, kLat = 512;
+constexpr int kBN = 64;             // selected keys per chunk
+constexpr int kNST = 3;             // chunk stages
+constexpr int kChunkBytes = kBN * 128;           // one 64-column chunk of a 64-row tile
+constexpr int kStageBytes = 9 * kChunkBytes;     // 64 rows x 576 columns
+constexpr int kTmQ = 0, kTmS = 288, kTmO = 352;  // TMEM columns
+constexpr int B_Q_READY = 0, B_FULL = 1, B_EMPTY = B_FULL + kNST, B_S_FULL = B_EMPTY + kNST,
+              B_P_FULL = B_S_FULL + 1, B_O_FULL = B_P_FULL + 1, B_DRAIN = B_O_FULL + 1,
+              kNumBars = B_DRAIN + 1;
+constexpr int kSmemBias = kNST * kStageBytes;               // float [kNST][64]
+constexpr int kSmemBar = kSmemBias + kNST * kBN * 4;
+constexpr int kSmemTmem = kSmemBar + kNumBars * 8;
+constexpr int kSmemAbort = kSmemTmem + 4;
+constexpr int kSmemAlloc = kSmemAbort + 4 + 1024;
+static_assert(kSmemAlloc <= 232448, "shared memory budget exceeded");
+static_assert(kTmO + 128 <= 512, "TMEM budget exceeded");
+
+__global__ void __launch_bounds__(288, 1) thd_sparse_mla_attn_kernel(const SmlaParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = thd::smem_addr(smem_raw);
+    uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
+    const uint32_t sbase = thd::smem_addr(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int quarter = blockIdx.x & 3;
+    const int hgroups = p.H / 128;
+    const int hg = (blockIdx.x >> 2) % hgroups;
+    const int64_t t = (blockIdx.x >> 2) / hgroups;
+    const int nch = p.K / kBN;
+
+    auto bar = [&](int i) -> uint32_t { return sbase + kSmemBar + 8u * i; };
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSmemAbort);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kSmemTmem);
+    float* bias = reinterpret_cast<float*>(smem + kSmemBias);
+
+    if (threadIdx.x == 0) {
+        thd::mbar_init(bar(B_Q_READY), 4);
+        for (int s = 0; s < kNST; ++s) {
+            thd::mbar_init(bar(B_FULL + s), 4);  // the four producer warps
+            thd::mbar_init(bar(B_EMPTY + s), 1);
+        }
+        thd::mbar_init(bar(B_S_FULL), 1);
+        thd::mbar_init(bar(B_P_FULL), 4);
+        thd::mbar_init(bar(B_O_FULL), 1);
+        thd::mbar_init(bar(B_DRAIN), 1);
+        *abort_flag = *reinterpret_cast<volatile int*>(p.status) != 0 ? 1 : 0;
+        thd::fence_barrier_init();
+    }
+    if (warp == 8) {
+        thd::tmem_alloc(thd::smem_addr(tmem_slot), 512);
+        thd::tmem_relinquish();
+    }
+    thd::tc_fence_before();
+    __syncthreads();
+    thd::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const bool skip = *abort_flag != 0;
+
+    if (warp >= 4 && warp < 8) {
+        // ---------------------------------------------- gather producer (128)
+        const int pt = threadIdx.x - 128;
+        const int32_t* irow = p.idx + t * p.K;
+        bool ok = !skip;
+        for (int c = 0; ok && c <= nch; ++c) {
+            if (c < nch) {
+                const int s = c % kNST;
+                ok = thd::warp_wait(bar(B_EMPTY + s), ((c / kNST) & 1) ^ 1, abort_flag, p.status);
+                if (!ok) break;
+                const uint32_t stage = sbase + s * kStageBytes;
+                for (int u = pt; u < kBN * 72; u += 128) {
+                    const int r = u / 72, uu = u % 72;
+                    const int gi = irow[c * kBN + r];
+                    const int64_t row = (gi >= 0 && gi < p.Tg) ? gi : 0;
+                    const uint32_t dst = stage + (uu >> 3) * kChunkBytes + r * 128 +
+                                         ((static_cast<uint32_t>(uu & 7) ^ static_cast<uint32_t>(r & 7)) << 4);
+                    cp_async16(dst, p.kv + row * kQDim + uu * 8);
+                }
+                if (pt < kBN) {
+                    const int gi = irow[c * kBN + pt];
+                    bias[s * kBN + pt] = (gi >= 0 && gi < p.Tg) ? 0.0f : -INFINITY;
+                }
+                cp_async_commit();
+            }
+            // Chunk c - 1 (this thread's copies) complete: publish it.
+            if (c >= 1) {
+                if (c < nch) cp_async_wait<1>(); else cp_async_wait<0>();
+                thd::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) thd::mbar_arrive(bar(B_FULL + (c - 1) % kNST));
+            }
+        }
+        if (!ok) cp_async_wait<0>();
+        __syncwarp();
+    } else if (warp == 8) {
+        // ------------------------------------------------------- MMA issuer
+        if (lane == 0 && !skip) {
+            constexpr uint32_t idesc_s = thd::idesc_bf16_f32(128, kBN, false);
+            constexpr uint32_t idesc_o = thd::idesc_bf16_f32(128, 128, true);
+            auto wait = [&](int i, uint32_t par) -> bool {
+                return thd::mbar_wait(bar(i), par, abort_flag, p.status, kStatusTimeout);
+            };
+            bool ok = wait(B_Q_READY, 0);
+            for (int c = 0; ok && c < nch; ++c) {
+                const int s = c % kNST;
+                ok = wait(B_FULL + s, (c / kNST) & 1);
+                if (!ok) break;
+                thd::tc_fence_after();
+                const uint32_t stage = sbase + s * kStageBytes;
+                const uint64_t dk = thd::smem_desc_sw128(stage, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < kQDim / 16; ++kk)  // S = Q kv^T
+                    thd::mma_bf16_ts(tmem_base + kTmS, tmem_base + kTmQ + kk * 8,
+                                     dk + (((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4), idesc_s,
+                                     kk > 0 ? 1u : 0u);
+                thd::mma_commit(bar(B_S_FULL));
+                ok = wait(B_P_FULL, c & 1);
+                if (!ok) break;
+                thd::tc_fence_after();
+                const uint64_t dv =
+                    thd::smem_desc_sw128(stage + 2 * quarter * kChunkBytes, kChunkBytes, 1024);
+#pragma unroll
+                for (int kk = 0; kk < kBN / 16; ++kk)  // latent quarter += P kv
+                    thd::mma_bf16_ts(tmem_base + kTmO, tmem_base + kTmS + kk * 8,
+                                     dv + ((kk * 16 * 128) >> 4), idesc_o, (c > 0 || kk > 0) ? 1u : 0u);
+                thd::mma_commit(bar(B_O_FULL));
+                thd::mma_commit(bar(B_EMPTY + s));
+            }
+            thd::mma_commit(bar(B_DRAIN));
+            thd::drain_wait(bar(B_DRAIN), 0);
+        }
+        __syncwarp();
+    } else {
+        // --------------------------------------------------- softmax (128)
+        const int row = warp * 32 + lane;
+        const int h = hg * 128 + row;
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+        bool ok = !skip;
+        if (ok) {
+            const uint4* src = reinterpret_cast<const uint4*>(p.q + (t * p.H + h) * kQDim);
+#pragma unroll 1
+            for (int i = 0; i < 9; ++i) {  // 64 elements (32 columns) at a time
+                uint32_t w[32];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const uint4 x = src[i * 8 + u];
+                    w[4 * u] = x.x; w[4 * u + 1] = x.y; w[4 * u + 2] = x.z; w[4 * u + 3] = x.w;
+                }
+                thd::tmem_st32(lane_base + kTmQ + 32 * i, w);
+            }
+            thd::tmem_wait_st();
+            thd::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) thd::mbar_arrive(bar(B_Q_READY));
+        }
+        float m_ref = -INFINITY, l = 0.0f;
+        constexpr float kTau = 8.0f;
+        const float sl2 = p.scale_log2;
+        for (int c = 0; ok && c < nch; ++c) {
+            const int s = c % kNST;
+            ok = thd::warp_wait(bar(B_FULL + s), (c / kNST) & 1, abort_flag, p.status) &&
+                 thd::warp_wait(bar(B_S_FULL), c & 1, abort_flag, p.status);
+            if (!ok) break;
+            thd::tc_fence_after();
+            uint32_t sr[64];
+            thd::tmem_ld32(lane_base + kTmS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+            thd::tmem_ld32(lane_base + kTmS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+            thd::tmem_wait_ld();
+            thd::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+            thd::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+            const float* b = bias + s * kBN;
+            float x[64];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+                x[j] = fmaf(__uint_as_float(sr[j]), sl2, b[j]);
+                mx = fmaxf(mx, x[j]);
+            }
+            float alpha = 1.0f;
+            bool rescale_o = false;
+            if (c == 0 || m_ref == -INFINITY) {
+                if (mx > m_ref) {
+                    alpha = thd::ex2_approx(m_ref - mx);
+                    m_ref = mx;
+                    rescale_o = c > 0;
+                }
+            } else if (mx > m_ref + kTau) {
+                alpha = thd::ex2_approx(m_ref - mx);
+                m_ref = mx;
+                rescale_o = true;
+            }
+            l *= alpha;
+            const float neg_m = m_ref == -INFINITY ? 0.0f : -m_ref;
+            uint32_t pk[32];
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+                const float p0 = thd::ex2_approx(x[2 * u] + neg_m);
+                const float p1 = thd::ex2_approx(x[2 * u + 1] + neg_m);
+                l += p0 + p1;
+                pk[u] = thd::pack_bf16x2(p0, p1);
+            }
+            thd::tmem_st16(lane_base + kTmS, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+            thd::tmem_st16(lane_base + kTmS + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
+            if (c > 0) {
+                // The previous chunk's product must be done before O is
+                // rescaled (and before this chunk's is issued).
+                ok = thd::warp_wait(bar(B_O_FULL), (c - 1) & 1, abort_flag, p.status);
+                if (!ok) break;
+                thd::tc_fence_after();
+                if (__any_sync(0xffffffffu, rescale_o)) {
+#pragma unroll 1
+                    for (int cc = 0; cc < 4; ++cc) {
+                        uint32_t r[32];
+                        thd::tmem_ld32(lane_base + kTmO + 32 * cc, r);
+                        thd::tmem_wait_ld();
+                        thd::reg_fence32(r);
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) * alpha);
+                        thd::tmem_st32(lane_base + kTmO + 32 * cc, r);
+                    }
+                }
+            }
+            thd::tmem_wait_st();
+            thd::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) thd::mbar_arrive(bar(B_P_FULL));
+        }
+        if (ok && nch > 0) ok = thd::warp_wait(bar(B_O_FULL), (nch - 1) & 1, abort_flag, p.status);
+        if (ok) {
+            thd::tc_fence_after();
+            const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
+            __nv_bfloat16* dst = p.latent + (t * p.H + h) * kLat + 128 * quarter;
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t r[32];
+                if (nch > 0) {
+                    thd::tmem_ld32(lane_base + kTmO + 32 * cc, r);
+                    thd::tmem_wait_ld();
+                    thd::reg_fence32(r);
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) r[u] = 0u;
+                }
+                uint32_t w[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u)
+                    w[u] = thd::pack_bf16x2(__uint_as_float(r[2 * u]) * inv_l,
+                                            __uint_as_float(r[2 * u + 1]) * inv_l);
+                uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * cc);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) d4[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+            }
+        }
+    }
+    thd::tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        thd::tc_fence_after();
+        thd::tmem_dealloc(tmem_base, 512);
+    }
+}
+
+// --------------------------------------------------------------- projection --
+// out[t, h, :vd] = latent[t, h, :512] @ W[h]^T: one CTA per (128 tokens,
+// head); K = 512 in 8 chunks of 64 through a 4-stage TMA ring.
+struct ProjParams {
+    __nv_bfloat16* out;  // [T, H, vd]
+    int* status;
+    int64_t T;
+    int H, vd;
+};
+
+constexpr int kPNST = 4;
+constexpr int kPA = 128 * 128;  // A chunk: 128 tokens x 64 latent columns
+
+template <int VD>
+__global__ void __launch_bounds__(192, 1) thd_sparse_mla_proj_kernel(
+    const __grid_constant__ CUtensorMap map_lat, const __grid_constant__ CUtensorMap map_w,
+    const ProjParams p) {
+    constexpr int kPB = VD * 128;  // B chunk: VD rows x 64 columns
+    constexpr int kStage = kPA + kPB;
+    constexpr int BAR = kPNST * kStage;
+    constexpr int TMEM_COLS = VD <= 32 ? 32 : VD <= 64 ? 64 : VD <= 128 ? 128 : 256;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = thd::smem_addr(smem_raw);
+    uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
+    const uint32_t sbase = thd::smem_addr(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.x % p.H;
+    const int64_t t0 = static_cast<int64_t>(blockIdx.x / p.H) * 128;
+    auto bar = [&](int i) -> uint32_t { return sbase + BAR + 8u * i; };  // FULL[4], EMPTY[4], ACC, DRAIN
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + BAR + 8 * (2 * kPNST + 2));
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + BAR + 8 * (2 * kPNST + 2) + 4);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPNST; ++s) {
+            thd::mbar_init(bar(s), 1);
+            thd::mbar_init(bar(kPNST + s), 1);
+        }
+        thd::mbar_init(bar(2 * kPNST), 1);
+        thd::mbar_init(bar(2 * kPNST + 1), 1);
+        *abort_flag = *reinterpret_cast<volatile int*>(p.status) != 0 ? 1 : 0;
+        thd::fence_barrier_init();
+    }
+    if (warp == 5) {
+        thd::tmem_alloc(thd::smem_addr(tmem_slot), TMEM_COLS);
+        thd::tmem_relinquish();
+    }
+    thd::tc_fence_before();
+    __syncthreads();
+    thd::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const bool skip = *abort_flag != 0;
+    constexpr int NCH = kLat / 64;
+    if (warp == 4) {
+        if (lane == 0 && !skip) {
+            thd::tma_prefetch_desc(&map_lat);
+            thd::tma_prefetch_desc(&map_w);
+            int issued = 0;
+            bool ok = true;
+            for (int c = 0; c < NCH && ok; ++c) {
+                const int s = c % kPNST;
+                ok = thd::mbar_wait(bar(kPNST + s), ((c / kPNST) & 1) ^ 1, abort_flag, p.status,
+                                    kStatusTimeout);
+                if (!ok) break;
+                thd::mbar_arrive_expect_tx(bar(s), kStage);
+                thd::tma_load_3d(sbase + s * kStage, &map_lat, bar(s), c * 64, h, static_cast<int>(t0));
+                thd::tma_load_3d(sbase + s * kStage + kPA, &map_w, bar(s), c * 64, 0, h);
+                issued = c + 1;
+            }
+            if (!ok)
+                for (int c = issued - kPNST > 0 ? issued - kPNST : 0; c < issued; ++c)
+                    thd::drain_wait(bar(c % kPNST), (c / kPNST) & 1);
+        }
+        __syncwarp();
+    } else if (warp == 5) {
+        if (lane == 0 && !skip) {
+            constexpr uint32_t idesc = thd::idesc_bf16_f32(128, VD, false);
+            bool ok = true;
+            for (int c = 0; c < NCH && ok; ++c) {
+                const int s = c % kPNST;
+                ok = thd::mbar_wait(bar(s), (c / kPNST) & 1, abort_flag, p.status, kStatusTimeout);
+                if (!ok) break;
+                thd::tc_fence_after();
+                const uint64_t da = thd::smem_desc_sw128(sbase + s * kStage, 16, 1024);
+                const uint64_t db = thd::smem_desc_sw128(sbase + s * kStage + kPA, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    thd::mma_bf16_ss(tmem_base, da + ((kk * 32) >> 4), db + ((kk * 32) >> 4), idesc,
+                                     (c > 0 || kk > 0) ? 1u : 0u);
+                thd::mma_commit(bar(kPNST + s));
+            }
+            if (ok) thd::mma_commit(bar(2 * kPNST));
+            thd::mma_commit(bar(2 * kPNST + 1));
+            thd::drain_wait(bar(2 * kPNST + 1), 0);
+        }
+        __syncwarp();
+    } else if (warp < 4) {
+        const int64_t t = t0 + warp * 32 + lane;
+        bool ok = !skip && thd::warp_wait(bar(2 * kPNST), 0, abort_flag, p.status);
+        if (ok) {
+            thd::tc_fence_after();
+            const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+#pragma unroll 1
+            for (int cc = 0; cc < VD / 32; ++cc) {
+                uint32_t r[32];
+                thd::tmem_ld32(lane_base + 32 * cc, r);
+                thd::tmem_wait_ld();
+                thd::reg_fence32(r);
+                uint32_t w[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u)
+                    w[u] = thd::pack_bf16x2(__uint_as_float(r[2 * u]), __uint_as_float(r[2 * u + 1]));
+                if (t < p.T) {
+                    uint4* d4 = reinterpret_cast<uint4*>(p.out + (t * p.H + h) * VD + 32 * cc);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        d4[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+                }
+            }
+        }
+    }
+    thd::tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        thd::tc_fence_after();
+        thd::tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+template <int VD>
+constexpr int proj_smem() {
+    return kPNST * (kPA + VD * 128) + 8 * (2 * kPNST + 2) + 8 + 1024;
+}
+
+// 3-D map over value_weight [H, VD, 512]: dims (512, VD, H), box (64, VD, 1).
+bool make_w_map(CUtensorMap* map, const void* base, int H, int vd) {
+    auto fn = thd::encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {512, static_cast<cuuint64_t>(vd), static_cast<cuuint64_t>(H)};
+    cuuint64_t strides[2] = {512 * 2, static_cast<cuuint64_t>(vd) * 512 * 2};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(vd), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int VD>
+int launch_proj(const CUtensorMap& ml, const CUtensorMap& mw, const ProjParams& pp, cudaStream_t st) {
+    auto k = thd_sparse_mla_proj_kernel<VD>;
+    static bool attr[64] = {};  // per device
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return THD_ERR_CUDA;
+    if (!attr[dev]) {
+        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, proj_smem<VD>()) !=
+            cudaSuccess)
+            return THD_ERR_CUDA;
+        attr[dev] = true;
+    }
+    const int64_t tiles = (pp.T + 127) / 128;
+    k<<<static_cast<unsigned>(tiles * pp.H), 192, proj_smem<VD>(), st>>>(ml, mw, pp);
+    return cudaGetLastError() == cudaSuccess ? THD_OK : THD_ERR_CUDA;
+}
+
+int* g_status[64] = {};
+
+}  // namespace
+
+extern "C" size_t thd_sparse_mla_workspace_bytes(int64_t T, int H) {
+    if (T <= 0 || H <= 0) return 0;
+    return static_cast<size_t>(T) * static_cast<size_t>(H) * kLat * 2;
+}
+
+extern "C" int thd_sparse_mla_fwd(const void* q, const void* kv, const int32_t* indices,
+                                  const void* value_weight, int64_t T, int64_t Tg, int H, int K,
+                                  int value_dim, float scale, void* out, void* workspace,
+                                  size_t workspace_bytes, void* stream_ptr) {
+    if (T < 0 || Tg < 0 || H <= 0 || K < 0) return THD_ERR_INVALID_ARG;
+    if (H % 128 != 0 || K % kBN != 0) return THD_ERR_UNSUPPORTED;
+    if (value_dim != 64 && value_dim != 128 && value_dim != 256) return THD_ERR_UNSUPPORTED;
+    if (!(std::isfinite(scale) && scale >= 0.0f)) return THD_ERR_INVALID_ARG;
+    if (T == 0) return THD_OK;
+    if (T * (H / 128) * 4 > 0x7fffffffLL || Tg > 0x7fffffffLL) return THD_ERR_INVALID_ARG;
+    if (!q || !kv || (!indices && K > 0) || !value_weight || !out || !workspace)
+        return THD_ERR_INVALID_ARG;
+    if (!thd::aligned16(q) || !thd::aligned16(kv) || !thd::aligned16(value_weight) ||
+        !thd::aligned16(out) || !thd::aligned16(workspace) ||
+        (reinterpret_cast<uintptr_t>(indices) & 3u))
+        return THD_ERR_INVALID_ARG;
+    if (workspace_bytes < thd_sparse_mla_workspace_bytes(T, H)) return THD_ERR_INVALID_ARG;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return THD_ERR_CUDA;
+    if (g_status[dev] == nullptr) {
+        if (cudaMalloc(&g_status[dev], sizeof(int)) != cudaSuccess) return THD_ERR_NO_MEMORY;
+        if (cudaMemset(g_status[dev], 0, sizeof(int)) != cudaSuccess) return THD_ERR_CUDA;
+    }
+    static bool attr[64] = {};  // per device
+    if (!attr[dev]) {
+        if (cudaFuncSetAttribute(thd_sparse_mla_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kSmemAlloc) != cudaSuccess)
+            return THD_ERR_CUDA;
+        attr[dev] = true;
+    }
+    SmlaParams p;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.kv = static_cast<const __nv_bfloat16*>(kv);
+    p.idx = indices;
+    p.latent = static_cast<__nv_bfloat16*>(workspace);
+    p.status = g_status[dev];
+    p.T = T;
+    p.Tg = Tg;
+    p.H = H;
+    p.K = Tg > 0 ? K : 0;  // no key rows: every slot is invalid
+    p.scale_log2 = scale * 1.4426950408889634f;
+    thd_sparse_mla_attn_kernel<<<static_cast<unsigned>(T * (H / 128) * 4), 288, kSmemAlloc, stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return THD_ERR_CUDA;
+
+    CUtensorMap ml, mw;
+    if (!thd::make_map(&ml, workspace, T, H, kLat, 128) || !make_w_map(&mw, value_weight, H, value_dim))
+        return THD_ERR_CUDA;
+    ProjParams pp{static_cast<__nv_bfloat16*>(out), g_status[dev], T, H, value_dim};
+    switch (value_dim) {
+        case 64: return launch_proj<64>(ml, mw, pp, stream);
+        case 128: return launch_proj<128>(ml, mw, pp, stream);
+        default: return launch_proj<256>(ml, mw, pp, stream);
+    }
+}
+
+extern "C" int thd_sparse_mla_get_error(void* stream_ptr) {
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return THD_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return THD_ERR_CUDA;
+    if (g_status[dev] == nullptr) return THD_OK;
+    int s = 0;
+    if (cudaMemcpy(&s, g_status[dev], sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return THD_ERR_CUDA;
+    if (s != 0 && cudaMemset(g_status[dev], 0, sizeof(int)) != cudaSuccess) return THD_ERR_CUDA;
+    return s;
+}

@@ -171,3 +171,32 @@ def bf16_bits(t: torch.Tensor) -> np.ndarray:
     """The raw bf16 bit patterns of a CPU bf16 tensor as a uint16 numpy array."""
     assert t.dtype == torch.bfloat16
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+# ------------------------------------------------------------------ sparse MLA
+
+def sparse_mla_case(seed: int, doc_lengths_: Sequence[int], H: int, K: int, value_dim: int,
+                    device=None) -> dict:
+    """Synthetic sparse-MLA inputs (shapes of "mistral_large4.attention"'s
+    sparse_mla): q [T, H, 576] and kv [T, 576] ~ N(0, 1) in bf16 (the last 64
+    query columns rotary), value_weight [H, value_dim, 512] ~ N(0, 1/512), and
+    for every token a random subset of up to K of the keys it may see (same
+    document, not after it; the caller's document / causal boundaries), in
+    random order, padded with -1; scale (128 + 64) ** -0.5 (a 192-wide MLA
+    query head: 128 latent-absorbed + 64 rotary)."""
+    rng = np.random.default_rng(seed)
+    cu = cu_seqlens_from_lengths(doc_lengths_)
+    T = int(cu[-1])
+    q = random_bf16(rng, (T, H, 576))
+    kv = random_bf16(rng, (T, 576))
+    w = random_bf16(rng, (H, value_dim, 512), std=512 ** -0.5)
+    idx = np.full((T, K), -1, dtype=np.int32)
+    for d in range(len(cu) - 1):
+        s, e = int(cu[d]), int(cu[d + 1])
+        for t in range(s, e):
+            n = min(K, t - s + 1)
+            sel = rng.choice(np.arange(s, t + 1), size=n, replace=False)
+            slots = rng.permutation(K)[:n]
+            idx[t, slots] = sel
+    return {"q": q, "kv": kv, "value_weight": w, "indices": torch.from_numpy(idx), "T": T,
+            "cu_seqlens": cu, "scale": (128 + 64) ** -0.5}

@@ -31,7 +31,7 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for want in ("thd_attn_fwd", "thd_attn_get_error", "thd_attn_status_string", "thd_attn_plan",
                  "thd_attn_abi_version", "thd_attn_bwd", "thd_attn_bwd_workspace_bytes",
-                 "thd_qk_norm_rope"):
+                 "thd_qk_norm_rope", "thd_sparse_mla_fwd", "thd_sparse_mla_workspace_bytes"):
         assert want in names
 
 
@@ -162,3 +162,34 @@ def _pro(lib, cu, Hq=4, Hkv=2, D=128, eps=1e-5, theta=500000.0, rope=1, ptr=0x10
 ])
 def test_prologue_rejects_bad_arguments_before_any_launch(lib, kw, code):
     assert _pro(lib, **kw) == code
+
+
+# ------------------------------------------------------------- sparse MLA ---
+
+def _smla(lib, T=4, Tg=4, H=128, K=64, vd=128, scale=0.1, ptr=0x10000, idx=0x10000, ws=0x10000,
+          ws_bytes=1 << 30, out=0x10000):
+    lib.thd_sparse_mla_fwd.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64, ctypes.c_int64] + \
+        [ctypes.c_int] * 3 + [ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                              ctypes.c_void_p]
+    return lib.thd_sparse_mla_fwd(ptr, ptr, idx, ptr, T, Tg, H, K, vd, scale, out, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(H=64), -2),              # heads in groups of 128
+    (dict(K=50), -2),              # slots in chunks of 64 (pad with -1)
+    (dict(vd=100), -2),
+    (dict(scale=float("nan")), -1),
+    (dict(T=-1), -1),
+    (dict(idx=0x10002), -1),       # misaligned int32 indices
+    (dict(out=0x10008), -1),       # misaligned bf16 output
+    (dict(ws_bytes=100), -1),      # workspace smaller than the latent
+    (dict(T=0), 0),                # nothing to do
+])
+def test_sparse_mla_rejects_bad_arguments_before_any_launch(lib, kw, code):
+    assert _smla(lib, **kw) == code
+
+
+def test_sparse_mla_workspace_size(lib):
+    lib.thd_sparse_mla_workspace_bytes.argtypes = [ctypes.c_int64, ctypes.c_int]
+    lib.thd_sparse_mla_workspace_bytes.restype = ctypes.c_size_t
+    assert lib.thd_sparse_mla_workspace_bytes(10, 128) == 10 * 128 * 512 * 2
