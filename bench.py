@@ -505,7 +505,8 @@ def run_sparse_mla(args, info, device):
     valid = int((c["indices"] >= 0).sum())
     flop = valid * H * 2 * (576 + 512) + T * H * 512 * vd * 2
     out = torch.empty((T, H, vd), dtype=torch.bfloat16, device=device)
-    ws = torch.empty((swa.thd_sparse_mla_workspace_bytes(T, H),), dtype=torch.uint8, device=device)
+    ws = torch.empty((swa.thd_sparse_mla_workspace_bytes(T, H, w["K"]),), dtype=torch.uint8,
+                     device=device)
     stream = torch.cuda.current_stream(device)
 
     def step():

@@ -298,14 +298,15 @@ int thd_qk_norm_rope(void* q, void* k, const int32_t* cu_seqlens, int n_docs,
  *                 boundaries; each valid slot counts once, as given)
  *   value_weight  bf16 device [H, value_dim, 512]
  *   out           bf16 device [T, H, value_dim], written
- *   workspace     device scratch >= thd_sparse_mla_workspace_bytes(T, H)
- *                 (the bf16 latent [T, H, 512]), 16-byte aligned
+ *   workspace     device scratch >= thd_sparse_mla_workspace_bytes(T, H, K)
+ *                 (the bf16 latent [T, H, 512], the token's valid slots moved
+ *                 to the front, their counts), 16-byte aligned
  * Supported: H a multiple of 128, K a multiple of 64 (pad with -1),
  * value_dim 64, 128 or 256 (else THD_ERR_UNSUPPORTED).  Argument errors
  * return before anything is enqueued; kernel stalls are reported by
  * thd_sparse_mla_get_error.
  */
-size_t thd_sparse_mla_workspace_bytes(int64_t T, int H);
+size_t thd_sparse_mla_workspace_bytes(int64_t T, int H, int K);
 int thd_sparse_mla_fwd(const void* q, const void* kv, const int32_t* indices,
                        const void* value_weight, int64_t T, int64_t Tg, int H, int K,
                        int value_dim, float scale, void* out,

@@ -86,7 +86,7 @@ def load_library():
                                         c_int, c_int, vp, ctypes.c_int64,
                                         ctypes.POINTER(ctypes.c_int64)]
     lib.thd_attn_plan_range.restype = c_int
-    lib.thd_sparse_mla_workspace_bytes.argtypes = [ctypes.c_int64, c_int]
+    lib.thd_sparse_mla_workspace_bytes.argtypes = [ctypes.c_int64, c_int, c_int]
     lib.thd_sparse_mla_workspace_bytes.restype = ctypes.c_size_t
     lib.thd_sparse_mla_fwd.argtypes = [vp, vp, vp, vp, ctypes.c_int64, ctypes.c_int64, c_int, c_int,
                                        c_int, ctypes.c_float, vp, vp, ctypes.c_size_t, vp]
@@ -382,7 +382,7 @@ def thd_sparse_mla_fwd(q, kv, indices, value_weight, scale: float, out=None, wor
         raise ValueError("shapes: q [T, H, 576], kv [Tg, 576], indices [T, K], value_weight [H, vd, 512]")
     if out is None:
         out = torch.empty((T, H, vd), dtype=torch.bfloat16, device=q.device)
-    need = int(lib.thd_sparse_mla_workspace_bytes(T, H))
+    need = int(lib.thd_sparse_mla_workspace_bytes(T, H, K))
     if workspace is None:
         workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=q.device)
     if stream is None:
@@ -397,9 +397,10 @@ def thd_sparse_mla_fwd(q, kv, indices, value_weight, scale: float, out=None, wor
     return out
 
 
-def thd_sparse_mla_workspace_bytes(T: int, H: int) -> int:
-    """Workspace bytes :func:`thd_sparse_mla_fwd` needs (the bf16 latent [T, H, 512])."""
-    return int(load_library().thd_sparse_mla_workspace_bytes(int(T), int(H)))
+def thd_sparse_mla_workspace_bytes(T: int, H: int, K: int) -> int:
+    """Workspace bytes :func:`thd_sparse_mla_fwd` needs (the bf16 latent
+    [T, H, 512], compacted indices [T, K], counts [T])."""
+    return int(load_library().thd_sparse_mla_workspace_bytes(int(T), int(H), int(K)))
 
 
 def thd_sparse_mla_get_error(stream=None) -> int:

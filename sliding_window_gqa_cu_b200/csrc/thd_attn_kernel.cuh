@@ -75,12 +75,14 @@ struct FwdConfig {
     static constexpr int MMA_WARP = NUM_SOFTMAX_WARPS + 1;
     static constexpr int NUM_THREADS = (NUM_SOFTMAX_WARPS + 4) * 32;
     // With three warpgroups a thread starts with 168 registers (3 warps per
-    // SM sub-partition); the control warpgroup hands most of its share to the
-    // softmax warpgroups: 2*128*208 + 128*88 = 384*168.
+    // SM sub-partition); the control warpgroup hands part of its share to the
+    // softmax warpgroups: 2*128*192 + 128*120 = 384*168.  (With 208 / 88 the
+    // control warps spilled; 192 / 120 spills nothing and measured 1-5 %
+    // faster.)
     static constexpr bool REG_SPLIT = NQ == 2;
     static constexpr int LAUNCH_REGS = 168;
-    static constexpr int SOFTMAX_REGS = 208;
-    static constexpr int CONTROL_REGS = 88;
+    static constexpr int SOFTMAX_REGS = 192;
+    static constexpr int CONTROL_REGS = 120;
     static_assert(!REG_SPLIT || (NQ * 128 * SOFTMAX_REGS + 128 * CONTROL_REGS <=
                                  NUM_THREADS * LAUNCH_REGS), "register split exceeds the launch");
 

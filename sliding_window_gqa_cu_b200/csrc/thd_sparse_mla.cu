@@ -3,7 +3,12 @@
 // For token t and head h: s_j = scale * <q[t, h, :576], kv[idx[t, j], :576]>
 // over the valid index slots j (idx >= 0), p = softmax(s), latent =
 // sum_j p_j kv[idx[t, j], :512], out[t, h, :] = value_weight[h] @ latent.
-// A row without a valid slot is zero.  Two kernels:
+// A row without a valid slot is zero.  Three kernels:
+//
+// 0. Compaction (thd_sparse_mla_compact_kernel): one warp per token moves the
+//    token's valid slots to the front of a copy of its index row (the order
+//    of slots does not change the softmax) and records their count, so that
+//    the attention processes ceil(count / 64) slot chunks, not K / 64.
 //
 // 1. Attention (thd_sparse_mla_attn_kernel): one CTA per (token, group of
 //    128 heads, quarter of the 512 latent columns).  The 128 query rows of
@@ -53,7 +58,8 @@ __device__ __forceinline__ void cp_async_wait() {
 struct SmlaParams {
     const __nv_bfloat16* q;    // [T, H, 576]
     const __nv_bfloat16* kv;   // [Tg, 576]
-    const int32_t* idx;        // [T, K]
+    const int32_t* idx;        // [T, K] valid slots first (compacted)
+    const int32_t* count;      // [T] valid slots per token
     __nv_bfloat16* latent;     // [T, H, 512] (workspace)
     int* status;
     int64_t T, Tg;
@@ -78,6 +84,28 @@ constexpr int kSmemAlloc = kSmemAbort + 4 + 1024;
 static_assert(kSmemAlloc <= 232448, "shared memory budget exceeded");
 static_assert(kTmO + 128 <= 512, "TMEM budget exceeded");
 
+__global__ void __launch_bounds__(256) thd_sparse_mla_compact_kernel(const int32_t* __restrict__ idx,
+                                                                      int64_t T, int K, int64_t Tg,
+                                                                      int32_t* __restrict__ idx_c,
+                                                                      int32_t* __restrict__ count) {
+    const int lane = threadIdx.x & 31;
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const int32_t* src = idx + t * K;
+    int32_t* dst = idx_c + t * K;
+    int n = 0;
+    for (int j0 = 0; j0 < K; j0 += 32) {
+        const int j = j0 + lane;
+        const int v = j < K ? src[j] : -1;
+        const bool ok = v >= 0 && v < Tg;
+        const unsigned m = __ballot_sync(0xffffffffu, ok);
+        if (ok) dst[n + __popc(m & ((1u << lane) - 1u))] = v;
+        n += __popc(m);
+    }
+    for (int j = n + lane; j < K; j += 32) dst[j] = -1;
+    if (lane == 0) count[t] = n;
+}
+
 __global__ void __launch_bounds__(288, 1) thd_sparse_mla_attn_kernel(const SmlaParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = thd::smem_addr(smem_raw);
@@ -88,7 +116,7 @@ __global__ void __launch_bounds__(288, 1) thd_sparse_mla_attn_kernel(const SmlaP
     const int hgroups = p.H / 128;
     const int hg = (blockIdx.x >> 2) % hgroups;
     const int64_t t = (blockIdx.x >> 2) / hgroups;
-    const int nch = p.K / kBN;
+    const int nch = (p.count[t] + kBN - 1) / kBN;  // chunks holding valid slots
 
     auto bar = [&](int i) -> uint32_t { return sbase + kSmemBar + 8u * i; };
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSmemAbort);
@@ -229,13 +257,19 @@ __global__ void __launch_bounds__(288, 1) thd_sparse_mla_attn_kernel(const SmlaP
             thd::tmem_wait_ld();
             thd::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
             thd::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-            const float* b = bias + s * kBN;
+            const float4* b4 = reinterpret_cast<const float4*>(bias + s * kBN);
             float x[64];
             float mx = -INFINITY;
 #pragma unroll
-            for (int j = 0; j < 64; ++j) {
-                x[j] = fmaf(__uint_as_float(sr[j]), sl2, b[j]);
-                mx = fmaxf(mx, x[j]);
+            for (int j4 = 0; j4 < 16; ++j4) {
+                const float4 b = b4[j4];
+                const float bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = 4 * j4 + e;
+                    x[j] = fmaf(__uint_as_float(sr[j]), sl2, bv[e]);
+                    mx = fmaxf(mx, x[j]);
+                }
             }
             float alpha = 1.0f;
             bool rescale_o = false;
@@ -485,11 +519,17 @@ int launch_proj(const CUtensorMap& ml, const CUtensorMap& mw, const ProjParams& 
 
 int* g_status[64] = {};
 
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
 }  // namespace
 
-extern "C" size_t thd_sparse_mla_workspace_bytes(int64_t T, int H) {
-    if (T <= 0 || H <= 0) return 0;
-    return static_cast<size_t>(T) * static_cast<size_t>(H) * kLat * 2;
+// Workspace: the bf16 latent [T, H, 512], the compacted indices [T, K] and
+// the per-token valid-slot counts [T] (each part 256-byte aligned).
+extern "C" size_t thd_sparse_mla_workspace_bytes(int64_t T, int H, int K) {
+    if (T <= 0 || H <= 0 || K < 0) return 0;
+    return align256(static_cast<size_t>(T) * static_cast<size_t>(H) * kLat * 2) +
+           align256(static_cast<size_t>(T) * static_cast<size_t>(K) * 4) +
+           align256(static_cast<size_t>(T) * 4);
 }
 
 extern "C" int thd_sparse_mla_fwd(const void* q, const void* kv, const int32_t* indices,
@@ -508,7 +548,7 @@ extern "C" int thd_sparse_mla_fwd(const void* q, const void* kv, const int32_t* 
         !thd::aligned16(out) || !thd::aligned16(workspace) ||
         (reinterpret_cast<uintptr_t>(indices) & 3u))
         return THD_ERR_INVALID_ARG;
-    if (workspace_bytes < thd_sparse_mla_workspace_bytes(T, H)) return THD_ERR_INVALID_ARG;
+    if (workspace_bytes < thd_sparse_mla_workspace_bytes(T, H, K)) return THD_ERR_INVALID_ARG;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return THD_ERR_CUDA;
@@ -523,16 +563,24 @@ extern "C" int thd_sparse_mla_fwd(const void* q, const void* kv, const int32_t* 
             return THD_ERR_CUDA;
         attr[dev] = true;
     }
+    char* ws = static_cast<char*>(workspace);
+    int32_t* idx_c = reinterpret_cast<int32_t*>(ws + align256(static_cast<size_t>(T) * H * kLat * 2));
+    int32_t* cnt = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(idx_c) +
+                                              align256(static_cast<size_t>(T) * K * 4));
+    const int Keff = Tg > 0 ? K : 0;  // no key rows: every slot is invalid
+    thd_sparse_mla_compact_kernel<<<static_cast<unsigned>((T + 7) / 8), 256, 0, stream>>>(
+        indices, T, Keff, Tg, idx_c, cnt);
     SmlaParams p;
     p.q = static_cast<const __nv_bfloat16*>(q);
     p.kv = static_cast<const __nv_bfloat16*>(kv);
-    p.idx = indices;
+    p.idx = idx_c;
+    p.count = cnt;
     p.latent = static_cast<__nv_bfloat16*>(workspace);
     p.status = g_status[dev];
     p.T = T;
     p.Tg = Tg;
     p.H = H;
-    p.K = Tg > 0 ? K : 0;  // no key rows: every slot is invalid
+    p.K = Keff;
     p.scale_log2 = scale * 1.4426950408889634f;
     thd_sparse_mla_attn_kernel<<<static_cast<unsigned>(T * (H / 128) * 4), 288, kSmemAlloc, stream>>>(p);
     if (cudaGetLastError() != cudaSuccess) return THD_ERR_CUDA;

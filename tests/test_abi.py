@@ -190,6 +190,7 @@ def test_sparse_mla_rejects_bad_arguments_before_any_launch(lib, kw, code):
 
 
 def test_sparse_mla_workspace_size(lib):
-    lib.thd_sparse_mla_workspace_bytes.argtypes = [ctypes.c_int64, ctypes.c_int]
+    lib.thd_sparse_mla_workspace_bytes.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int]
     lib.thd_sparse_mla_workspace_bytes.restype = ctypes.c_size_t
-    assert lib.thd_sparse_mla_workspace_bytes(10, 128) == 10 * 128 * 512 * 2
+    # latent 10*128*512*2, indices 10*64*4 -> 2560 (256-aligned), counts 40 -> 256
+    assert lib.thd_sparse_mla_workspace_bytes(10, 128, 64) == 1310720 + 2560 + 256
