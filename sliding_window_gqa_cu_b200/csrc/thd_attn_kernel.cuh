@@ -319,7 +319,35 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 }
                 mma_commit(bar(C::B_SLOT_EMPTY + (2 * jj) % C::NSLOT));
             }
-            for (int j = 0; ok && j < n; ++j) {
+            for (int j = 0; ok && j < n && C::NSB == 1; ++j) {
+                // One S buffer per head: PV(j) and QK(j+1) of a head go out as
+                // one run of 2 * 8 MMAs (QK(j+1) may overwrite S = P(j) only
+                // after PV(j), which the in-order tensor pipe guarantees), with
+                // one commit: S(j+1) ready also means O holds PV(j), so O gets
+                // its own commit only after the last tile.  Fewer boundaries
+                // between MMA runs keep the tensor pipe fed.
+                const int vslot = (2 * j + 1) % C::NSLOT;
+                const bool has_next = j + 1 < n;
+                const int kslot = (2 * j + 2) % C::NSLOT;
+                ok = wait_slot(2 * j + 1) && (!has_next || wait_slot(2 * j + 2));
+                if (!ok) break;
+                for (int q = 0; q < C::NQ && ok; ++q) {
+                    ok = mbar_wait(bar(C::B_P_FULL + q), j & 1, abort_flag, p.status, kStatusTimeout);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(q, 0, vslot, j > 0);
+                    if (has_next) {
+                        issue_qk(q, 0, kslot);
+                        mma_commit(bar(C::B_S_FULL + q));
+                    } else {
+                        mma_commit(bar(C::B_O_FULL + q));
+                    }
+                }
+                if (!ok) break;
+                mma_commit(bar(C::B_SLOT_EMPTY + vslot));                   // V(j) done
+                if (has_next) mma_commit(bar(C::B_SLOT_EMPTY + kslot));   // K(j+1) done
+            }
+            for (int j = 0; ok && j < n && C::NSB == 2; ++j) {
                 const int vslot = (2 * j + 1) % C::NSLOT;
                 ok = wait_slot(2 * j + 1);
                 if (!ok) break;
@@ -477,7 +505,9 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
             l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
         }
 
-        if (ok) ok = warp_wait(bar(C::B_O_FULL + q), (n - 1) & 1, abort_flag, p.status);
+        // With one S buffer O_FULL completes once (after the last PV); with
+        // two, once per tile.
+        if (ok) ok = warp_wait(bar(C::B_O_FULL + q), C::NSB == 1 ? 0u : (n - 1) & 1, abort_flag, p.status);
         if (ok) {
             tc_fence_after();
             const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
