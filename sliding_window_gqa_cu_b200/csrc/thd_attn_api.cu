@@ -254,7 +254,7 @@ int launch_bwd(DeviceState* ds, const BwdPlanEntry& plan, const CUtensorMap& mq,
                const CUtensorMap& mdo, const CUtensorMap& mk, const CUtensorMap& mv,
                const thd::BwdParams& prm, const void* out, const void* dout, const float* sinks,
                float* dsinks, float* delta, float* sink_part, cudaStream_t stream) {
-    using Cq = thd::BwdConfig<D, D == 64 ? 8 : 4>;  // one CTA per SM (all 512 TMEM columns)
+    using Cq = thd::BwdConfig<D, D == 64 ? 8 : 5>;  // one CTA per SM (all 512 TMEM columns)
     using Ckv = thd::BwdConfig<D, D == 64 ? 4 : 2>;
     auto kq = thd::thd_attn_bwd_dq_kernel<Cq>;
     auto kkv = thd::thd_attn_bwd_dkdv_kernel<Ckv>;

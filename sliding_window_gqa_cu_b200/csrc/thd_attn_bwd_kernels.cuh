@@ -16,20 +16,23 @@
 //   * dq kernel: one CTA per (128-row query tile, query head), looping over
 //     the key tiles the tile sees: S = Q K^T, dP = dO V^T, dS written as bf16
 //     over S in TMEM, dq += dS K (dS from TMEM, K from shared memory as an
-//     MN-major operand).
+//     MN-major operand).  S alternates between two TMEM buffers, so the
+//     tensor core computes dq(j), dP(j + 1) and S(j + 2) while the
+//     elementwise warps exponentiate S(j + 1).
 //   * dkdv kernel: one CTA per (128-key tile, kv head), looping over the
-//     query heads of the group and the query tiles that see the keys:
+//     query heads of the group and the 128-query tiles that see the keys:
 //     S^T = K Q^T and dP^T = V dO^T (TMEM lane = key), P^T and dS^T written as
 //     bf16 over them, dv += P^T dO and dk += dS^T Q (TMEM operands, dO and Q
 //     as MN-major operands); dk and dv stay in TMEM for the whole group.
 //
 // Warps (both kernels): 0-7 elementwise, 8 TMA producer, 9 MMA issuer, 10-11
-// idle.  Elementwise warp w owns TMEM lanes [32 (w % 4), 32 (w % 4) + 32)
-// and the 64 columns [64 h, 64 h + 64) of S and dP, h = w / 4: no row-wide
-// reduction is needed (the log-sum-exp is known), so the two warps on a
-// sub-partition work on independent halves of every tile.  Half h writes
-// its 64 bf16 results (P, dS) over its own columns [64 h, 64 h + 32).  Every
-// wait is bounded and reports a timeout in the device status word.
+// idle.  Elementwise warp w owns TMEM lanes [32 (w % 4), 32 (w % 4) + 32).
+// No row-wide reduction is needed (the log-sum-exp is known), so the warps
+// on a sub-partition work on independent halves of every tile: the 64
+// columns [64 h, 64 h + 64) of S and dP (or S^T and dP^T), h = w / 4, with
+// the half's 64 bf16 results (P, dS) written over its own columns
+// [64 h, 64 h + 32).  Every wait is bounded and reports a timeout in the
+// device status word.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -157,6 +160,7 @@ struct BwdConfig {
     static constexpr int TM_DP = 128;     // dP or dP^T, then dS^T (dkdv)
     static constexpr int TM_ACC0 = 256;   // dq (dq kernel) or dv (dkdv kernel)
     static constexpr int TM_ACC1 = 256 + D;  // dk (dkdv kernel)
+    static constexpr int TM_S2 = 384;     // dq kernel: second S buffer (odd key tiles)
     static constexpr int TMEM_COLS = 512;
 
     static constexpr int PRODUCER_WARP = 8;
@@ -165,6 +169,7 @@ struct BwdConfig {
 
     static_assert(D == 64 || D == 128, "backward kernels: head dim 64 or 128");
     static_assert(TM_ACC1 + D <= 512, "TMEM budget exceeded");
+    static_assert(TM_ACC0 + D <= TM_S2 && TM_S2 + BN <= TMEM_COLS, "dq kernel TMEM budget exceeded");
     static_assert(NSLOT >= 2, "ring needs two slots");
 };
 
@@ -174,8 +179,8 @@ struct DqLayout {
     static constexpr int B_IN_FULL = 0;                       // Q and dO landed
     static constexpr int B_SLOT_FULL = 1;
     static constexpr int B_SLOT_EMPTY = B_SLOT_FULL + C::NSLOT;
-    static constexpr int B_S_FULL = B_SLOT_EMPTY + C::NSLOT;  // S done
-    static constexpr int B_DP_FULL = B_S_FULL + 1;            // dP done
+    static constexpr int B_S_FULL = B_SLOT_EMPTY + C::NSLOT;  // [2] S of an even / odd tile done
+    static constexpr int B_DP_FULL = B_S_FULL + 2;            // dP done
     static constexpr int B_DS_FULL = B_DP_FULL + 1;           // dS in TMEM (8 warps)
     static constexpr int B_ACC_FULL = B_DS_FULL + 1;          // dq accumulated
     static constexpr int B_DRAIN = B_ACC_FULL + 1;
@@ -218,6 +223,7 @@ thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
             mbar_init(bar(L::B_SLOT_EMPTY + s), 1);
         }
         mbar_init(bar(L::B_S_FULL), 1);
+        mbar_init(bar(L::B_S_FULL + 1), 1);
         mbar_init(bar(L::B_DP_FULL), 1);
         mbar_init(bar(L::B_DS_FULL), 8);
         mbar_init(bar(L::B_ACC_FULL), 1);
@@ -286,36 +292,52 @@ thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
             auto wait_slot = [&](int pos) -> bool {
                 return wait(L::B_SLOT_FULL + pos % C::NSLOT, (pos / C::NSLOT) & 1);
             };
-            bool ok = wait(L::B_IN_FULL, 0);
-            for (int j = 0; ok && j < n; ++j) {
-                const int kslot = (2 * j) % C::NSLOT, vslot = (2 * j + 1) % C::NSLOT;
-                ok = wait_slot(2 * j) && wait_slot(2 * j + 1);
-                if (!ok) break;
+            // Two S buffers: S(j + 2) and dP(j + 1) run on the tensor core
+            // while the elementwise warps turn S(j + 1) into exponentials.
+            auto issue_s = [&](int j) -> bool {  // S(j) = Q K(j)^T into buffer j % 2
+                if (!wait_slot(2 * j)) return false;
                 tc_fence_after();
-                const uint64_t dk = dkv0 + ((kslot * C::TILE_BYTES) >> 4);
+                const uint64_t dk = dkv0 + ((((2 * j) % C::NSLOT) * C::TILE_BYTES) >> 4);
+                const uint32_t ts = tmem_base + ((j & 1) ? C::TM_S2 : C::TM_S);
+#pragma unroll
+                for (int kk = 0; kk < C::D / 16; ++kk) {
+                    const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
+                    mma_bf16_ss(ts, dq0 + o, dk + o, idesc_s, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bar(L::B_S_FULL + (j & 1)));
+                return true;
+            };
+            auto issue_dp = [&](int j) -> bool {  // dP(j) = dO V(j)^T
+                if (!wait_slot(2 * j + 1)) return false;
+                tc_fence_after();
+                const int vslot = (2 * j + 1) % C::NSLOT;
                 const uint64_t dv = dkv0 + ((vslot * C::TILE_BYTES) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < C::D / 16; ++kk) {  // S = Q K^T
-                    const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
-                    mma_bf16_ss(tmem_base + C::TM_S, dq0 + o, dk + o, idesc_s, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(bar(L::B_S_FULL));  // the exponentials start under dP
-#pragma unroll
-                for (int kk = 0; kk < C::D / 16; ++kk) {  // dP = dO V^T
+                for (int kk = 0; kk < C::D / 16; ++kk) {
                     const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
                     mma_bf16_ss(tmem_base + C::TM_DP, ddo0 + o, dv + o, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar(L::B_DP_FULL));
                 mma_commit(bar(L::B_SLOT_EMPTY + vslot));  // V(j) consumed
+                return true;
+            };
+            bool ok = wait(L::B_IN_FULL, 0) && issue_s(0) && issue_dp(0) && (n < 2 || issue_s(1));
+            for (int j = 0; ok && j < n; ++j) {
                 ok = wait(L::B_DS_FULL, j & 1);
                 if (!ok) break;
                 tc_fence_after();
+                const int kslot = (2 * j) % C::NSLOT;
                 const uint64_t dkmn = dkmn0 + ((kslot * C::TILE_BYTES) >> 4);
+                const uint32_t ts = tmem_base + ((j & 1) ? C::TM_S2 : C::TM_S);
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; ++kk)  // dq += dS K
-                    mma_bf16_ts(tmem_base + C::TM_ACC0, tmem_base + C::TM_S + pcol(kk),
+                    mma_bf16_ts(tmem_base + C::TM_ACC0, ts + pcol(kk),
                                 dkmn + ((kk * 16 * 128) >> 4), idesc_acc, (j > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(bar(L::B_SLOT_EMPTY + kslot));  // K(j) consumed
+                // dP(j + 1) overwrites dP(j), read before dS(j) was signalled;
+                // S(j + 2) overwrites dS(j), issued after the MMAs reading it.
+                if (j + 1 < n) ok = issue_dp(j + 1);
+                if (ok && j + 2 < n) ok = issue_s(j + 2);
             }
             if (ok) mma_commit(bar(L::B_ACC_FULL));
             mma_commit(bar(L::B_DRAIN));
@@ -344,9 +366,10 @@ thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
 
         bool ok = !skip;
         for (int j = 0; ok && j < n; ++j) {
-            ok = warp_wait(bar(L::B_S_FULL), j & 1, abort_flag, prm.status);
+            ok = warp_wait(bar(L::B_S_FULL + (j & 1)), (j >> 1) & 1, abort_flag, prm.status);
             if (!ok) break;
             tc_fence_after();
+            const uint32_t tm_s = (j & 1) ? C::TM_S2 : C::TM_S;
             const int kh = it.kv_start + j * C::BN + 64 * h;  // first key of this half
             const bool full = row_valid && kh >= s_doc && kh + 63 <= r_lo &&
                               (W == 0 || kh >= r_hi - W + 1);
@@ -355,8 +378,8 @@ thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
             float pv[64];
             {
                 uint32_t sr[64];
-                tmem_ld32(lane_base + C::TM_S + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                tmem_ld32(lane_base + C::TM_S + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                tmem_ld32(lane_base + tm_s + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                tmem_ld32(lane_base + tm_s + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
                 tmem_wait_ld();
                 reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
                 reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
@@ -382,7 +405,7 @@ thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
                                         pv[32 * cc + 2 * u + 1] * (__uint_as_float(dr[2 * u + 1]) - Di));
                 // dS of this half's columns [32 cc, 32 cc + 32) goes to TMEM
                 // columns 64 h + [16 cc, 16 cc + 16) (S of this half, read).
-                tmem_st16(lane_base + C::TM_S + 64 * h + 16 * cc, pk);
+                tmem_st16(lane_base + tm_s + 64 * h + 16 * cc, pk);
             }
             tmem_wait_st();
             tc_fence_before();
