@@ -156,6 +156,46 @@ int thd_attn_fwd_range(const void* q, const void* k, const void* v,
                        void* out, float* lse,
                        void* stream);
 
+/*
+ * The forward from HOST buffers, with the copies overlapped with the
+ * attention ("API" section of the sliding-window attention page: the same
+ * packed-THD forward as thd_attn_fwd).  The pack is split into n_chunks
+ * token ranges of equal length; range c's q / k / v rows are copied to the
+ * device on a copy stream, its query rows are computed as thd_attn_fwd_range
+ * does on `stream` once they have landed (they read only key rows of their
+ * own document at or before them, all copied by then), and its out / lse
+ * rows are copied back on a second copy stream; copies of later ranges run
+ * while earlier ranges compute.  The result equals thd_attn_fwd on the same
+ * rows.
+ *   q_host, k_host, v_host   bf16 host [T, Hq, D] / [T, Hkv, D] (page-locked
+ *                            for the copies to overlap; pageable memory
+ *                            works but serialises them)
+ *   sinks_host_or_null       fp32 host [Hq] or NULL
+ *   out_host, lse_host       bf16 host [T, Hq, D], fp32 host [T, Hq]: written
+ *   q_dev .. lse_dev         device buffers of the same shapes (sinks_dev
+ *                            [Hq], NULL exactly when sinks_host is), owned by
+ *                            the caller, used as staging; 16-byte aligned as
+ *                            thd_attn_fwd requires
+ *   n_chunks                 1 .. 64 (the schedule cache keeps 16 ranges, so
+ *                            up to about 8 stays cached between calls)
+ * Asynchronous: returns once everything is queued; `stream` completes after
+ * the last device-to-host copy, so synchronising it makes out_host and
+ * lse_host valid.  The host buffers must stay untouched until then.  Calls
+ * are serialised inside the library (one set of copy streams per device).
+ * Errors: THD_ERR_INVALID_ARG for a NULL buffer, a sinks pair with one NULL,
+ * n_chunks out of range or an invalid cu_seqlens (checked before any CUDA
+ * call); otherwise thd_attn_fwd_range's errors, or THD_ERR_CUDA for a failed
+ * copy.  T = 0 is a no-op.
+ */
+int thd_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
+                      const int32_t* cu_seqlens, int n_docs,
+                      int Hq, int Hkv, int D, int window, float scale,
+                      const float* sinks_host_or_null,
+                      void* out_host, float* lse_host,
+                      void* q_dev, void* k_dev, void* v_dev, float* sinks_dev_or_null,
+                      void* out_dev, float* lse_dev,
+                      int n_chunks, void* stream);
+
 /* Host-only: the schedule thd_attn_fwd_range uses (q0 of a tile that would
  * reach before q_begin > 0 is raised to q_begin).  Same conventions as
  * thd_attn_plan. */

@@ -20,7 +20,10 @@ from typing import Optional
 
 import numpy as np
 
-__all__ = ["thd_attn_fwd", "thd_attn_fwd_noalloc", "thd_attn_get_error", "thd_attn_plan",
+__all__ = ["thd_attn_fwd", "thd_attn_fwd_noalloc", "thd_attn_fwd_range", "thd_attn_fwd_host",
+           "thd_attn_bwd", "thd_attn_bwd_workspace_bytes", "thd_qk_norm_rope",
+           "thd_sparse_mla_fwd", "thd_sparse_mla_workspace_bytes", "thd_sparse_mla_get_error",
+           "thd_attn_get_error", "thd_attn_plan", "thd_attn_plan_range",
            "ThdAttnError", "library_path", "load_library", "STATUS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -82,6 +85,9 @@ def load_library():
     lib.thd_attn_fwd_range.argtypes = [vp, vp, vp, i32p, c_int, ctypes.c_int64, ctypes.c_int64,
                                        c_int, c_int, c_int, c_int, ctypes.c_float, vp, vp, vp, vp]
     lib.thd_attn_fwd_range.restype = c_int
+    lib.thd_attn_fwd_host.argtypes = [vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int,
+                                      ctypes.c_float, vp, vp, vp, vp, vp, vp, vp, vp, vp, c_int, vp]
+    lib.thd_attn_fwd_host.restype = c_int
     lib.thd_attn_plan_range.argtypes = [i32p, c_int, ctypes.c_int64, ctypes.c_int64, c_int, c_int,
                                         c_int, c_int, vp, ctypes.c_int64,
                                         ctypes.POINTER(ctypes.c_int64)]
@@ -339,6 +345,70 @@ def thd_attn_fwd_range(q, k, v, cu_seqlens, q_begin: int, q_end: int, window: in
     if rc != 0:
         raise ThdAttnError(rc, "thd_attn_fwd_range")
     return out, lse
+
+
+def thd_attn_fwd_host(q_host, k_host, v_host, cu_seqlens, window: int = 0,
+                      scale: Optional[float] = None, sinks_host=None, out_host=None,
+                      lse_host=None, device_buffers=None, n_chunks: int = 8, stream=None):
+    """The forward from host tensors with the copies overlapped with the
+    attention (token ranges pipelined over two copy streams and ``stream``).
+
+    q_host, k_host, v_host: bf16 CPU tensors [T, Hq, D] / [T, Hkv, D]
+    (page-locked for the copies to overlap); sinks_host: fp32 CPU [Hq] or
+    None.  ``device_buffers`` is an optional dict of CUDA staging tensors
+    ``q, k, v, out, lse`` (and ``sinks``) of the same shapes, reused across
+    calls; missing ones are allocated on the current device.  Returns
+    ``(out_host, lse_host)``; they are valid once ``stream`` (default: the
+    current stream) has been synchronised.
+    """
+    import torch
+
+    lib = load_library()
+    T, Hq, D = q_host.shape
+    Hkv = k_host.shape[1]
+    for name, t in (("q_host", q_host), ("k_host", k_host), ("v_host", v_host)):
+        if t.dtype != torch.bfloat16 or t.is_cuda or not t.is_contiguous() or t.dim() != 3:
+            raise ValueError(f"{name} must be a contiguous bf16 CPU tensor")
+    if v_host.shape != k_host.shape or k_host.shape[0] != T or k_host.shape[2] != D:
+        raise ValueError("k and v must be [tokens, kv_heads, head_dim] with q's tokens and head_dim")
+    cu = _cu_array(cu_seqlens)
+    if int(cu[-1]) != T:
+        raise ValueError(f"cu_seqlens[-1]={int(cu[-1])} does not match {T} tokens")
+    if scale is None:
+        scale = D ** -0.5
+    dev = torch.device("cuda", torch.cuda.current_device())
+    bufs = dict(device_buffers or {})
+    shapes = {"q": ((T, Hq, D), torch.bfloat16), "k": ((T, Hkv, D), torch.bfloat16),
+              "v": ((T, Hkv, D), torch.bfloat16), "out": ((T, Hq, D), torch.bfloat16),
+              "lse": ((T, Hq), torch.float32)}
+    if sinks_host is not None:
+        if sinks_host.dtype != torch.float32 or sinks_host.is_cuda or sinks_host.numel() != Hq:
+            raise ValueError("sinks_host must be an fp32 CPU tensor of Hq values")
+        sinks_host = sinks_host.contiguous()
+        shapes["sinks"] = ((Hq,), torch.float32)
+    for name, (shape, dtype) in shapes.items():
+        if name not in bufs:
+            bufs[name] = torch.empty(shape, dtype=dtype, device=dev)
+        t = bufs[name]
+        if tuple(t.shape) != shape or t.dtype != dtype or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"device buffer {name} must be a contiguous CUDA {dtype} tensor {shape}")
+    if out_host is None:
+        out_host = torch.empty((T, Hq, D), dtype=torch.bfloat16, pin_memory=True)
+    if lse_host is None:
+        lse_host = torch.empty((T, Hq), dtype=torch.float32, pin_memory=True)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    rc = lib.thd_attn_fwd_host(
+        q_host.data_ptr(), k_host.data_ptr(), v_host.data_ptr(),
+        cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), cu.size - 1, Hq, Hkv, D, int(window),
+        float(scale), sinks_host.data_ptr() if sinks_host is not None else None,
+        out_host.data_ptr(), lse_host.data_ptr(), bufs["q"].data_ptr(), bufs["k"].data_ptr(),
+        bufs["v"].data_ptr(), bufs["sinks"].data_ptr() if sinks_host is not None else None,
+        bufs["out"].data_ptr(), bufs["lse"].data_ptr(), int(n_chunks),
+        ctypes.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise ThdAttnError(rc, "thd_attn_fwd_host")
+    return out_host, lse_host
 
 
 def thd_attn_plan_range(cu_seqlens, q_begin: int, q_end: int, Hq: int, Hkv: int, D: int,

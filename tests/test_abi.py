@@ -194,3 +194,27 @@ def test_sparse_mla_workspace_size(lib):
     lib.thd_sparse_mla_workspace_bytes.restype = ctypes.c_size_t
     # latent 10*128*512*2, indices 10*64*4 -> 2560 (256-aligned), counts 40 -> 256
     assert lib.thd_sparse_mla_workspace_bytes(10, 128, 64) == 1310720 + 2560 + 256
+
+
+def _host(lib, cu=(0, 5, 9), n_chunks=4, sinks_h=None, sinks_d=None, q_h=0x10000, out_d=0x20000):
+    lib.thd_attn_fwd_host.argtypes = [ctypes.c_void_p] * 3 + [ctypes.POINTER(ctypes.c_int32)] + \
+        [ctypes.c_int] * 5 + [ctypes.c_float] + [ctypes.c_void_p] * 9 + [ctypes.c_int, ctypes.c_void_p]
+    arr = (ctypes.c_int32 * len(cu))(*cu)
+    p = 0x30000
+    return lib.thd_attn_fwd_host(q_h, p, p, arr, len(cu) - 1, 4, 2, 64, 0, 0.125, sinks_h, p, p,
+                                 p, p, p, sinks_d, out_d, p, n_chunks, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n_chunks=0), -1),
+    (dict(n_chunks=65), -1),
+    (dict(sinks_h=0x40000), -1),          # host sinks without device sinks
+    (dict(sinks_d=0x40000), -1),          # device sinks without host sinks
+    (dict(cu=(1, 5, 9)), -1),             # cu_seqlens must start at 0
+    (dict(cu=(0, 5, 3)), -1),             # and not decrease
+    (dict(q_h=None), -1),
+    (dict(out_d=None), -1),
+    (dict(cu=(0, 0, 0)), 0),              # nothing to do
+])
+def test_host_pipeline_rejects_bad_arguments_before_any_cuda_call(lib, kw, code):
+    assert _host(lib, **kw) == code
