@@ -357,6 +357,22 @@ int thd_sparse_mla_get_error(void* stream);
 /* ABI version of this header: (major << 16) | minor. */
 int thd_attn_abi_version(void);
 
+/*
+ * Self-test of the stall detector that guards every wait in the kernels (no
+ * fault, trap or unbounded wait is involved).  Launches two 32-thread blocks
+ * on a private stream and waits for them (about 2.5 s): block 0 waits on a
+ * barrier that nothing signals, with the kernels' own bounded wait, which
+ * gives up after its 2 s limit and records THD_ERR_TIMEOUT in the device
+ * status word; block 1 starts waiting 0.5 s later and gives up as soon as it
+ * sees that status.  waited_ns (host, [2]) receives how long each block
+ * waited (-1 if a wait was satisfied, which never happens).  Afterwards
+ * thd_attn_get_error returns THD_ERR_TIMEOUT once.  Returns
+ * THD_ERR_INVALID_ARG for a NULL waited_ns (before any CUDA call), an
+ * earlier unread status unchanged without launching, THD_ERR_CUDA if the
+ * launch fails.
+ */
+int thd_attn_selftest_stall(int64_t* waited_ns);
+
 #ifdef __cplusplus
 }
 #endif

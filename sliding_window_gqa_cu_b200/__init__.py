@@ -23,7 +23,7 @@ import numpy as np
 __all__ = ["thd_attn_fwd", "thd_attn_fwd_noalloc", "thd_attn_fwd_range", "thd_attn_fwd_host",
            "thd_attn_bwd", "thd_attn_bwd_workspace_bytes", "thd_qk_norm_rope",
            "thd_sparse_mla_fwd", "thd_sparse_mla_workspace_bytes", "thd_sparse_mla_get_error",
-           "thd_attn_get_error", "thd_attn_plan", "thd_attn_plan_range",
+           "thd_attn_get_error", "thd_attn_selftest_stall", "thd_attn_plan", "thd_attn_plan_range",
            "ThdAttnError", "library_path", "load_library", "STATUS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -88,6 +88,8 @@ def load_library():
     lib.thd_attn_fwd_host.argtypes = [vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int,
                                       ctypes.c_float, vp, vp, vp, vp, vp, vp, vp, vp, vp, c_int, vp]
     lib.thd_attn_fwd_host.restype = c_int
+    lib.thd_attn_selftest_stall.argtypes = [ctypes.POINTER(ctypes.c_int64)]
+    lib.thd_attn_selftest_stall.restype = c_int
     lib.thd_attn_plan_range.argtypes = [i32p, c_int, ctypes.c_int64, ctypes.c_int64, c_int, c_int,
                                         c_int, c_int, vp, ctypes.c_int64,
                                         ctypes.POINTER(ctypes.c_int64)]
@@ -479,6 +481,18 @@ def thd_sparse_mla_get_error(stream=None) -> int:
     if stream is None:
         stream = torch.cuda.current_stream()
     return int(load_library().thd_sparse_mla_get_error(ctypes.c_void_p(stream.cuda_stream)))
+
+
+def thd_attn_selftest_stall() -> tuple:
+    """Runs the stall-detector self-test (about 2.5 s; see thd_attn.h) and
+    returns how long its two blocks waited, in ns.  Afterwards
+    :func:`thd_attn_get_error` returns the timeout status once."""
+    lib = load_library()
+    w = (ctypes.c_int64 * 2)()
+    rc = lib.thd_attn_selftest_stall(w)
+    if rc != 0:
+        raise ThdAttnError(rc, "thd_attn_selftest_stall")
+    return int(w[0]), int(w[1])
 
 
 def thd_attn_get_error(stream=None) -> int:

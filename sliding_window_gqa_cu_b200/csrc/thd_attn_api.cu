@@ -290,11 +290,59 @@ int launch_bwd(DeviceState* ds, const BwdPlanEntry& plan, const CUtensorMap& mq,
     return cudaGetLastError() == cudaSuccess ? THD_OK : THD_ERR_CUDA;
 }
 
+// Stall-detector self-test: block 0 waits on an mbarrier that nothing
+// signals, with the kernels' own bounded wait, and gives up after its limit,
+// recording THD_ERR_TIMEOUT in the status word; block 1 starts waiting half a
+// second later and must give up as soon as it sees that status, before its
+// own limit runs out.  Plain waits on the wall clock: nothing faults or hangs.
+__device__ long long g_selftest_waited[2];
+
+__global__ void __launch_bounds__(32) thd_stall_selftest_kernel(int* status) {
+    __shared__ __align__(8) uint64_t bar_storage;
+    __shared__ int abort_flag;
+    const uint32_t bar = thd::smem_addr(&bar_storage);
+    if (threadIdx.x == 0) {
+        thd::mbar_init(bar, 1);
+        abort_flag = 0;
+        thd::fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        if (blockIdx.x == 1) thd::spin_ns(500000000ull);
+        const uint64_t t0 = thd::global_timer_ns();
+        const bool ok = thd::mbar_wait(bar, 0, &abort_flag, status, thd::kStatusTimeout);
+        g_selftest_waited[blockIdx.x] = ok ? -1 : static_cast<long long>(thd::global_timer_ns() - t0);
+    }
+}
+
 }  // namespace
 
 extern "C" {
 
 int thd_attn_abi_version(void) { return (1 << 16) | 1; }
+
+int thd_attn_selftest_stall(int64_t* waited_ns) {
+    if (waited_ns == nullptr) return THD_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState* ds = nullptr;
+    int rc = device_state(&ds, nullptr);
+    if (rc != THD_OK) return rc;
+    int status = 0;
+    if (cudaMemcpy(&status, ds->d_status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return THD_ERR_CUDA;
+    if (status != 0) return status;  // an earlier error is still unread
+    cudaStream_t s = nullptr;
+    if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return THD_ERR_CUDA;
+    thd_stall_selftest_kernel<<<2, 32, 0, s>>>(ds->d_status);
+    long long w[2] = {0, 0};
+    const bool good = cudaGetLastError() == cudaSuccess && cudaStreamSynchronize(s) == cudaSuccess &&
+                      cudaMemcpyFromSymbol(w, g_selftest_waited, sizeof(w)) == cudaSuccess;
+    cudaStreamDestroy(s);
+    if (!good) return THD_ERR_CUDA;
+    waited_ns[0] = w[0];
+    waited_ns[1] = w[1];
+    return THD_OK;
+}
 
 const char* thd_attn_status_string(int status) {
     switch (status) {

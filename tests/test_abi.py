@@ -218,3 +218,8 @@ def _host(lib, cu=(0, 5, 9), n_chunks=4, sinks_h=None, sinks_d=None, q_h=0x10000
 ])
 def test_host_pipeline_rejects_bad_arguments_before_any_cuda_call(lib, kw, code):
     assert _host(lib, **kw) == code
+
+
+def test_stall_selftest_rejects_null_before_any_cuda_call(lib):
+    lib.thd_attn_selftest_stall.argtypes = [ctypes.c_void_p]
+    assert lib.thd_attn_selftest_stall(None) == -1
