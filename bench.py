@@ -94,7 +94,7 @@ def measured_peaks():
 
 # Sources that decide the forward kernels' DRAM traffic: the kernels and the
 # schedule (item order).  Host-only entry-point code is not part of it.
-E2E_CHUNKS = 8  # token ranges of the end-to-end call (copies overlap the attention)
+E2E_CHUNKS = 16  # token ranges of the end-to-end call (copies overlap the attention)
 
 TRAFFIC_SOURCES = ("sm100_ptx.cuh", "thd_attn_kernel.cuh", "thd_attn_split_kernel.cuh",
                    "scheduler.cpp", "scheduler.h")

@@ -176,8 +176,9 @@ int thd_attn_fwd_range(const void* q, const void* k, const void* v,
  *                            [Hq], NULL exactly when sinks_host is), owned by
  *                            the caller, used as staging; 16-byte aligned as
  *                            thd_attn_fwd requires
- *   n_chunks                 1 .. 64 (the schedule cache keeps 16 ranges, so
- *                            up to about 8 stays cached between calls)
+ *   n_chunks                 1 .. 64 (each range has its own cached schedule;
+ *                            the cache keeps 40, so up to about 32 ranges
+ *                            stay cached between calls)
  * Asynchronous: returns once everything is queued; `stream` completes after
  * the last device-to-host copy, so synchronising it makes out_host and
  * lse_host valid.  The host buffers must stay untouched until then.  Calls

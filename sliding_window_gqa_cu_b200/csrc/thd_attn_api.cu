@@ -73,7 +73,7 @@ struct DeviceState {
     std::list<BwdPlanEntry> bwd_plans;  // most recently used first
 };
 
-constexpr size_t kMaxPlans = 16;
+constexpr size_t kMaxPlans = 40;  // per direction; the host pipeline's ranges each take one
 
 std::mutex g_mu;
 std::unordered_map<int, DeviceState> g_devices;
