@@ -19,7 +19,7 @@
 //    and latent += P kv[:, quarter] (MN-major operand).  TMEM: Q 288
 //    columns + S / P 64 + the latent quarter 128 = 480 of 512, which is why
 //    the latent is split over four CTAs (each recomputes S: QK^T runs four
-//    times per token; see the design notes).  Online softmax as in the
+//    times per token).  Online softmax as in the
 //    attention forward (exp2 domain, lazy rescale).  Writes the normalised
 //    latent (bf16) to a workspace [T, H, 512].
 // 2. Projection (thd_sparse_mla_proj_kernel): per head a GEMM
