@@ -56,7 +56,9 @@ enum thd_status {
     THD_ERR_CUDA = -3,         /* a CUDA runtime/driver call failed */
     THD_ERR_TIMEOUT = -4,      /* a bounded wait inside the kernel ran out */
     THD_ERR_NO_MEMORY = -5,    /* the schedule cache could not be allocated */
-    THD_ERR_TOO_LARGE = -6     /* thd_attn_fwd_noalloc: the schedule exceeds its fixed scratch */
+    THD_ERR_TOO_LARGE = -6,    /* thd_attn_fwd_noalloc: the schedule exceeds its fixed scratch */
+    THD_ERR_STALE_SCRATCH = -7 /* thd_attn_fwd_noalloc: a launch found another call's schedule
+                                  in the shared scratch and did nothing */
 };
 
 /*
@@ -158,8 +160,10 @@ int thd_attn_fwd_range(const void* q, const void* k, const void* v,
 
 /*
  * The forward from HOST buffers, with the copies overlapped with the
- * attention ("API" section of the sliding-window attention page: the same
- * packed-THD forward as thd_attn_fwd).  The pack is split into n_chunks
+ * attention.  The pages have no counterpart of this entry point: it computes
+ * the same packed-THD forward as thd_attn_fwd (MuseMagiPlan.attention,
+ * "muse_spark.magi_cp" page) for callers whose tensors live in host memory.
+ * The pack is split into n_chunks
  * token ranges of equal length; range c's q / k / v rows are copied to the
  * device on a copy stream, its query rows are computed as thd_attn_fwd_range
  * does on `stream` once they have landed (they read only key rows of their
@@ -213,25 +217,32 @@ int thd_attn_plan_range(const int32_t* cu_seqlens, int n_docs, int64_t q_begin, 
  *
  * Arguments and results are those of thd_attn_fwd, plus
  *   device_status_or_null  optional caller-owned device int.  If given, a
- *              kernel stall is recorded there as THD_ERR_TIMEOUT (the caller
- *              zeroes it; while it is non-zero, launches skip their work).
- *              If NULL, the scratch's own status word is used and cleared
- *              before each launch.
+ *              kernel stall (THD_ERR_TIMEOUT) or a stale schedule
+ *              (THD_ERR_STALE_SCRATCH) is recorded there; the caller zeroes
+ *              it, and while it is non-zero, launches skip their work.  If
+ *              NULL, the scratch's own status word is used: it keeps the
+ *              first error until thd_attn_noalloc_get_error reads and clears
+ *              it, and while it is non-zero, launches skip their work.
  *
  * Scratch: a fixed array inside the library's device image (one per GPU that
- * loads the library, kept until the process exits) holds a 256-byte status
- * header and up to 65,536 work items (2 MiB + 256 B).  A schedule needs
- * ceil(len/128) items per document per query-head pair (per query head when
- * Hq/Hkv is odd or D == 256); larger schedules return THD_ERR_TOO_LARGE
- * before anything is enqueued.  No call allocates device or host heap memory
- * (no cudaMalloc, cudaFree or allocating library routine).
+ * loads the library, kept until the process exits) holds a 256-byte header
+ * (status word and schedule tag) and up to 65,536 work items (2 MiB + 256 B).
+ * A schedule needs ceil(len/128) items per document per query-head pair (per
+ * query head when Hq/Hkv is odd or D == 256); larger schedules return
+ * THD_ERR_TOO_LARGE before anything is enqueued.  No call allocates device
+ * or host heap memory (no cudaMalloc, cudaFree or allocating library
+ * routine).
  *
  * The first call on a device does the set-up (looks up the scratch's device
- * address and clears its status header, synchronously): make that first call
+ * address and clears its header, synchronously): make that first call
  * before any stream capture.  Every call shares the scratch and it keeps the
- * last call's contents: the schedule is re-uploaded only when the arguments
- * change.  Calls that overlap on the GPU (for example on two streams of one
- * device) race on the scratch; serialise them.
+ * last call's contents: the schedule is re-uploaded, with a new tag, only
+ * when the arguments differ from the previous call's on this device.  Each
+ * launch checks on the GPU that the scratch still holds the schedule it was
+ * enqueued for; if another call's schedule is there, it records
+ * THD_ERR_STALE_SCRATCH and writes nothing.  Calls that overlap on the GPU
+ * (for example on two streams of one device) race on the scratch; serialise
+ * them.
  */
 int thd_attn_fwd_noalloc(const void* q, const void* k, const void* v,
                          const int32_t* cu_seqlens, int n_docs,
@@ -240,6 +251,15 @@ int thd_attn_fwd_noalloc(const void* q, const void* k, const void* v,
                          void* out, float* lse,
                          int* device_status_or_null,
                          void* stream);
+
+/*
+ * Status of thd_attn_fwd_noalloc calls that used the scratch's own status
+ * word (device_status_or_null == NULL): synchronises `stream`, returns the
+ * first error recorded since the last read (THD_OK if none, or if no call
+ * has run on this device yet) and clears it.  Allocates nothing.  Returns
+ * THD_ERR_CUDA if the synchronisation or the read fails.
+ */
+int thd_attn_noalloc_get_error(void* stream);
 
 /*
  * ------------------------------------------------------------------ backward

@@ -23,7 +23,7 @@ import numpy as np
 __all__ = ["thd_attn_fwd", "thd_attn_fwd_noalloc", "thd_attn_fwd_range", "thd_attn_fwd_host",
            "thd_attn_bwd", "thd_attn_bwd_workspace_bytes", "thd_qk_norm_rope",
            "thd_sparse_mla_fwd", "thd_sparse_mla_workspace_bytes", "thd_sparse_mla_get_error",
-           "thd_attn_get_error", "thd_attn_selftest_stall", "thd_attn_plan", "thd_attn_plan_range",
+           "thd_attn_get_error", "thd_attn_noalloc_get_error", "thd_attn_selftest_stall", "thd_attn_plan", "thd_attn_plan_range",
            "ThdAttnError", "library_path", "load_library", "STATUS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -31,7 +31,8 @@ _LIB_NAME = "libthdattn.so"
 _lib = None
 
 STATUS = {0: "THD_OK", -1: "THD_ERR_INVALID_ARG", -2: "THD_ERR_UNSUPPORTED", -3: "THD_ERR_CUDA",
-          -4: "THD_ERR_TIMEOUT", -5: "THD_ERR_NO_MEMORY", -6: "THD_ERR_TOO_LARGE"}
+          -4: "THD_ERR_TIMEOUT", -5: "THD_ERR_NO_MEMORY", -6: "THD_ERR_TOO_LARGE",
+          -7: "THD_ERR_STALE_SCRATCH"}
 
 WORK_ITEM_FIELDS = ("q0", "q1", "doc_start", "head0", "kv_start", "n_kv", "n_heads", "block_n")
 
@@ -77,6 +78,8 @@ def load_library():
     lib.thd_attn_fwd_noalloc.argtypes = [vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int,
                                          ctypes.c_float, vp, vp, vp, vp, vp]
     lib.thd_attn_fwd_noalloc.restype = c_int
+    lib.thd_attn_noalloc_get_error.argtypes = [vp]
+    lib.thd_attn_noalloc_get_error.restype = c_int
     lib.thd_attn_bwd_workspace_bytes.argtypes = [ctypes.c_int64, c_int]
     lib.thd_attn_bwd_workspace_bytes.restype = ctypes.c_size_t
     lib.thd_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int,
@@ -513,7 +516,8 @@ def thd_attn_fwd_noalloc(q, k, v, cu_seqlens, out, lse=None, window: int = 0,
     ``device_status`` word) and the library uses only a fixed scratch array
     compiled into its device image.  This wrapper allocates nothing either.
     The first call on a device does a one-time synchronous set-up; calls that
-    overlap on the GPU share the scratch and must be serialised.
+    overlap on the GPU share the scratch and must be serialised.  Without
+    ``device_status``, errors are read with :func:`thd_attn_noalloc_get_error`.
     """
     import torch
 
@@ -537,3 +541,12 @@ def thd_attn_fwd_noalloc(q, k, v, cu_seqlens, out, lse=None, window: int = 0,
     if rc != 0:
         raise ThdAttnError(rc, "thd_attn_fwd_noalloc")
     return out, lse
+
+
+def thd_attn_noalloc_get_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the status word of the
+    allocation-free entry point's scratch."""
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(load_library().thd_attn_noalloc_get_error(ctypes.c_void_p(stream.cuda_stream)))

@@ -127,7 +127,28 @@ struct FwdParams {
     int window;
     float scale_log2;    // scale * log2(e)
     int q_offset;        // pack row of row 0 of q / out / lse (0 unless a token range)
+    // Optional schedule check (allocation-free entry point): when set, the
+    // launch runs only if *plan_tag equals expected_tag, i.e. the shared
+    // scratch still holds the schedule this launch was enqueued for.
+    const unsigned long long* plan_tag = nullptr;
+    unsigned long long expected_tag = 0;
 };
+
+// Error code recorded when a launch finds another call's schedule in the
+// allocation-free scratch (the launch then does nothing).
+constexpr int kStatusStaleScratch = -7;
+
+// CTA start-up decision, taken by one thread: skip the work if an earlier
+// CTA or launch recorded an error that the host has not read yet, or if the
+// schedule this launch was enqueued for is no longer in place.
+__device__ __forceinline__ int launch_should_skip(const FwdParams& p) {
+    if (p.plan_tag != nullptr &&
+        *reinterpret_cast<const volatile unsigned long long*>(p.plan_tag) != p.expected_tag) {
+        atomicCAS(p.status, 0, kStatusStaleScratch);
+        return 1;
+    }
+    return *reinterpret_cast<volatile int*>(p.status) != 0 ? 1 : 0;
+}
 
 // Wait by lane 0 of the calling warp; the result is broadcast to the warp so
 // that the warp-collective tcgen05 instructions after it stay convergent.
@@ -215,7 +236,7 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         mbar_init(bar(C::B_DRAIN), 1);
         // A timeout recorded by an earlier CTA (or launch) makes every later
         // CTA skip its work until the host reads and clears the status.
-        *abort_flag = *reinterpret_cast<volatile int*>(p.status) != 0 ? 1 : 0;
+        *abort_flag = launch_should_skip(p);
         fence_barrier_init();
     }
     if (warp == C::MMA_WARP) {

@@ -10,13 +10,18 @@
 // of this library's device image, so no call allocates anything.
 //
 // Scratch: one file-scope static __device__ array per GPU that loads the
-// library, held until the process exits.  Layout: bytes [0, 256) hold the
-// status word, then up to kMaxItems work items of 32 bytes (2 MiB + 256 B in
-// total).  Every call shares it and it keeps the last call's contents: the
-// schedule is re-uploaded only when the arguments change, and the status
-// word is cleared (stream-ordered) before each launch unless the caller
-// supplies its own status word.  Calls that overlap on the GPU (e.g. on two
-// streams of one device) race on this array.
+// library, held until the process exits.  Layout: bytes [0, 4) hold the
+// status word, bytes [128, 136) the tag of the schedule in place, then from
+// byte 256 up to kMaxItems work items of 32 bytes (2 MiB + 256 B in total).
+// Every call shares it and it keeps the last call's contents: the schedule
+// (with a new tag) is re-uploaded only when the arguments change, and every
+// launch checks that the tag it was enqueued with is still in place, so a
+// launch that would read another call's schedule records an error and does
+// nothing instead.  The status word is kept until
+// thd_attn_noalloc_get_error reads and clears it (while it is non-zero,
+// launches skip their work), unless the caller supplies its own status word.
+// Calls that overlap on the GPU (e.g. on two streams of one device) race on
+// this array.
 //
 // Host side: the schedule is built into a static host array and sorted in
 // place; no heap memory is taken either.
@@ -27,6 +32,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <cstddef>
 #include <cstring>
 #include <mutex>
 
@@ -40,6 +46,7 @@ namespace {
 
 constexpr int64_t kMaxItems = 65536;
 constexpr size_t kHeaderBytes = 256;
+constexpr size_t kTagOffset = 128;  // the schedule's tag, uploaded with the items
 constexpr size_t kScratchBytes = kHeaderBytes + kMaxItems * sizeof(thd::WorkItem);
 constexpr int kMaxDevices = 64;
 constexpr int kMaxCachedDocs = 4096;  // boundaries remembered to skip re-uploads
@@ -55,11 +62,23 @@ struct NoAllocDevice {
     int n_docs = 0, Hq = 0, Hkv = 0, D = 0, window = 0;
     int32_t cu[kMaxCachedDocs + 1];
     int64_t n_items = 0;
+    unsigned long long tag = 0;       // tag of the schedule now in the scratch
+    unsigned long long next_tag = 1;  // every upload gets a new one
 };
+
+// Host image of the scratch from byte kTagOffset on: the tag, padding to
+// byte kHeaderBytes, then the work items; one copy uploads tag and items.
+struct HostUpload {
+    unsigned long long tag;
+    unsigned char pad[kHeaderBytes - kTagOffset - sizeof(unsigned long long)];
+    thd_work_item items[kMaxItems];
+};
+static_assert(offsetof(HostUpload, items) == kHeaderBytes - kTagOffset, "upload layout");
 
 std::mutex g_mu;
 NoAllocDevice g_dev[kMaxDevices];
-thd_work_item g_host_items[kMaxItems];
+HostUpload g_upload;
+thd_work_item* const g_host_items = g_upload.items;
 
 using NCfg64x2 = thd::FwdConfig<64, 2, 1, 128, 8>;
 using NCfg64x1 = thd::FwdConfig<64, 1, 2, 128, 8>;
@@ -202,11 +221,14 @@ extern "C" int thd_attn_fwd_noalloc(const void* q, const void* k, const void* v,
     if (!same_plan) {
         write_plan(cu_seqlens, n_docs, Hq, Hkv, window, ks, n_items);
         st->have_plan = false;
+        g_upload.tag = st->next_tag++;
         // Pageable source: the call returns once the host array is staged,
         // so the next call may overwrite it.
-        if (cudaMemcpyAsync(d_items, g_host_items, sizeof(thd::WorkItem) * n_items,
+        if (cudaMemcpyAsync(st->scratch + kTagOffset, &g_upload,
+                            (kHeaderBytes - kTagOffset) + sizeof(thd::WorkItem) * n_items,
                             cudaMemcpyHostToDevice, stream) != cudaSuccess)
             return THD_ERR_CUDA;
+        st->tag = g_upload.tag;
         if (n_docs <= kMaxCachedDocs) {
             st->n_docs = n_docs;
             st->Hq = Hq;
@@ -219,11 +241,11 @@ extern "C" int thd_attn_fwd_noalloc(const void* q, const void* k, const void* v,
         }
     }
 
-    int* status = device_status_or_null;
-    if (status == nullptr) {
-        status = reinterpret_cast<int*>(st->scratch);
-        if (cudaMemsetAsync(status, 0, sizeof(int), stream) != cudaSuccess) return THD_ERR_CUDA;
-    }
+    // The scratch's own status word is not cleared here: an error stays
+    // recorded (and later launches skip their work) until
+    // thd_attn_noalloc_get_error reads it.
+    int* status = device_status_or_null != nullptr ? device_status_or_null
+                                                   : reinterpret_cast<int*>(st->scratch);
 
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, q, T, Hq, D, 128) ||
@@ -242,6 +264,8 @@ extern "C" int thd_attn_fwd_noalloc(const void* q, const void* k, const void* v,
     prm.window = window;
     prm.scale_log2 = scale * 1.4426950408889634f;
     prm.q_offset = 0;
+    prm.plan_tag = reinterpret_cast<const unsigned long long*>(st->scratch + kTagOffset);
+    prm.expected_tag = st->tag;
 
     if (ks.pair) return launch_pair<NSplitCfg256>(st, 5, n_items, mq, mk, mv, prm, stream);
     if (D == 64) {
@@ -253,4 +277,20 @@ extern "C" int thd_attn_fwd_noalloc(const void* q, const void* k, const void* v,
                           : launch<NCfg128x1>(st, 3, n_items, mq, mk, mv, prm, stream);
     }
     return launch<NCfg256x1>(st, 4, n_items, mq, mk, mv, prm, stream);
+}
+
+extern "C" int thd_attn_noalloc_get_error(void* stream_ptr) {
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return THD_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return THD_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return THD_ERR_UNSUPPORTED;
+    NoAllocDevice* st = &g_dev[dev];
+    if (!st->ready) return THD_OK;  // no launch on this device yet
+    int status = 0;
+    if (cudaMemcpy(&status, st->scratch, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return THD_ERR_CUDA;
+    if (status != 0 && cudaMemset(st->scratch, 0, sizeof(int)) != cudaSuccess) return THD_ERR_CUDA;
+    return status;
 }

@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_abi_version_and_status_strings(lib):
     assert lib.thd_attn_abi_version() >> 16 == 1
-    for code in (0, -1, -2, -3, -4, -5):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7):
         assert lib.thd_attn_status_string(code) not in (None, b"", b"unknown status")
     assert lib.thd_attn_status_string(7) == b"unknown status"
 
