@@ -8,19 +8,26 @@ TFLOP/s over valid (unmasked) query-key pairs, FLOP = 4 * pairs * D * Hq.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
-``--pass bwd`` times the backward (thd_attn_bwd: dq, dk, dv, dsink) on the
-same pack instead, FLOP = 2.5x the forward's (the usual count of a backward
-that recomputes P); ``--pass prologue`` times the in-place Q/K prologue
-(thd_qk_norm_rope), bytes = Q and K read and written once; ``--pass
-sparse_mla`` times sparse MLA (thd_sparse_mla_fwd) on its own synthetic
-workload (4,096 tokens, 128 heads, up to 2,048 selected keys, value dim
-128), FLOP = valid slots x heads x 2 x (576 + 512) + the value projection.
-Each prints one JSON line of the same shape with its own metric.
+The default run prints one JSON line whose headline (`value`) is that pack's
+forward, and which also carries, measured in the same run with the same
+steps and warm-up:
+  per_config  the forward on the other benchmark packs (8,192-token causal,
+              32,768-token window 4096, 131,072-token MQA document at D = 256)
+  passes      the backward (thd_attn_bwd: dq, dk, dv, dsink; FLOP = 2.5x the
+              forward's, the usual count of a backward that recomputes P) on
+              the 64k pack and on the 128k document, the in-place Q/K prologue
+              (thd_qk_norm_rope; bytes = Q and K read and written once), and
+              sparse MLA (thd_sparse_mla_fwd) on its own synthetic workload
+              (4,096 tokens, 128 heads, up to 2,048 selected keys, value dim
+              128; FLOP = valid slots x heads x 2 x (576 + 512) + the value
+              projection).
+``--no-extras`` leaves those out.  ``--pass bwd|prologue|sparse_mla`` prints
+one line for that pass alone (``--workload`` selects the pack).
 
-Prints one JSON line on stdout (rank 0).  Multi-GPU runs are launched with
-torchrun, one process per GPU; every rank runs its own pack of the same shape
-(no data-path collective), the timed region is bracketed by a barrier and a
-device synchronisation, and the time is the max over ranks.
+Multi-GPU runs are launched with torchrun, one process per GPU; every rank
+runs its own pack of the same shape (no data-path collective), the timed
+region is bracketed by a barrier and a device synchronisation, and the time is
+the max over ranks.
 """
 from __future__ import annotations
 
@@ -77,6 +84,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd", "prologue", "sparse_mla"],
                     default="fwd", help="what one step runs (default: the forward, the headline)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="headline only: leave out per_config and passes")
     return ap.parse_args(argv)
 
 
@@ -259,6 +268,168 @@ def run_reference(args, info):
 
 # ------------------------------------------------------------------ GPU arm --
 
+EXTRA_CONFIGS = ("pack8k_gqa4_d128_causal", "pack32k_gqa4_d128_w4096", "doc128k_mqa_d256_w8192_sink")
+BWD_WORKLOADS = ("pack64k_gqa8_d128_causal_sink", "doc128k_mqa_d256_w8192_sink")
+
+
+def timed_loop(step, args, device, stream, label):
+    """W untimed steps, then K steps between a barrier and a device
+    synchronisation on both sides, with a CUDA event pair around every step
+    on the launching stream.  Returns (max-over-ranks ms of the K steps,
+    max-over-ranks mean ms per step, host start, host end)."""
+    for _ in range(args.warmup):
+        step()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    multirank.barrier(device)
+    torch.cuda.synchronize(device)
+    h0 = time.time()
+    torch.cuda.nvtx.range_push(label)
+    start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    end.record(stream)
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize(device)
+    h1 = time.time()
+    multirank.barrier(device)
+    total = multirank.max_over_ranks(start.elapsed_time(end), device)
+    per = multirank.max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ev), device)
+    return total, per, h0, h1
+
+
+def check_status(swa, stream, what):
+    status = swa.thd_attn_get_error(stream)
+    if status != 0:
+        raise RuntimeError(f"{what}: kernel reported status {status}")
+
+
+def fwd_case(swa, cfg, args, info, device, stream, T_override=None):
+    """Device tensors of one pack and a step that runs its forward."""
+    pack = workloads.make_pack(cfg, args.seed, tensor_seed=multirank.tensor_seed(args.seed, info.rank),
+                               T_override=T_override)
+    cu = pack["cu_seqlens"]
+    q, k, v = (pack[n].to(device) for n in "qkv")
+    sinks = pack["sinks"].to(device) if pack["sinks"] is not None else None
+    T = pack["T"]
+    out = torch.empty((T, cfg.Hq, cfg.D), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((T, cfg.Hq), dtype=torch.float32, device=device)
+
+    def step():
+        swa.thd_attn_fwd(q, k, v, cu, cfg.window, cfg.scale, sinks, out=out, lse=lse, stream=stream)
+    return pack, dict(q=q, k=k, v=v, sinks=sinks, out=out, lse=lse), step
+
+
+def summarise(ms_total, per_ms, args, work, unit, peak, peaks, clocks_sum, kernel, extra=None):
+    scale = 1e12 if unit == "TFLOP/s" else 1e9
+    achieved = work / (per_ms / 1e3) / scale
+    d = {"ms_per_step": ms_total / args.steps, "value": work * args.steps / (ms_total / 1e3) / scale,
+         "unit": unit, "frac": achieved / peak, "peak": peak, "kernel": kernel,
+         "clocks": {k: clocks_sum.get(k) for k in ("sm_mhz", "sm_max_mhz", "reasons")}}
+    if unit == "TFLOP/s":
+        d["frac_of_sustained"] = achieved / float(peaks.get("bf16_tflops_sustained", peak))
+    if extra:
+        d.update(extra)
+    return d
+
+
+def measure_fwd_extra(swa, name, args, info, device, stream, clocks, peaks):
+    cfg = workloads.CONFIGS[name]
+    pack, _, step = fwd_case(swa, cfg, args, info, device, stream)
+    pairs = metrics.valid_pairs(pack["cu_seqlens"], cfg.window)
+    flops = 4 * pairs * cfg.D * cfg.Hq
+    step()
+    check_status(swa, stream, name)
+    tot, per, h0, h1 = timed_loop(step, args, device, stream, f"thd_attn_fwd {name}")
+    check_status(swa, stream, name)
+    peak = float(peaks["bf16_tflops"])
+    return summarise(tot, per, args, flops * info.world, UNIT, peak * info.world, peaks,
+                     clocks.summary(h0, h1), kernel_name(cfg.D, cfg.Hq // cfg.Hkv),
+                     {"valid_pairs": int(pairs), "tokens": pack["T"], "gflop_per_step": flops / 1e9,
+                      "traffic": traffic_per_launch(name)})
+
+
+def measure_bwd(swa, name, args, info, device, stream, clocks, peaks):
+    cfg = workloads.CONFIGS[name]
+    pack, t, _ = fwd_case(swa, cfg, args, info, device, stream, T_override=args.tokens)
+    cu, T = pack["cu_seqlens"], pack["T"]
+    pairs = metrics.valid_pairs(cu, cfg.window)
+    out, lse = swa.thd_attn_fwd(t["q"], t["k"], t["v"], cu, cfg.window, cfg.scale, t["sinks"],
+                                stream=stream)
+    g = torch.Generator(device="cpu").manual_seed(7)
+    dout = torch.randn((T, cfg.Hq, cfg.D), generator=g).to(torch.bfloat16).to(device)
+    ws = torch.empty((max(16, swa.thd_attn_bwd_workspace_bytes(T, cfg.Hq)),), dtype=torch.uint8,
+                     device=device)
+    dq, dk, dv = torch.empty_like(t["q"]), torch.empty_like(t["k"]), torch.empty_like(t["v"])
+    work = 2.5 * 4 * pairs * cfg.D * cfg.Hq
+
+    def step():
+        swa.thd_attn_bwd(t["q"], t["k"], t["v"], out, lse, dout, cu, cfg.window, cfg.scale,
+                         t["sinks"], dq=dq, dk=dk, dv=dv, workspace=ws, stream=stream)
+    step()
+    check_status(swa, stream, f"bwd {name}")
+    tot, per, h0, h1 = timed_loop(step, args, device, stream, f"thd_attn_bwd {name}")
+    check_status(swa, stream, f"bwd {name}")
+    peak = float(peaks["bf16_tflops"])
+    return summarise(tot, per, args, work * info.world, UNIT, peak * info.world, peaks,
+                     clocks.summary(h0, h1), "thd_attn_bwd_dq_kernel + thd_attn_bwd_dkdv_kernel",
+                     {"workload": name, "valid_pairs": int(pairs), "tokens": T,
+                      "launches_per_step": 4 if t["sinks"] is not None else 3,
+                      "metric": "THD varlen attention bwd TFLOP/s (valid pairs, 2.5x forward FLOP)"})
+
+
+def measure_prologue(swa, name, args, info, device, stream, clocks, peaks):
+    cfg = workloads.CONFIGS[name]
+    pack, t, _ = fwd_case(swa, cfg, args, info, device, stream, T_override=args.tokens)
+    cu, T = pack["cu_seqlens"], pack["T"]
+    work = 2 * T * (cfg.Hq + cfg.Hkv) * cfg.D * 2  # bytes: Q and K read and written once
+
+    def step():
+        swa.thd_qk_norm_rope(t["q"], t["k"], cu, stream=stream)
+    step()
+    check_status(swa, stream, "prologue")
+    tot, per, h0, h1 = timed_loop(step, args, device, stream, f"thd_qk_norm_rope {name}")
+    check_status(swa, stream, "prologue")
+    peak = float(peaks["hbm_gbs"])
+    return summarise(tot, per, args, work * info.world, "GB/s", peak * info.world, peaks,
+                     clocks.summary(h0, h1), "thd_qk_norm_rope_kernel",
+                     {"workload": name, "tokens": T, "bound": "hbm",
+                      "metric": "Q/K prologue (scaleless RMSNorm + split-half RoPE) GB/s"})
+
+
+SPARSE_MLA_WORKLOAD = dict(name="sparse_mla_t4096_h128_k2048_v128", lens=[4096], H=128, K=2048, vd=128)
+
+
+def measure_sparse_mla(swa, args, info, device, stream, clocks, peaks):
+    w = SPARSE_MLA_WORKLOAD
+    c = workloads.sparse_mla_case(args.seed + 7919 * info.rank, w["lens"], w["H"], w["K"], w["vd"])
+    q, kv, idx, wt = (c[n].to(device) for n in ("q", "kv", "indices", "value_weight"))
+    T, H, vd = c["T"], w["H"], w["vd"]
+    valid = int((c["indices"] >= 0).sum())
+    flop = valid * H * 2 * (576 + 512) + T * H * 512 * vd * 2
+    out = torch.empty((T, H, vd), dtype=torch.bfloat16, device=device)
+    ws = torch.empty((swa.thd_sparse_mla_workspace_bytes(T, H, w["K"]),), dtype=torch.uint8,
+                     device=device)
+
+    def step():
+        swa.thd_sparse_mla_fwd(q, kv, idx, wt, c["scale"], out=out, workspace=ws, stream=stream)
+    step()
+    if swa.thd_sparse_mla_get_error(stream) != 0:
+        raise RuntimeError("sparse MLA: kernel reported an error status")
+    tot, per, h0, h1 = timed_loop(step, args, device, stream, "thd_sparse_mla_fwd")
+    if swa.thd_sparse_mla_get_error(stream) != 0:
+        raise RuntimeError("sparse MLA: kernel reported an error status")
+    peak = float(peaks["bf16_tflops"])
+    return summarise(tot, per, args, flop * info.world, UNIT, peak * info.world, peaks,
+                     clocks.summary(h0, h1), "thd_sparse_mla_attn_kernel + thd_sparse_mla_proj_kernel",
+                     {"workload": w["name"], "tokens": T, "heads": H, "selected_keys": w["K"],
+                      "value_dim": vd, "valid_slots": valid, "launches_per_step": 2,
+                      "metric": "sparse MLA fwd TFLOP/s (valid slots, incl. value projection)"})
+
+
 def run_ours(args, info):
     import sliding_window_gqa_cu_b200 as swa
 
@@ -268,57 +439,26 @@ def run_ours(args, info):
     device = torch.device("cuda", info.local_rank)
     torch.cuda.set_device(device)
     swa.load_library()
+    stream = torch.cuda.current_stream(device)
+    peaks, peak_src = measured_peaks()
+    peak = float(peaks["bf16_tflops"])
 
     cfg = workloads.CONFIGS[args.workload]
-    pack = workloads.make_pack(cfg, args.seed, tensor_seed=multirank.tensor_seed(args.seed, info.rank),
-                               T_override=args.tokens)
-    cu = pack["cu_seqlens"]
-    T = pack["T"]
+    pack, t, step = fwd_case(swa, cfg, args, info, device, stream, T_override=args.tokens)
+    cu, T = pack["cu_seqlens"], pack["T"]
     pairs = metrics.valid_pairs(cu, cfg.window)
     flops = 4 * pairs * cfg.D * cfg.Hq
-    q, k, v = (pack[n].to(device) for n in "qkv")
-    sinks = pack["sinks"].to(device) if pack["sinks"] is not None else None
-    out = torch.empty((T, cfg.Hq, cfg.D), dtype=torch.bfloat16, device=device)
-    lse = torch.empty((T, cfg.Hq), dtype=torch.float32, device=device)
-    stream = torch.cuda.current_stream(device)
-
-    def step():
-        swa.thd_attn_fwd(q, k, v, cu, cfg.window, cfg.scale, sinks, out=out, lse=lse, stream=stream)
 
     t_plan0 = time.perf_counter()
     step()  # first call builds and uploads the tile schedule
     torch.cuda.synchronize(device)
     first_call_ms = (time.perf_counter() - t_plan0) * 1e3
-    status = swa.thd_attn_get_error(stream)
-    if status != 0:
-        raise RuntimeError(f"kernel reported status {status}")
+    check_status(swa, stream, cfg.name)
 
     clocks = ClockSampler(device)
-    for _ in range(args.warmup):
-        step()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    multirank.barrier(device)
-    torch.cuda.synchronize(device)
-    h0 = time.time()
-    start.record(stream)
-    for i in range(args.steps):
-        ev[i][0].record(stream)
-        step()
-        ev[i][1].record(stream)
-    end.record(stream)
-    torch.cuda.synchronize(device)
-    h1 = time.time()
-    multirank.barrier(device)
-    clocks.stop()
-    status = swa.thd_attn_get_error(stream)
-    if status != 0:
-        raise RuntimeError(f"kernel reported status {status}")
-    elapsed_ms = start.elapsed_time(end)
-    launch_ms = [a.elapsed_time(b) for a, b in ev]
-    max_ms = multirank.max_over_ranks(elapsed_ms, device)
-    max_launch = multirank.max_over_ranks(statistics.mean(launch_ms), device)
+    max_ms, max_launch, h0, h1 = timed_loop(step, args, device, stream, f"thd_attn_fwd {cfg.name}")
+    check_status(swa, stream, cfg.name)
+    csum = clocks.summary(h0, h1)
     value = multirank.aggregate_rate(flops * args.steps, info.world, max_ms / 1e3) / 1e12
 
     # end to end through the public API with pinned host buffers
@@ -326,14 +466,13 @@ def run_ours(args, info):
     if not args.no_e2e:
         qh, kh, vh = (pack[n].pin_memory() for n in "qkv")
         sh = pack["sinks"].pin_memory() if pack["sinks"] is not None else None
-        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        lh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh) + ((sh,) if sh is not None else ()))
+        oh = torch.empty(t["out"].shape, dtype=t["out"].dtype).pin_memory()
+        lh = torch.empty(t["lse"].shape, dtype=t["lse"].dtype).pin_memory()
+        h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh) + ((sh,) if sh is not None else ()))
         d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
-
-        bufs = {"q": q, "k": k, "v": v, "out": out, "lse": lse}
+        bufs = {n: t[n] for n in ("q", "k", "v", "out", "lse")}
         if sh is not None:
-            bufs["sinks"] = sinks
+            bufs["sinks"] = t["sinks"]
 
         def e2e_step():
             # host -> device copies, attention and device -> host copies of
@@ -351,14 +490,13 @@ def run_ours(args, info):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize(device)
+        check_status(swa, stream, "e2e")
         e2e_ms = multirank.max_over_ranks(e0.elapsed_time(e1), device)
         e2e = {"value": multirank.aggregate_rate(flops * args.e2e_steps, info.world, e2e_ms / 1e3) / 1e12,
                "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms / args.e2e_steps,
                "path": f"thd_attn_fwd_host, pinned host buffers, {E2E_CHUNKS} overlapped token ranges"}
 
-    peaks, peak_src = measured_peaks()
-    peak = float(peaks["bf16_tflops"])
     achieved = flops / (max_launch / 1e3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic_per_launch(cfg.name),
@@ -369,15 +507,41 @@ def run_ours(args, info):
                 "kernel": kernel_name(cfg.D, cfg.Hq // cfg.Hkv),
                 "algorithmic_flops_per_launch": flops,
                 "algorithmic_bytes_per_launch": metrics.algorithmic_bytes(T, cfg.Hq, cfg.Hkv, cfg.D)}
+    del pack, t, step
 
     cpu = None
     if info.is_root and info.world == 1 and not args.no_cpu_baseline:
-        tf, spent, rows, fl, threads = cpu_oracle_sample(pack, args.cpu_seconds, seed=12345)
+        cpack = workloads.make_pack(cfg, args.seed, T_override=args.tokens)
+        tf, spent, rows, fl, threads = cpu_oracle_sample(cpack, args.cpu_seconds, seed=12345)
         cpu = {"value": tf, "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": f"{rows} random (token, head) rows of the same pack, fp64, "
                          f"{fl / 1e9:.1f} GFLOP in {spent:.1f} s"}
+        del cpack
 
-    csum = clocks.summary(h0, h1)
+    per_config, passes = None, None
+    if not args.no_extras and args.tokens is None:
+        per_config = {}
+        for name in EXTRA_CONFIGS:
+            if name == cfg.name:
+                continue
+            per_config[name] = measure_fwd_extra(swa, name, args, info, device, stream, clocks, peaks)
+            torch.cuda.empty_cache()
+        passes = {}
+        for name in BWD_WORKLOADS:
+            try:
+                passes["bwd " + name] = measure_bwd(swa, name, args, info, device, stream, clocks,
+                                                    peaks)
+            except swa.ThdAttnError as e:  # a head dim the backward does not support
+                if e.code != -2:
+                    raise
+                passes["bwd " + name] = {"unsupported": str(e)}
+            torch.cuda.empty_cache()
+        passes["prologue " + DEFAULT_WORKLOAD] = measure_prologue(swa, DEFAULT_WORKLOAD, args, info,
+                                                                  device, stream, clocks, peaks)
+        torch.cuda.empty_cache()
+        passes["sparse_mla"] = measure_sparse_mla(swa, args, info, device, stream, clocks, peaks)
+    clocks.stop()
+
     if info.is_root:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": info.world,
@@ -390,20 +554,25 @@ def run_ours(args, info):
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps, "clocks": {k: csum[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
             "first_call_ms_with_schedule_build": first_call_ms,
+            "per_config": per_config, "passes": passes,
         }
         log(f"[bench] {cfg.name}: {max_ms / args.steps:.3f} ms/step, {value:.1f} TFLOP/s "
-            f"({100 * value / info.world / peak:.1f}% of measured {peak:.0f}, "
+            f"({100 * value / info.world / peak:.1f}% of {peak_src} {peak:.0f}, "
             f"{100 * value / info.world / DATASHEET_BF16_TFLOPS:.1f}% of 2250), clocks {csum}")
+        for group in (per_config or {}), (passes or {}):
+            for name, d in group.items():
+                if "unsupported" in d:
+                    log(f"[bench]   {name}: {d['unsupported']}")
+                    continue
+                log(f"[bench]   {name}: {d['ms_per_step']:.3f} ms/step, {d['value']:.1f} {d['unit']} "
+                    f"({100 * d['frac']:.1f}% of {d['peak'] / info.world:.0f}), clocks {d['clocks']}")
         print(json.dumps(line), flush=True)
     multirank.shutdown()
     return 0
 
 
-# ------------------------------------------------- backward and prologue --
-
 def run_other_pass(args, info):
-    """--pass bwd / prologue: device-timed steps of thd_attn_bwd or
-    thd_qk_norm_rope on the same synthetic pack (inputs resident in HBM)."""
+    """--pass bwd / prologue / sparse_mla: one line for that pass alone."""
     import sliding_window_gqa_cu_b200 as swa
 
     if not torch.cuda.is_available():
@@ -412,150 +581,37 @@ def run_other_pass(args, info):
     device = torch.device("cuda", info.local_rank)
     torch.cuda.set_device(device)
     swa.load_library()
-    if args.pass_ == "sparse_mla":
-        return run_sparse_mla(args, info, device)
-    cfg = workloads.CONFIGS[args.workload]
-    pack = workloads.make_pack(cfg, args.seed, tensor_seed=multirank.tensor_seed(args.seed, info.rank),
-                               T_override=args.tokens)
-    cu = pack["cu_seqlens"]
-    T = pack["T"]
-    pairs = metrics.valid_pairs(cu, cfg.window)
-    q, k, v = (pack[n].to(device) for n in "qkv")
-    sinks = pack["sinks"].to(device) if pack["sinks"] is not None else None
     stream = torch.cuda.current_stream(device)
     peaks, peak_src = measured_peaks()
-    if args.pass_ == "bwd":
-        out, lse = swa.thd_attn_fwd(q, k, v, cu, cfg.window, cfg.scale, sinks, stream=stream)
-        g = torch.Generator(device="cpu").manual_seed(7)
-        dout = torch.randn((T, cfg.Hq, cfg.D), generator=g).to(torch.bfloat16).to(device)
-        ws = torch.empty((max(16, swa.thd_attn_bwd_workspace_bytes(T, cfg.Hq)),), dtype=torch.uint8,
-                         device=device)
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        work = 2.5 * 4 * pairs * cfg.D * cfg.Hq
-        launches = 4 if sinks is not None else 3
-
-        def step():
-            swa.thd_attn_bwd(q, k, v, out, lse, dout, cu, cfg.window, cfg.scale, sinks, dq=dq, dk=dk,
-                             dv=dv, workspace=ws, stream=stream)
-        metric, unit = "THD varlen attention bwd TFLOP/s (valid pairs, 2.5x forward FLOP)", "TFLOP/s"
-        peak = float(peaks["bf16_tflops"])
-        bound, kern = "tensor", "thd_attn_bwd_dq_kernel + thd_attn_bwd_dkdv_kernel"
-    else:
-        work = 2 * T * (cfg.Hq + cfg.Hkv) * cfg.D * 2  # bytes: Q and K read and written once
-        launches = 1
-
-        def step():
-            swa.thd_qk_norm_rope(q, k, cu, stream=stream)
-        metric, unit = "Q/K prologue (scaleless RMSNorm + split-half RoPE) GB/s", "GB/s"
-        peak = float(peaks["hbm_gbs"])
-        bound, kern = "hbm", "thd_qk_norm_rope_kernel"
-    step()
-    torch.cuda.synchronize(device)
-    if swa.thd_attn_get_error(stream) != 0:
-        raise RuntimeError("kernel reported an error status")
     clocks = ClockSampler(device)
-    for _ in range(args.warmup):
-        step()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    multirank.barrier(device)
-    torch.cuda.synchronize(device)
-    h0 = time.time()
-    start.record(stream)
-    for _ in range(args.steps):
-        step()
-    end.record(stream)
-    torch.cuda.synchronize(device)
-    h1 = time.time()
-    multirank.barrier(device)
+    if args.pass_ == "bwd":
+        d = measure_bwd(swa, args.workload, args, info, device, stream, clocks, peaks)
+    elif args.pass_ == "prologue":
+        d = measure_prologue(swa, args.workload, args, info, device, stream, clocks, peaks)
+    else:
+        d = measure_sparse_mla(swa, args, info, device, stream, clocks, peaks)
     clocks.stop()
-    ms = multirank.max_over_ranks(start.elapsed_time(end), device)
-    scale = 1e12 if unit == "TFLOP/s" else 1e9
-    value = multirank.aggregate_rate(work * args.steps, info.world, ms / 1e3) / scale
-    achieved = work / (ms / args.steps / 1e3) / scale
-    csum = clocks.summary(h0, h1)
     if info.is_root:
+        cfg = workloads.CONFIGS[args.workload]
+        launches = d.pop("launches_per_step", 1)
         line = {
-            "metric": metric, "value": value, "unit": unit, "n_gpus": info.world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "metric": d.pop("metric"), "value": d["value"], "unit": d["unit"], "n_gpus": info.world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": d["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "pass": args.pass_,
-            "config": workload_config(cfg, cu, pairs, {"parallelism": f"pack-parallel x{info.world}"}),
-            "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                         "frac": achieved / peak, "traffic": None, "kernel": kern,
+            "config": ({"workload": d["workload"]} if args.pass_ == "sparse_mla" else
+                       workload_config(cfg, workloads.pack_cu_seqlens(cfg, args.seed) if args.tokens is None
+                                       else np.array([0, d["tokens"]]), d.get("valid_pairs", 0),
+                                       {"parallelism": f"pack-parallel x{info.world}"})),
+            "roofline": {"bound": d.get("bound", "tensor"), "achieved": d["frac"] * d["peak"] / info.world,
+                         "peak": d["peak"] / info.world, "unit": d["unit"], "frac": d["frac"],
+                         "traffic": None, "kernel": d["kernel"],
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json)"},
             "cpu_baseline": None, "e2e": None, "gpu_launches": launches * args.steps,
-            "clocks": {k: csum[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+            "clocks": d["clocks"],
         }
-        log(f"[bench] {cfg.name} {args.pass_}: {ms / args.steps:.3f} ms/step, {value:.1f} {unit} "
-            f"({100 * achieved / peak:.1f}% of measured {peak:.0f}), clocks {csum}")
-        print(json.dumps(line), flush=True)
-    multirank.shutdown()
-    return 0
-
-
-SPARSE_MLA_WORKLOAD = dict(name="sparse_mla_t4096_h128_k2048_v128", lens=[4096], H=128, K=2048, vd=128)
-
-
-def run_sparse_mla(args, info, device):
-    """--pass sparse_mla: device-timed thd_sparse_mla_fwd (attention + value
-    projection, two launches) on a synthetic one-document workload."""
-    import sliding_window_gqa_cu_b200 as swa
-
-    w = SPARSE_MLA_WORKLOAD
-    c = workloads.sparse_mla_case(args.seed + 7919 * info.rank, w["lens"], w["H"], w["K"], w["vd"])
-    q, kv, idx, wt = (c[n].to(device) for n in ("q", "kv", "indices", "value_weight"))
-    T, H, vd = c["T"], w["H"], w["vd"]
-    valid = int((c["indices"] >= 0).sum())
-    flop = valid * H * 2 * (576 + 512) + T * H * 512 * vd * 2
-    out = torch.empty((T, H, vd), dtype=torch.bfloat16, device=device)
-    ws = torch.empty((swa.thd_sparse_mla_workspace_bytes(T, H, w["K"]),), dtype=torch.uint8,
-                     device=device)
-    stream = torch.cuda.current_stream(device)
-
-    def step():
-        swa.thd_sparse_mla_fwd(q, kv, idx, wt, c["scale"], out=out, workspace=ws, stream=stream)
-    step()
-    if swa.thd_sparse_mla_get_error(stream) != 0:
-        raise RuntimeError("kernel reported an error status")
-    clocks = ClockSampler(device)
-    for _ in range(args.warmup):
-        step()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    multirank.barrier(device)
-    torch.cuda.synchronize(device)
-    h0 = time.time()
-    start.record(stream)
-    for _ in range(args.steps):
-        step()
-    end.record(stream)
-    torch.cuda.synchronize(device)
-    h1 = time.time()
-    multirank.barrier(device)
-    clocks.stop()
-    ms = multirank.max_over_ranks(start.elapsed_time(end), device)
-    value = multirank.aggregate_rate(flop * args.steps, info.world, ms / 1e3) / 1e12
-    achieved = flop / (ms / args.steps / 1e3) / 1e12
-    peaks, peak_src = measured_peaks()
-    peak = float(peaks["bf16_tflops"])
-    csum = clocks.summary(h0, h1)
-    if info.is_root:
-        line = {
-            "metric": "sparse MLA fwd TFLOP/s (valid slots, incl. value projection)", "value": value,
-            "unit": "TFLOP/s", "n_gpus": info.world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "pass": "sparse_mla",
-            "config": {"workload": w["name"], "tokens": T, "heads": H, "selected_keys": w["K"],
-                       "value_dim": vd, "valid_slots": valid,
-                       "l2": "inputs larger than L2 (q = %.2f GB), no flush" % (T * H * 576 * 2 / 1e9)},
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": None,
-                         "kernel": "thd_sparse_mla_attn_kernel + thd_sparse_mla_proj_kernel",
-                         "peak_source": f"{peak_src} (MEASURED_PEAKS.json)"},
-            "cpu_baseline": None, "e2e": None, "gpu_launches": 2 * args.steps,
-            "clocks": {k: csum[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
-        }
-        log(f"[bench] {w['name']}: {ms / args.steps:.3f} ms/step, {value:.1f} TFLOP/s "
-            f"({100 * achieved / peak:.1f}% of measured {peak:.0f}), clocks {csum}")
+        log(f"[bench] {args.pass_}: {d['ms_per_step']:.3f} ms/step, {d['value']:.1f} {d['unit']} "
+            f"({100 * d['frac']:.1f}% of {peak_src} {d['peak'] / info.world:.0f}), clocks {d['clocks']}")
         print(json.dumps(line), flush=True)
     multirank.shutdown()
     return 0

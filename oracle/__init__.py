@@ -9,9 +9,12 @@ Two independent formulations live here:
 * :func:`attention` / :func:`attention_rows` -- the plain fp64 loop over
   documents, heads and queries in ``thd_attn_oracle.c`` (see that file's
   header for the definition and the page passages it restates);
-* :func:`attention_bwd` / :func:`attention_bwd_q_rows` -- the fp64 gradient
-  of that forward (dq, dk, dv, dsink), the plain derivative written out in the
-  same C file;
+* :func:`attention_bwd` / :func:`attention_bwd_q_rows` /
+  :func:`attention_bwd_kv_rows` -- the fp64 gradient of that forward (dq, dk,
+  dv, dsink), the plain derivative written out in the same C file, for the
+  whole pack or for selected query rows (dq) or key rows (dk, dv);
+  :func:`attention_dsink` -- the sink gradient alone from the forward's
+  output and log-sum-exp;
 * :mod:`oracle.prologue` -- the Q/K prologue (scaleless RMSNorm, then
   split-half RoPE at per-document positions) in plain fp64 numpy;
 * :mod:`oracle.sparse_mla` -- sparse MLA over gathered latent KV with the
@@ -75,6 +78,10 @@ def _bind(lib):
     lib.oracle_thd_attn_bwd_q_rows.argtypes = [vp, vp, vp, vp, c_int, i32p, c_int, c_int, c_int,
                                                c_int, c_int, c_double, fp, i64p, ctypes.c_int64, dp]
     lib.oracle_thd_attn_bwd_q_rows.restype = c_int
+    lib.oracle_thd_attn_bwd_kv_rows.argtypes = [vp, vp, vp, vp, c_int, i32p, c_int, c_int, c_int,
+                                                c_int, c_int, c_double, fp, i64p, ctypes.c_int64,
+                                                dp, dp]
+    lib.oracle_thd_attn_bwd_kv_rows.restype = c_int
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = c_int
     return lib
@@ -221,6 +228,43 @@ def attention_bwd_q_rows(q, k, v, dout, cu_seqlens, window: int, scale: float, r
     if rc != 0:
         raise ValueError("oracle rejected its arguments")
     return out
+
+
+def attention_bwd_kv_rows(q, k, v, dout, cu_seqlens, window: int, scale: float, rows, sinks=None,
+                          lib=None):
+    """fp64 dk and dv for selected (key token, kv_head) rows ``rows`` [n, 2];
+    returns (dk [n, D], dv [n, D])."""
+    lib = lib or load()
+    qa, ka, va, dt, cu, T, Hq, Hkv, D = _common(q, k, v, cu_seqlens)
+    da = _dout(dout, dt)
+    s = _sinks(sinks)
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 2))
+    dk = np.zeros((r.shape[0], D))
+    dv = np.zeros((r.shape[0], D))
+    rc = lib.oracle_thd_attn_bwd_kv_rows(
+        qa.ctypes.data, ka.ctypes.data, va.ctypes.data, da.ctypes.data, dt,
+        cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), len(cu) - 1, Hq, Hkv, D,
+        int(window), float(scale),
+        s.ctypes.data_as(ctypes.POINTER(ctypes.c_float)) if s is not None else None,
+        r.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), r.shape[0],
+        dk.ctypes.data_as(ctypes.POINTER(ctypes.c_double)),
+        dv.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return dk, dv
+
+
+def attention_dsink(q, k, v, dout, cu_seqlens, window: int, scale: float, sinks, lib=None):
+    """fp64 sink gradient alone: dsink[h] = -sum_i exp(sink_h - lse[i,h]) *
+    D[i,h] with D[i,h] = sum_c dO[i,h,c] out[i,h,c], where out and lse are the
+    forward oracle's (:func:`attention`).  Returns [Hq]."""
+    out, lse = attention(q, k, v, cu_seqlens, window, scale, sinks, lib=lib)
+    da = _dout(dout, _as_input(q)[1])
+    if da.dtype == np.uint16:
+        da = _bits_to_f64(da)
+    Di = np.einsum("ihc,ihc->ih", da, out)
+    s = _sinks(sinks).astype(np.float64)
+    return -(np.exp(s[None, :] - lse) * Di).sum(0)
 
 
 def num_threads(lib=None) -> int:

@@ -339,6 +339,111 @@ int oracle_thd_attn_bwd_q_rows(const void *q, const void *k, const void *v, cons
     return 0;
 }
 
+/*
+ * dk and dv for selected (key token, kv head) rows only: rows[2r] = key j,
+ * rows[2r+1] = kv head g.  By the definition above,
+ *   dk[j,g] = scale * sum_{h in g} sum_{i : j in V(i)} dS_ij q[i,h],
+ *   dv[j,g] =         sum_{h in g} sum_{i : j in V(i)} P_ij dO[i,h],
+ * and the queries that see key j of document [s, e) are i in [j, e) with
+ * (W == 0 or i < j + W).  Each term needs the row quantities lse_i and D_i
+ * of its query row (i, h), which depend on the whole row; they are computed
+ * once per distinct row first (same formulas as row_probs and D_i above),
+ * then the per-pair terms are summed.  dk_rows, dv_rows: [n_rows, D].
+ */
+static int64_t last_query(int64_t j, int64_t e, int window) {
+    /* one past the last query that sees key j */
+    return (window > 0 && j + window < e) ? j + window : e;
+}
+
+int oracle_thd_attn_bwd_kv_rows(const void *q, const void *k, const void *v, const void *dout,
+                                int dtype, const int32_t *cu_seqlens, int n_docs, int Hq,
+                                int Hkv, int D, int window, double scale, const float *sinks,
+                                const int64_t *rows, int64_t n_rows, double *dk_rows,
+                                double *dv_rows) {
+    if (check_args(cu_seqlens, n_docs, Hq, Hkv, D, window)) return -1;
+    const int64_t T = n_docs > 0 ? cu_seqlens[n_docs] : 0;
+    for (int64_t r = 0; r < n_rows; r++)
+        if (rows[2 * r] < 0 || rows[2 * r] >= T || rows[2 * r + 1] < 0 || rows[2 * r + 1] >= Hkv)
+            return -1;
+    const int G = Hq / Hkv;
+    /* 1. mark the query rows (i, h) the requested keys need */
+    unsigned char *need = (unsigned char *)calloc((size_t)(T * Hq > 0 ? T * Hq : 1), 1);
+    for (int64_t r = 0; r < n_rows; r++) {
+        const int64_t j = rows[2 * r];
+        const int g = (int)rows[2 * r + 1];
+        const int d = find_doc(cu_seqlens, n_docs, j);
+        const int64_t e = cu_seqlens[d + 1];
+        for (int64_t i = j; i < last_query(j, e, window); i++)
+            for (int hh = 0; hh < G; hh++) need[i * Hq + g * G + hh] = 1;
+    }
+    int64_t n_need = 0;
+    for (int64_t x = 0; x < T * Hq; x++) n_need += need[x];
+    int64_t *list = (int64_t *)malloc((size_t)(n_need > 0 ? n_need : 1) * sizeof(int64_t));
+    int64_t *slot = (int64_t *)malloc((size_t)(T * Hq > 0 ? T * Hq : 1) * sizeof(int64_t));
+    n_need = 0;
+    for (int64_t x = 0; x < T * Hq; x++) {
+        slot[x] = -1;
+        if (need[x]) { slot[x] = n_need; list[n_need++] = x; }
+    }
+    /* 2. lse_i and D_i = sum_c dO[i,h,c] out[i,h,c] of every needed row */
+    double *lse = (double *)malloc((size_t)(n_need > 0 ? n_need : 1) * sizeof(double));
+    double *Dv = (double *)malloc((size_t)(n_need > 0 ? n_need : 1) * sizeof(double));
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t u = 0; u < n_need; u++) {
+        const int64_t i = list[u] / Hq;
+        const int h = (int)(list[u] % Hq), g = h / G;
+        const int64_t s = cu_seqlens[find_doc(cu_seqlens, n_docs, i)];
+        const int64_t lo = first_key(i, s, window);
+        double *p = (double *)malloc((size_t)(i - lo + 1) * sizeof(double));
+        double *o = (double *)calloc((size_t)D, sizeof(double));
+        double psink;
+        row_probs(q, k, dtype, Hq, Hkv, D, scale, sinks, i, h, g, lo, p, &lse[u], &psink);
+        for (int64_t jj = lo; jj <= i; jj++)
+            for (int c = 0; c < D; c++)
+                o[c] += p[jj - lo] * load_elem(v, (jj * Hkv + g) * (int64_t)D + c, dtype);
+        double Di = 0.0;
+        for (int c = 0; c < D; c++) Di += load_elem(dout, (i * Hq + h) * (int64_t)D + c, dtype) * o[c];
+        Dv[u] = Di;
+        free(o);
+        free(p);
+    }
+    /* 3. the sums over (h, i) for each requested key row */
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n_rows; r++) {
+        const int64_t j = rows[2 * r];
+        const int g = (int)rows[2 * r + 1];
+        const int d = find_doc(cu_seqlens, n_docs, j);
+        const int64_t e = cu_seqlens[d + 1];
+        double *dk_out = dk_rows + r * D, *dv_out = dv_rows + r * D;
+        for (int c = 0; c < D; c++) { dk_out[c] = 0.0; dv_out[c] = 0.0; }
+        for (int hh = 0; hh < G; hh++) {
+            const int h = g * G + hh;
+            for (int64_t i = j; i < last_query(j, e, window); i++) {
+                const int64_t u = slot[i * Hq + h];
+                double sc = 0.0, dP = 0.0;
+                for (int c = 0; c < D; c++) {
+                    sc += load_elem(q, (i * Hq + h) * (int64_t)D + c, dtype) *
+                          load_elem(k, (j * Hkv + g) * (int64_t)D + c, dtype);
+                    dP += load_elem(dout, (i * Hq + h) * (int64_t)D + c, dtype) *
+                          load_elem(v, (j * Hkv + g) * (int64_t)D + c, dtype);
+                }
+                const double P = exp(scale * sc - lse[u]);
+                const double dS = P * (dP - Dv[u]);
+                for (int c = 0; c < D; c++) {
+                    dk_out[c] += scale * dS * load_elem(q, (i * Hq + h) * (int64_t)D + c, dtype);
+                    dv_out[c] += P * load_elem(dout, (i * Hq + h) * (int64_t)D + c, dtype);
+                }
+            }
+        }
+    }
+    free(Dv);
+    free(lse);
+    free(slot);
+    free(list);
+    free(need);
+    return 0;
+}
+
 /* Threads OpenMP would use for the calls above. */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

@@ -11,8 +11,10 @@ mean |err| <= 2e-3 * max |ref| (max |ref| floored at 1e-3 for tensors that
 vanish exactly).
 
 Small packs are compared element by element on every row; the full-size
-benchmark packs on sampled dq rows (computed one by one by the oracle) and on
-exact sum invariants of dk and dv.
+benchmark packs on sampled dq rows and sampled dk / dv rows (each computed one
+by one by the oracle: dq per query row, dk and dv per key row), on exact sum
+invariants of dk and dv where there is no sink, and on the sink gradient of a
+4,096-token slice against the oracle's whole-slice value.
 """
 import numpy as np
 import pytest
@@ -149,6 +151,38 @@ def sample_rows(cu, window, Hq, rng, n_random=256):
     return np.array(sorted(rows), dtype=np.int64)
 
 
+def kv_sample_rows(cu, window, Hkv, rng):
+    """(key token, kv head) rows for the key-side check: keys at each
+    document's end and its last tile edges (few queries see them, so the
+    oracle stays cheap), every tile edge of the two shortest documents, and
+    the first key of the two longest (seen by a whole window, or document, of
+    queries when that is short enough)."""
+    cu = [int(x) for x in cu]
+    docs = [(cu[d], cu[d + 1]) for d in range(len(cu) - 1) if cu[d + 1] > cu[d]]
+    rows = set()
+    for s, e in docs:
+        for t in (e - 1, e - 2, e - 64, e - 127, e - 128, e - 129, e - 200):
+            if s <= t < e:
+                rows.add((t, int(rng.integers(Hkv))))
+    for s, e in sorted(docs, key=lambda d: d[1] - d[0])[:2]:
+        for t in (s, s + 1, s + 127, s + 128, s + 129):
+            if s <= t < e:
+                rows.add((t, int(rng.integers(Hkv))))
+    if window > 0:
+        for s, e in sorted(docs, key=lambda d: d[0] - d[1])[:2]:
+            rows.add((s, int(rng.integers(Hkv))))
+            rows.add((s + (e - s) // 2, int(rng.integers(Hkv))))
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+def assert_sample_close(got, ref, what):
+    scale = max(np.abs(ref).max(), SCALE_FLOOR)
+    err = np.abs(got - ref)
+    assert np.isfinite(got).all(), f"{what}: non-finite"
+    assert err.max() <= REL_MAX * scale, f"{what}: max err {err.max():.3e} vs {scale:.3e}"
+    assert err.mean() <= REL_MEAN * scale, f"{what}: mean err {err.mean():.3e} vs {scale:.3e}"
+
+
 @pytest.mark.parametrize("name", ["pack64k_gqa8_d128_causal_sink", "pack32k_gqa4_d128_w4096"])
 def test_full_size_pack_bwd(name):
     cfg = workloads.CONFIGS[name]
@@ -160,10 +194,13 @@ def test_full_size_pack_bwd(name):
     rows = sample_rows(p["cu_seqlens"], cfg.window, cfg.Hq, np.random.default_rng(1))
     ref = oracle.attention_bwd_q_rows(p["q"], p["k"], p["v"], dout, p["cu_seqlens"], cfg.window,
                                       cfg.scale, rows, p["sinks"])
-    got = dq[rows[:, 0], rows[:, 1]].double().numpy()
-    scale = np.abs(ref).max()
-    assert np.abs(got - ref).max() <= REL_MAX * scale
-    assert np.abs(got - ref).mean() <= REL_MEAN * scale
+    assert_sample_close(dq[rows[:, 0], rows[:, 1]].double().numpy(), ref, f"{name} dq rows")
+    # key side, element by element on sampled (key, kv head) rows
+    krows = kv_sample_rows(p["cu_seqlens"], cfg.window, cfg.Hkv, np.random.default_rng(2))
+    rk, rv = oracle.attention_bwd_kv_rows(p["q"], p["k"], p["v"], dout, p["cu_seqlens"],
+                                          cfg.window, cfg.scale, krows, p["sinks"])
+    assert_sample_close(dk[krows[:, 0], krows[:, 1]].double().numpy(), rk, f"{name} dk rows")
+    assert_sample_close(dv[krows[:, 0], krows[:, 1]].double().numpy(), rv, f"{name} dv rows")
     if p["sinks"] is None:
         # Exact invariants without a sink: softmax is shift invariant, so the
         # key gradients of a (document, kv head) sum to zero, and the value
@@ -179,3 +216,16 @@ def test_full_size_pack_bwd(name):
                 assert (got_v - want_v).abs().max() <= 2e-2 * want_v.abs().max() + 1e-3 * (b - a) ** 0.5
                 ksum = dkf[a:b, g].sum(0).abs().max()
                 assert ksum <= 2e-2 * dkf[a:b, g].abs().sum(0).max()
+
+
+def test_sink_gradient_on_a_4k_slice():
+    """dsink sums over every query row, so it is checked on the first 4,096
+    tokens of the 64k pack (its sinks, heads and scale) against the oracle's
+    sink gradient of the whole slice."""
+    cfg = workloads.CONFIGS["pack64k_gqa8_d128_causal_sink"]
+    p = workloads.make_pack(cfg, 0, T_override=4096)
+    dout = dout_for(p, 6)
+    _, _, _, ds = run_gpu_bwd(p, dout)
+    ref = oracle.attention_dsink(p["q"], p["k"], p["v"], dout, p["cu_seqlens"], cfg.window,
+                                 cfg.scale, p["sinks"])
+    assert_sample_close(ds.double().numpy(), ref, "dsink (4k slice)")

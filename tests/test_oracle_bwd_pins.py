@@ -130,3 +130,42 @@ def test_q_rows_entry_point_equals_full_backward():
     rows = np.array([[0, 0], [49, 3], [50, 1], [56, 2], [86, 0], [60, 3]])
     got = oracle.attention_bwd_q_rows(q, k, v, dout, p["cu_seqlens"], 6, p["scale"], rows, s)
     assert np.allclose(got, dq[rows[:, 0], rows[:, 1]], atol=1e-13)
+
+
+@pytest.mark.parametrize("lens,Hq,Hkv,window,sinks", [
+    ([37, 0, 91, 1, 20], 4, 2, 0, True),
+    ([37, 0, 91, 1, 20], 6, 2, 9, False),
+    ([60, 33], 3, 3, 5, True),      # MHA
+    ([80], 4, 1, 0, False),         # MQA
+])
+def test_kv_rows_entry_point_equals_full_backward(lens, Hq, Hkv, window, sinks):
+    # Every (key token, kv head) row of small packs, with and without a window
+    # or sink, equals the full backward's dk and dv (same derivative, summed
+    # over the queries that see the key instead of scattered from each query).
+    p, q, k, v, s, dout = _f64_pack(31, lens, Hq, Hkv, 16, window, sinks)
+    _, rk, rv, _ = oracle.attention_bwd(q, k, v, dout, p["cu_seqlens"], window, p["scale"], s)
+    T = q.shape[0]
+    rows = np.array([(j, g) for j in range(T) for g in range(Hkv)], dtype=np.int64)
+    dk, dv = oracle.attention_bwd_kv_rows(q, k, v, dout, p["cu_seqlens"], window, p["scale"], rows, s)
+    assert np.abs(dk - rk[rows[:, 0], rows[:, 1]]).max() <= 1e-12
+    assert np.abs(dv - rv[rows[:, 0], rows[:, 1]]).max() <= 1e-12
+    # a shuffled subset in any order gives the same rows
+    sub = rows[np.random.default_rng(0).permutation(len(rows))[:11]]
+    dk2, dv2 = oracle.attention_bwd_kv_rows(q, k, v, dout, p["cu_seqlens"], window, p["scale"], sub, s)
+    assert np.abs(dk2 - rk[sub[:, 0], sub[:, 1]]).max() <= 1e-12
+    assert np.abs(dv2 - rv[sub[:, 0], sub[:, 1]]).max() <= 1e-12
+
+
+@pytest.mark.parametrize("window", [0, 7])
+def test_dsink_from_forward_equals_full_backward(window):
+    p, q, k, v, s, dout = _f64_pack(32, [40, 3, 70], 6, 2, 16, window, True)
+    _, _, _, rs = oracle.attention_bwd(q, k, v, dout, p["cu_seqlens"], window, p["scale"], s)
+    got = oracle.attention_dsink(q, k, v, dout, p["cu_seqlens"], window, p["scale"], s)
+    assert np.abs(got - rs).max() <= 1e-12 * max(1.0, np.abs(rs).max())
+
+
+def test_kv_rows_rejects_out_of_range_rows():
+    p, q, k, v, s, dout = _f64_pack(33, [10], 2, 1, 16, 0, False)
+    with pytest.raises(ValueError):
+        oracle.attention_bwd_kv_rows(q, k, v, dout, p["cu_seqlens"], 0, p["scale"],
+                                     np.array([[0, 1]]), s)   # kv head 1 of 1

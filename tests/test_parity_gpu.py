@@ -2,10 +2,12 @@
 
 Tolerances (from the hot path's numerical contract): bf16 output max-abs
 error 2e-2 and mean-abs error 2e-3; fp32 log-sum-exp max-abs error 1e-3.
-Small packs are compared element by element on every row; the full-size
-benchmark packs are compared on sampled rows the oracle computes one by one
-(document edges, query-tile edges, window edges and random rows), in the same
-launch configuration the benchmark times.
+Small packs, the 8k and the 32k benchmark packs are compared element by
+element on every row.  The 64k pack and the 128k document are compared on a
+dense subset of rows the oracle computes one by one (two full query heads,
+1/61 of all rows, document, tile and window edges), in the same launch
+configuration the benchmark times; tests/test_full_oracle_gpu.py checks every
+row of those two on request.
 """
 import numpy as np
 import pytest
@@ -174,13 +176,38 @@ def sample_rows(cu, window, Hq, rng, n_random=384):
     return np.array(sorted(rows), dtype=np.int64)
 
 
-@pytest.mark.parametrize("name", workloads.CONFIG_ORDER[1:])
-def test_full_size_pack_sampled_rows(name):
+@pytest.mark.parametrize("name", ["pack8k_gqa4_d128_causal", "pack32k_gqa4_d128_w4096"])
+def test_full_size_pack_every_row(name):
+    """Every (token, head) row of the 8k and 32k benchmark packs, element by
+    element, against the full oracle (FlintMagiPlan.attention's window and
+    sink semantics, "flint.magi" page)."""
+    cfg = workloads.CONFIGS[name]
+    p = workloads.make_pack(cfg, 0)
+    full_parity(p, name)
+
+
+def dense_subset_rows(cu, window, Hq, Hkv, stride=61):
+    """Every row of the first query head of the first kv group and of the last
+    query head of the last kv group, every stride-th (token, head) row of the
+    flattened pack (stride prime to the head counts, so all heads and token
+    positions mod 128 are hit), plus document, tile and window edges."""
+    T = int(cu[-1])
+    rows = {(t, h) for h in (0, Hq - 1) for t in range(T)}
+    rows.update((r // Hq, r % Hq) for r in range(7, T * Hq, stride))
+    rows.update(map(tuple, sample_rows(cu, window, Hq, np.random.default_rng(0))))
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+@pytest.mark.parametrize("name", ["pack64k_gqa8_d128_causal_sink", "doc128k_mqa_d256_w8192_sink"])
+def test_full_size_pack_dense_subset(name):
+    """The 64k pack and the 128k document, in the launch configuration the
+    benchmark times: two full query heads (one at each end of the kv groups)
+    and 1/61 of all other rows, element by element against the oracle."""
     cfg = workloads.CONFIGS[name]
     p = workloads.make_pack(cfg, 0)
     out, lse = run_gpu(p)
     assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
-    rows = sample_rows(p["cu_seqlens"], cfg.window, cfg.Hq, np.random.default_rng(0))
+    rows = dense_subset_rows(p["cu_seqlens"], cfg.window, cfg.Hq, cfg.Hkv)
     ref_o, ref_l = oracle.attention_rows(p["q"], p["k"], p["v"], p["cu_seqlens"], cfg.window,
                                          cfg.scale, rows, p["sinks"])
     got_o = out[rows[:, 0], rows[:, 1]]
