@@ -68,19 +68,24 @@ def test_unmutated_copy_passes(tmp_path):
     assert _pins_fail(lib) == []
 
 
-# The C source holds the forward first, then the backward after this marker;
-# a forward mutant changes the forward part only, a backward mutant the
-# backward part only.
+# The C source holds the forward first, then the backward after this marker,
+# then the key-rows backward entry point after the second marker (pinned
+# against the full backward in test_oracle_bwd_pins.py); a forward mutant
+# changes the forward part only, a backward mutant the full backward only.
 BWD_MARKER = " * Backward."
+KV_ROWS_MARKER = " * dk and dv for selected"
 
 
 def _mutate(old, new, backward):
     src = open(oracle._SRC).read()
     cut = src.index(BWD_MARKER)
-    head, tail = src[:cut], src[cut:]
-    part = tail if backward else head
+    cut2 = src.index(KV_ROWS_MARKER)
+    head, mid, rest = src[:cut], src[cut:cut2], src[cut2:]
+    part = mid if backward else head
     assert part.count(old) == 1, f"mutation anchor {old[:40]!r} not unique"
-    return head + tail.replace(old, new) if backward else head.replace(old, new) + tail
+    if backward:
+        return head + mid.replace(old, new) + rest
+    return head.replace(old, new) + mid + rest
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
