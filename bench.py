@@ -25,9 +25,10 @@ steps and warm-up:
 one line for that pass alone (``--workload`` selects the pack).
 
 Multi-GPU runs are launched with torchrun, one process per GPU; every rank
-runs its own pack of the same shape (no data-path collective), the timed
-region is bracketed by a barrier and a device synchronisation, and the time is
-the max over ranks.
+runs its own pack of the same shape (no data-path collective; "weak"), or,
+with ``--shard heads``, its kv-head groups of one pack (cp.head_shard; no
+collective either; "strong").  The timed region is bracketed by a barrier and
+a device synchronisation, and the time is the max over ranks.
 """
 from __future__ import annotations
 
@@ -59,8 +60,13 @@ DATASHEET_BF16_TFLOPS = 2250.0
 def kernel_name(D: int, group: int) -> str:
     """The kernel the library launches for this shape (label only): the
     CTA-pair kernel with the key-split softmax at head dim 256 with an even
-    GQA group, else the one-CTA kernel."""
-    return "thd_attn_fwd_split_kernel" if D == 256 and group % 2 == 0 else "thd_attn_fwd_kernel"
+    GQA group, the CTA-pair kernel with two heads per CTA at head dim 128
+    with a group that is a multiple of four, else the one-CTA kernel."""
+    if D == 256 and group % 2 == 0:
+        return "thd_attn_fwd_split_kernel"
+    if D == 128 and group % 4 == 0:
+        return "thd_attn_fwd_pair_kernel"
+    return "thd_attn_fwd_kernel"
 
 
 def log(*a):
@@ -86,6 +92,9 @@ def parse_args(argv=None):
                     default="fwd", help="what one step runs (default: the forward, the headline)")
     ap.add_argument("--no-extras", action="store_true",
                     help="headline only: leave out per_config and passes")
+    ap.add_argument("--shard", choices=["packs", "heads"], default="packs",
+                    help="multi-GPU form: every rank its own pack (weak scaling, default) or "
+                         "every rank its kv-head groups of one pack (strong scaling, no collective)")
     return ap.parse_args(argv)
 
 
@@ -106,7 +115,7 @@ def measured_peaks():
 E2E_CHUNKS = 16  # token ranges of the end-to-end call (copies overlap the attention)
 
 TRAFFIC_SOURCES = ("sm100_ptx.cuh", "thd_attn_kernel.cuh", "thd_attn_split_kernel.cuh",
-                   "scheduler.cpp", "scheduler.h")
+                   "thd_attn_pair_kernel.cuh", "scheduler.cpp", "scheduler.h")
 
 
 def kernel_source_hash() -> str:
@@ -308,15 +317,27 @@ def check_status(swa, stream, what):
 
 
 def fwd_case(swa, cfg, args, info, device, stream, T_override=None):
-    """Device tensors of one pack and a step that runs its forward."""
-    pack = workloads.make_pack(cfg, args.seed, tensor_seed=multirank.tensor_seed(args.seed, info.rank),
-                               T_override=T_override)
+    """Device tensors of one pack and a step that runs its forward.  With
+    ``--shard heads`` every rank holds the same pack and keeps only its head
+    slice (cp.head_shard): q/k/v/sinks/out/lse have the slice's head counts."""
+    heads = getattr(args, "shard", "packs") == "heads"
+    seed = args.seed if heads else multirank.tensor_seed(args.seed, info.rank)
+    pack = workloads.make_pack(cfg, args.seed, tensor_seed=seed, T_override=T_override)
     cu = pack["cu_seqlens"]
+    if heads:
+        from sliding_window_gqa_cu_b200 import cp
+        q_lo, q_hi, kv_lo, kv_hi = cp.head_shard(cfg.Hq, cfg.Hkv, info.world, info.rank)
+        pack["q"] = pack["q"][:, q_lo:q_hi].contiguous()
+        pack["k"] = pack["k"][:, kv_lo:kv_hi].contiguous()
+        pack["v"] = pack["v"][:, kv_lo:kv_hi].contiguous()
+        if pack["sinks"] is not None:
+            pack["sinks"] = pack["sinks"][q_lo:q_hi].contiguous()
+    Hq_r = pack["q"].shape[1]
     q, k, v = (pack[n].to(device) for n in "qkv")
     sinks = pack["sinks"].to(device) if pack["sinks"] is not None else None
     T = pack["T"]
-    out = torch.empty((T, cfg.Hq, cfg.D), dtype=torch.bfloat16, device=device)
-    lse = torch.empty((T, cfg.Hq), dtype=torch.float32, device=device)
+    out = torch.empty((T, Hq_r, cfg.D), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((T, Hq_r), dtype=torch.float32, device=device)
 
     def step():
         swa.thd_attn_fwd(q, k, v, cu, cfg.window, cfg.scale, sinks, out=out, lse=lse, stream=stream)
@@ -447,7 +468,8 @@ def run_ours(args, info):
     pack, t, step = fwd_case(swa, cfg, args, info, device, stream, T_override=args.tokens)
     cu, T = pack["cu_seqlens"], pack["T"]
     pairs = metrics.valid_pairs(cu, cfg.window)
-    flops = 4 * pairs * cfg.D * cfg.Hq
+    Hq_r = t["q"].shape[1]  # query heads this rank computes (all of them unless --shard heads)
+    flops = 4 * pairs * cfg.D * Hq_r
 
     t_plan0 = time.perf_counter()
     step()  # first call builds and uploads the tile schedule
@@ -463,7 +485,7 @@ def run_ours(args, info):
 
     # end to end through the public API with pinned host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and args.shard == "packs":
         qh, kh, vh = (pack[n].pin_memory() for n in "qkv")
         sh = pack["sinks"].pin_memory() if pack["sinks"] is not None else None
         oh = torch.empty(t["out"].shape, dtype=t["out"].dtype).pin_memory()
@@ -504,9 +526,10 @@ def run_ours(args, info):
                 else "fallback 1.59 PFLOP/s",
                 "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
                 "frac_of_datasheet_2250": achieved / DATASHEET_BF16_TFLOPS,
-                "kernel": kernel_name(cfg.D, cfg.Hq // cfg.Hkv),
+                "kernel": kernel_name(cfg.D, Hq_r // t["k"].shape[1]),
                 "algorithmic_flops_per_launch": flops,
-                "algorithmic_bytes_per_launch": metrics.algorithmic_bytes(T, cfg.Hq, cfg.Hkv, cfg.D)}
+                "algorithmic_bytes_per_launch": metrics.algorithmic_bytes(T, Hq_r, t["k"].shape[1],
+                                                                          cfg.D)}
     del pack, t, step
 
     cpu = None
@@ -519,7 +542,7 @@ def run_ours(args, info):
         del cpack
 
     per_config, passes = None, None
-    if not args.no_extras and args.tokens is None:
+    if not args.no_extras and args.tokens is None and args.shard == "packs":
         per_config = {}
         for name in EXTRA_CONFIGS:
             if name == cfg.name:
@@ -546,10 +569,13 @@ def run_ours(args, info):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": info.world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "strong" if args.shard == "heads" else "weak",
+            "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": workload_config(cfg, cu, pairs, {"parallelism": f"pack-parallel x{info.world}",
-                                                       "per_rank_tflop": flops / 1e12}),
+            "config": workload_config(cfg, cu, pairs, {
+                "parallelism": (f"head-sharded x{info.world} (one pack, no collective)"
+                                if args.shard == "heads" else f"pack-parallel x{info.world}"),
+                "per_rank_tflop": flops / 1e12}),
             "pct_of_peak": 100.0 * value / info.world / peak,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps, "clocks": {k: csum[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
@@ -574,6 +600,9 @@ def run_ours(args, info):
 def run_other_pass(args, info):
     """--pass bwd / prologue / sparse_mla: one line for that pass alone."""
     import sliding_window_gqa_cu_b200 as swa
+
+    if args.shard != "packs":
+        raise SystemExit("--shard heads applies to the forward only")
 
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device (the CUDA path has no CPU fallback)")

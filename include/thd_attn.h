@@ -292,7 +292,7 @@ typedef struct thd_bwd_kv_item {
 size_t thd_attn_bwd_workspace_bytes(int64_t total_tokens, int Hq);
 
 /*
- * Backward of thd_attn_fwd for head dim 64 or 128 (256: THD_ERR_UNSUPPORTED).
+ * Backward of thd_attn_fwd for head dim 64, 128 or 256.
  *   q, k, v, cu_seqlens, n_docs, Hq, Hkv, D, window, scale, sinks_or_null
  *              exactly as passed to thd_attn_fwd
  *   out        bf16 device [T, Hq, D]: the forward's output

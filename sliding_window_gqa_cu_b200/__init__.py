@@ -203,7 +203,7 @@ def thd_attn_fwd(q, k, v, cu_seqlens, window: int = 0, scale: Optional[float] = 
 def thd_attn_bwd(q, k, v, out, lse, dout, cu_seqlens, window: int = 0,
                  scale: Optional[float] = None, sinks=None, dq=None, dk=None, dv=None,
                  workspace=None, stream=None):
-    """Backward of :func:`thd_attn_fwd` (head dim 64 or 128).
+    """Backward of :func:`thd_attn_fwd` (head dim 64, 128 or 256).
 
     q, k, v, cu_seqlens, window, scale, sinks: as passed to the forward;
     out, lse: the forward's results; dout: bf16 CUDA [T, Hq, D] gradient of the

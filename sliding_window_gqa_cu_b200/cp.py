@@ -1,4 +1,13 @@
-"""Context-parallel forward over the ranks of one node (one process per GPU).
+"""Multi-GPU forms of the forward over the ranks of one node (one process per GPU).
+
+Head sharding (no collective): the kv-head groups of the repeat_kv mapping
+("muse_glimmer.model" page) are independent problems, so rank r computes the
+query heads :func:`head_shard` gives it -- whole kv groups when the kv heads
+divide evenly over the ranks, else an even slice of one group's query heads
+with that group's K/V replicated -- on the whole pack, and writes exactly those
+heads of the output.  :func:`head_sharded_attention_fwd` is the local call.
+
+Context parallelism:
 
 The Magi plans of the "muse_spark.magi_cp" page shard a packed microbatch's
 tokens over the context-parallel ranks and let the attention engine exchange
@@ -64,3 +73,39 @@ def cp_attention_fwd(q_local: torch.Tensor, k_local: torch.Tensor, v_local: torc
         raise ValueError(f"rank {rank} owns rows [{b}, {e}) of the pack")
     k_full, v_full = gather_kv(k_local, v_local, T, group)
     return thd_attn_fwd_range(q_local, k_full, v_full, cu_seqlens, b, e, window, scale, sinks)
+
+
+def head_shard(Hq: int, Hkv: int, world: int, rank: int) -> tuple[int, int, int, int]:
+    """Heads of ``rank`` in the head-sharded forward: ``(q_lo, q_hi, kv_lo,
+    kv_hi)``, the query heads [q_lo, q_hi) and the kv heads [kv_lo, kv_hi)
+    they read (query head h reads kv head h // (Hq / Hkv)).
+
+    Hkv % world == 0: whole kv groups, Hkv / world of them per rank.
+    world % Hkv == 0 and Hq % world == 0: world / Hkv ranks share a group,
+    each with Hq / world of its query heads and a copy of its K/V.
+    Anything else raises ValueError."""
+    if world <= 0 or not (0 <= rank < world) or Hkv <= 0 or Hq % Hkv:
+        raise ValueError("need 0 <= rank < world and Hq a multiple of Hkv")
+    G = Hq // Hkv
+    if Hkv % world == 0:
+        n = Hkv // world
+        return rank * n * G, (rank + 1) * n * G, rank * n, (rank + 1) * n
+    if world % Hkv == 0 and Hq % world == 0:
+        per = Hq // world  # query heads per rank, inside one group
+        q_lo = rank * per
+        g = q_lo // G
+        return q_lo, q_lo + per, g, g + 1
+    raise ValueError(f"{Hq} query / {Hkv} kv heads do not split evenly over {world} ranks")
+
+
+def head_sharded_attention_fwd(q_local: torch.Tensor, k_local: torch.Tensor,
+                               v_local: torch.Tensor, cu_seqlens, window: int = 0,
+                               scale: Optional[float] = None, sinks_local=None):
+    """This rank's heads of the packed-THD attention forward: q_local
+    [T, q_hi - q_lo, D] and k_local / v_local [T, kv_hi - kv_lo, D] are the
+    head slices of :func:`head_shard` (dense, contiguous), sinks_local the
+    same query heads' sink logits.  No collective: the result is those heads
+    of the whole forward, [T, q_hi - q_lo, D] and [T, q_hi - q_lo]."""
+    from . import thd_attn_fwd
+
+    return thd_attn_fwd(q_local, k_local, v_local, cu_seqlens, window, scale, sinks_local)

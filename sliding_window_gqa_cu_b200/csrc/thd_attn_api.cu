@@ -18,6 +18,7 @@
 #include "tma_map.h"
 #include "thd_attn_kernel.cuh"
 #include "thd_attn_split_kernel.cuh"
+#include "thd_attn_pair_kernel.cuh"
 #include "thd_attn_bwd_kernels.cuh"
 
 namespace {
@@ -32,11 +33,12 @@ using Cfg128x2 = thd::FwdConfig<128, 2, 1, 128, 5>;
 using Cfg128x1 = thd::FwdConfig<128, 1, 2, 128, 6>;
 using Cfg256x1 = thd::FwdConfig<256, 1, 2, 64, 5>;
 using SplitCfg256 = thd::SplitConfig<256, 2, 4>;  // 2 heads per item over a CTA pair
+using PairCfg128 = thd::PairConfig<128, 8, THD_PAIR_EXP_EMU>;  // 4 heads per item over a CTA pair
 
-constexpr int kNumVariants = 6;
+constexpr int kNumVariants = 7;
 
 int variant_index(const KernelShape& ks) {
-    if (ks.pair) return 5;
+    if (ks.pair) return ks.D == 256 ? 5 : 6;
     if (ks.D == 64) return ks.nq == 2 ? 0 : 1;
     if (ks.D == 128) return ks.nq == 2 ? 2 : 3;
     return 4;
@@ -63,7 +65,7 @@ struct BwdPlanEntry {
     int64_t n_kv_items = 0;
 };
 
-constexpr int kNumBwdVariants = 4;  // {dq, dkdv} x {D = 64, D = 128}
+constexpr int kNumBwdVariants = 7;  // {dq, dkdv} x {D = 64, D = 128}, then dq, dv, dk at D = 256
 
 struct DeviceState {
     int* d_status = nullptr;
@@ -182,6 +184,24 @@ int launch_pair(DeviceState* ds, int vidx, const PlanEntry& plan, const CUtensor
     return cudaGetLastError() == cudaSuccess ? THD_OK : THD_ERR_CUDA;
 }
 
+// CTA-pair shapes with two heads per CTA: two CTAs (one cluster) per item.
+template <class C>
+int launch_pair2(DeviceState* ds, int vidx, const PlanEntry& plan, const CUtensorMap& mq,
+                 const CUtensorMap& mk, const CUtensorMap& mv, const thd::FwdParams& prm,
+                 cudaStream_t stream) {
+    auto kern = thd::thd_attn_fwd_pair_kernel<C>;
+    if (!ds->attr_set[vidx]) {
+        if (!thd::pair_launch_registers_ok<C>()) return THD_ERR_UNSUPPORTED;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_ALLOC) != cudaSuccess)
+            return THD_ERR_CUDA;
+        ds->attr_set[vidx] = true;
+    }
+    kern<<<static_cast<unsigned>(2 * plan.n_items), C::NUM_THREADS, C::SMEM_ALLOC, stream>>>(
+        mq, mk, mv, prm);
+    return cudaGetLastError() == cudaSuccess ? THD_OK : THD_ERR_CUDA;
+}
+
 // Uploads `n` items to a new device buffer (synchronously on `stream`).
 template <class T>
 int upload(const std::vector<T>& v, T** out, cudaStream_t stream) {
@@ -213,8 +233,9 @@ int get_bwd_plan(DeviceState* ds, const int32_t* cu, int n_docs, int Hq, int Hkv
             return THD_OK;
         }
     }
-    // dq items: the forward's query tiles and key ranges, one query head each.
-    const KernelShape qs{D, 1, 1, 128, 4, false};
+    // dq items: the forward's query tiles and key ranges, one query head each
+    // (64-key tiles at head dim 256).
+    const KernelShape qs{D, 1, 1, D == 256 ? 64 : 128, 4, false};
     std::vector<thd_work_item> qi = thd::build_plan(cu, n_docs, Hq, Hkv, window, qs);
     std::vector<thd_bwd_kv_item> ki = thd::build_bwd_kv_plan(cu, n_docs, Hq, Hkv, D, window);
     std::vector<thd::WorkItem> qv(qi.size());
@@ -287,6 +308,57 @@ int launch_bwd(DeviceState* ds, const BwdPlanEntry& plan, const CUtensorMap& mq,
     if (plan.n_kv_items > 0)
         kkv<<<static_cast<unsigned>(plan.n_kv_items), Ckv::NUM_THREADS,
               thd::DkvLayout<Ckv>::SMEM_ALLOC, stream>>>(mq, mdo, mk, mv, prm);
+    return cudaGetLastError() == cudaSuccess ? THD_OK : THD_ERR_CUDA;
+}
+
+// Head dim 256: dq with 64-key tiles, then the key side in two launches (dv
+// alone, dk alone) with 64-query tiles.
+template <class C>
+int set_smem_attr(DeviceState* ds, int vidx, const void* kern, int bytes) {
+    if (ds->bwd_attr_set[vidx]) return THD_OK;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return THD_ERR_CUDA;
+    ds->bwd_attr_set[vidx] = true;
+    return THD_OK;
+}
+
+int launch_bwd256(DeviceState* ds, const BwdPlanEntry& plan, const CUtensorMap& mq128,
+                  const CUtensorMap& mdo128, const CUtensorMap& mk128, const CUtensorMap& mv128,
+                  const CUtensorMap& mq64, const CUtensorMap& mdo64, const CUtensorMap& mk64,
+                  const CUtensorMap& mv64, const thd::BwdParams& prm, const void* out,
+                  const void* dout, const float* sinks, float* dsinks, float* delta,
+                  float* sink_part, cudaStream_t stream) {
+    using Cq = thd::BwdConfig<256, 3, 64>;
+    using Cdv = thd::BwdConfig<256, 2, 64, thd::kDvOnly>;
+    using Cdk = thd::BwdConfig<256, 1, 64, thd::kDkOnly>;
+    auto kq = thd::thd_attn_bwd_dq_kernel<Cq>;
+    auto kdv = thd::thd_attn_bwd_dkdv_kernel<Cdv>;
+    auto kdk = thd::thd_attn_bwd_dkdv_kernel<Cdk>;
+    int rc = set_smem_attr<Cq>(ds, 4, reinterpret_cast<const void*>(kq), thd::DqLayout<Cq>::SMEM_ALLOC);
+    if (rc == THD_OK)
+        rc = set_smem_attr<Cdv>(ds, 5, reinterpret_cast<const void*>(kdv), thd::DkvLayout<Cdv>::SMEM_ALLOC);
+    if (rc == THD_OK)
+        rc = set_smem_attr<Cdk>(ds, 6, reinterpret_cast<const void*>(kdk), thd::DkvLayout<Cdk>::SMEM_ALLOC);
+    if (rc != THD_OK) return rc;
+    const int64_t rows = prm.T * prm.Hq;
+    thd::thd_attn_bwd_preprocess_kernel<256><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), prm.lse,
+        sinks, delta, sink_part, rows, prm.Hq);
+    if (dsinks != nullptr) {
+        if (sinks != nullptr)
+            thd::thd_attn_bwd_dsink_kernel<<<prm.Hq, 256, 0, stream>>>(sink_part, prm.T, prm.Hq, dsinks);
+        else if (cudaMemsetAsync(dsinks, 0, sizeof(float) * prm.Hq, stream) != cudaSuccess)
+            return THD_ERR_CUDA;
+    }
+    if (plan.n_q_items > 0)
+        kq<<<static_cast<unsigned>(plan.n_q_items), Cq::NUM_THREADS, thd::DqLayout<Cq>::SMEM_ALLOC,
+             stream>>>(mq128, mdo128, mk64, mv64, prm);
+    if (plan.n_kv_items > 0) {
+        kdv<<<static_cast<unsigned>(plan.n_kv_items), Cdv::NUM_THREADS,
+              thd::DkvLayout<Cdv>::SMEM_ALLOC, stream>>>(mq64, mdo64, mk128, mv128, prm);
+        kdk<<<static_cast<unsigned>(plan.n_kv_items), Cdk::NUM_THREADS,
+              thd::DkvLayout<Cdk>::SMEM_ALLOC, stream>>>(mq64, mdo64, mk128, mv128, prm);
+    }
     return cudaGetLastError() == cudaSuccess ? THD_OK : THD_ERR_CUDA;
 }
 
@@ -438,7 +510,8 @@ int thd_attn_fwd_range(const void* q, const void* k, const void* v, const int32_
         case 2: return launch<Cfg128x2>(ds, 2, *plan, mq, mk, mv, prm, stream);
         case 3: return launch<Cfg128x1>(ds, 3, *plan, mq, mk, mv, prm, stream);
         case 4: return launch<Cfg256x1>(ds, 4, *plan, mq, mk, mv, prm, stream);
-        default: return launch_pair<SplitCfg256>(ds, 5, *plan, mq, mk, mv, prm, stream);
+        case 5: return launch_pair<SplitCfg256>(ds, 5, *plan, mq, mk, mv, prm, stream);
+        default: return launch_pair2<PairCfg128>(ds, 6, *plan, mq, mk, mv, prm, stream);
     }
 }
 
@@ -461,7 +534,6 @@ int thd_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
                  float* dsinks_or_null, void* workspace, size_t workspace_bytes, void* stream_ptr) {
     int rc = thd::validate_args(cu_seqlens, n_docs, Hq, Hkv, D, window);
     if (rc != THD_OK) return rc;
-    if (D != 64 && D != 128) return THD_ERR_UNSUPPORTED;
     if (!(std::isfinite(scale) && scale > 0.0f)) return THD_ERR_INVALID_ARG;
     const int64_t T = cu_seqlens[n_docs];
     cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
@@ -494,6 +566,10 @@ int thd_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
     if (!make_map(&mq, q, T, Hq, D, 128) || !make_map(&mdo, dout, T, Hq, D, 128) ||
         !make_map(&mk, k, T, Hkv, D, 128) || !make_map(&mv, v, T, Hkv, D, 128))
         return THD_ERR_CUDA;
+    CUtensorMap mq64, mdo64, mk64, mv64;  // head dim 256: tiles of 64 rows
+    if (D == 256 && (!make_map(&mq64, q, T, Hq, D, 64) || !make_map(&mdo64, dout, T, Hq, D, 64) ||
+                     !make_map(&mk64, k, T, Hkv, D, 64) || !make_map(&mv64, v, T, Hkv, D, 64)))
+        return THD_ERR_CUDA;
     float* delta = static_cast<float*>(workspace);
     float* sink_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                                 align256(static_cast<size_t>(T) * Hq * sizeof(float)));
@@ -516,8 +592,11 @@ int thd_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
     if (D == 64)
         return launch_bwd<64>(ds, *plan, mq, mdo, mk, mv, prm, out, dout, sinks_or_null,
                               dsinks_or_null, delta, sink_part, stream);
-    return launch_bwd<128>(ds, *plan, mq, mdo, mk, mv, prm, out, dout, sinks_or_null,
-                           dsinks_or_null, delta, sink_part, stream);
+    if (D == 128)
+        return launch_bwd<128>(ds, *plan, mq, mdo, mk, mv, prm, out, dout, sinks_or_null,
+                               dsinks_or_null, delta, sink_part, stream);
+    return launch_bwd256(ds, *plan, mq, mdo, mk, mv, mq64, mdo64, mk64, mv64, prm, out, dout,
+                         sinks_or_null, dsinks_or_null, delta, sink_part, stream);
 }
 
 int thd_attn_get_error(void* stream_ptr) {

@@ -20,10 +20,18 @@
 //     tensor core computes dq(j), dP(j + 1) and S(j + 2) while the
 //     elementwise warps exponentiate S(j + 1).
 //   * dkdv kernel: one CTA per (128-key tile, kv head), looping over the
-//     query heads of the group and the 128-query tiles that see the keys:
+//     query tiles that see the keys (from the document end backward) and,
+//     for each, the query heads of the group:
 //     S^T = K Q^T and dP^T = V dO^T (TMEM lane = key), P^T and dS^T written as
 //     bf16 over them, dv += P^T dO and dk += dS^T Q (TMEM operands, dO and Q
 //     as MN-major operands); dk and dv stay in TMEM for the whole group.
+//
+// Head dim 256: the operand that streams through the ring (K/V tiles in the
+// dq kernel, Q/dO tiles in the dkdv kernel) comes in tiles of BN = 64 rows so
+// that the resident 128-row tiles and the ring fit in shared memory, and the
+// key-side kernel runs twice, once accumulating dv only and once dk only (two
+// 256-column accumulators do not fit in TMEM together); the dk launch
+// recomputes S^T.
 //
 // Warps (both kernels): 0-7 elementwise, 8 TMA producer, 9 MMA issuer, 10-11
 // idle.  Elementwise warp w owns TMEM lanes [32 (w % 4), 32 (w % 4) + 32).
@@ -67,10 +75,11 @@ struct BwdParams {
 constexpr float kLog2e = 1.4426950408889634f;
 
 // TMEM column (relative to S or dP) of the bf16 operand for K-step kk of an
-// MMA over 128 columns: half kk / 4 is packed into [64 (kk / 4), +32), eight
-// columns (16 values) per step.
+// MMA over BN columns: half kk / (BN / 32) is packed into [BN/2 half,
+// BN/2 half + BN/4), eight columns (16 values) per step.
+template <int BN>
 __device__ __forceinline__ constexpr uint32_t pcol(int kk) {
-    return static_cast<uint32_t>(64 * (kk >> 2) + 8 * (kk & 3));
+    return static_cast<uint32_t>((BN / 2) * (kk / (BN / 32)) + 8 * (kk % (BN / 32)));
 }
 
 // -------------------------------------------------------------- preprocess --
@@ -146,31 +155,41 @@ __global__ void __launch_bounds__(256) thd_attn_bwd_dsink_kernel(const float* __
 
 // ------------------------------------------------------------ shared shape --
 
-template <int D_, int NSLOT_>
+// What the key-side kernel accumulates: dk and dv together (head dim <= 128),
+// or one of them (head dim 256, two launches).
+enum BwdKvMode { kDkDv = 0, kDvOnly = 1, kDkOnly = 2 };
+
+template <int D_, int NSLOT_, int BN_ = 128, int MODE_ = kDkDv>
 struct BwdConfig {
     static constexpr int D = D_;
     static constexpr int NSLOT = NSLOT_;  // dq: K/V ring slots; dkdv: Q/dO pairs
     static constexpr int BM = 128;        // TMEM lanes (queries for dq, keys for dkdv)
-    static constexpr int BN = 128;        // columns of S per tile
+    static constexpr int BN = BN_;        // columns of S per tile (keys for dq, queries for dkdv)
+    static constexpr int MODE = MODE_;    // dkdv kernel only
+    static constexpr int HALF = BN / 2;   // columns of S per elementwise warp
     static constexpr int KCH = D / 64;
     static constexpr int BOX_BYTES = 128 * 128;   // one 64-column chunk of a 128-row tile
     static constexpr int TILE_BYTES = 128 * D * 2;
+    static constexpr int NBOX_BYTES = BN * 128;   // one 64-column chunk of a BN-row tile
+    static constexpr int NTILE_BYTES = BN * D * 2;
 
     static constexpr int TM_S = 0;        // S (dq) or S^T (dkdv), then P / dS bf16
     static constexpr int TM_DP = 128;     // dP or dP^T, then dS^T (dkdv)
     static constexpr int TM_ACC0 = 256;   // dq (dq kernel) or dv (dkdv kernel)
-    static constexpr int TM_ACC1 = 256 + D;  // dk (dkdv kernel)
-    static constexpr int TM_S2 = 384;     // dq kernel: second S buffer (odd key tiles)
+    static constexpr int TM_ACC1 = MODE == kDkDv ? 256 + D : 256;  // dk (dkdv kernel)
+    static constexpr int TM_S2 = BN == 128 ? 384 : BN;  // dq kernel: second S buffer (odd key tiles)
     static constexpr int TMEM_COLS = 512;
 
     static constexpr int PRODUCER_WARP = 8;
     static constexpr int MMA_WARP = 9;
     static constexpr int NUM_THREADS = 384;
 
-    static_assert(D == 64 || D == 128, "backward kernels: head dim 64 or 128");
-    static_assert(TM_ACC1 + D <= 512, "TMEM budget exceeded");
-    static_assert(TM_ACC0 + D <= TM_S2 && TM_S2 + BN <= TMEM_COLS, "dq kernel TMEM budget exceeded");
-    static_assert(NSLOT >= 2, "ring needs two slots");
+    static_assert(D == 64 || D == 128 || D == 256, "backward kernels: head dim 64, 128 or 256");
+    static_assert(BN == 128 || BN == 64, "S tiles of 128 or 64 columns");
+    static_assert(TM_ACC0 + D <= 512, "TMEM budget exceeded");
+    static_assert(BN == 64 ? (TM_S2 + BN <= TM_DP) : (TM_ACC0 + D <= TM_S2 && TM_S2 + BN <= TMEM_COLS),
+                  "dq kernel TMEM budget exceeded");
+    static_assert(NSLOT >= 1, "ring needs a slot");
 };
 
 // ------------------------------------------------------------------ dq ------
@@ -187,12 +206,13 @@ struct DqLayout {
     static constexpr int NUM_BARS = B_DRAIN + 1;
     static constexpr int SMEM_Q = 0;
     static constexpr int SMEM_DO = SMEM_Q + C::TILE_BYTES;
-    static constexpr int SMEM_SLOTS = SMEM_DO + C::TILE_BYTES;
-    static constexpr int SMEM_BAR = SMEM_SLOTS + C::NSLOT * C::TILE_BYTES;
+    static constexpr int SMEM_SLOTS = SMEM_DO + C::TILE_BYTES;  // [NSLOT] K or V tile of BN rows
+    static constexpr int SMEM_BAR = SMEM_SLOTS + C::NSLOT * C::NTILE_BYTES;
     static constexpr int SMEM_TMEM_SLOT = SMEM_BAR + NUM_BARS * 8;
     static constexpr int SMEM_ABORT = SMEM_TMEM_SLOT + 4;
     static constexpr int SMEM_ALLOC = SMEM_ABORT + 4 + 1024;
     static_assert(SMEM_ALLOC <= 232448, "shared memory budget exceeded");
+    static_assert(C::NSLOT >= 2, "dq ring needs two slots");
 };
 
 template <class C>
@@ -265,9 +285,9 @@ thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 if (!ok) break;
                 const CUtensorMap* map = (pos & 1) ? &tmap_v : &tmap_k;
                 const int kt = it.kv_start + (pos >> 1) * C::BN;
-                mbar_arrive_expect_tx(bar(L::B_SLOT_FULL + slot), C::TILE_BYTES);
+                mbar_arrive_expect_tx(bar(L::B_SLOT_FULL + slot), C::NTILE_BYTES);
                 for (int c = 0; c < C::KCH; ++c)
-                    tma_load_3d(sbase + L::SMEM_SLOTS + slot * C::TILE_BYTES + c * C::BOX_BYTES, map,
+                    tma_load_3d(sbase + L::SMEM_SLOTS + slot * C::NTILE_BYTES + c * C::NBOX_BYTES, map,
                                 bar(L::B_SLOT_FULL + slot), c * 64, g, kt);
                 issued = pos + 1;
             }
@@ -285,7 +305,7 @@ thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
             const uint64_t dq0 = smem_desc_sw128(sbase + L::SMEM_Q, 16, 1024);
             const uint64_t ddo0 = smem_desc_sw128(sbase + L::SMEM_DO, 16, 1024);
             const uint64_t dkv0 = smem_desc_sw128(sbase + L::SMEM_SLOTS, 16, 1024);
-            const uint64_t dkmn0 = smem_desc_sw128(sbase + L::SMEM_SLOTS, C::BOX_BYTES, 1024);
+            const uint64_t dkmn0 = smem_desc_sw128(sbase + L::SMEM_SLOTS, C::NBOX_BYTES, 1024);
             auto wait = [&](int idx, uint32_t parity) -> bool {
                 return mbar_wait(bar(idx), parity, abort_flag, prm.status, kStatusTimeout);
             };
@@ -297,12 +317,13 @@ thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
             auto issue_s = [&](int j) -> bool {  // S(j) = Q K(j)^T into buffer j % 2
                 if (!wait_slot(2 * j)) return false;
                 tc_fence_after();
-                const uint64_t dk = dkv0 + ((((2 * j) % C::NSLOT) * C::TILE_BYTES) >> 4);
+                const uint64_t dk = dkv0 + ((((2 * j) % C::NSLOT) * C::NTILE_BYTES) >> 4);
                 const uint32_t ts = tmem_base + ((j & 1) ? C::TM_S2 : C::TM_S);
 #pragma unroll
                 for (int kk = 0; kk < C::D / 16; ++kk) {
                     const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
-                    mma_bf16_ss(ts, dq0 + o, dk + o, idesc_s, kk > 0 ? 1u : 0u);
+                    const uint32_t on = ((kk >> 2) * C::NBOX_BYTES + (kk & 3) * 32) >> 4;
+                    mma_bf16_ss(ts, dq0 + o, dk + on, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar(L::B_S_FULL + (j & 1)));
                 return true;
@@ -311,11 +332,12 @@ thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 if (!wait_slot(2 * j + 1)) return false;
                 tc_fence_after();
                 const int vslot = (2 * j + 1) % C::NSLOT;
-                const uint64_t dv = dkv0 + ((vslot * C::TILE_BYTES) >> 4);
+                const uint64_t dv = dkv0 + ((vslot * C::NTILE_BYTES) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < C::D / 16; ++kk) {
                     const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
-                    mma_bf16_ss(tmem_base + C::TM_DP, ddo0 + o, dv + o, idesc_s, kk > 0 ? 1u : 0u);
+                    const uint32_t on = ((kk >> 2) * C::NBOX_BYTES + (kk & 3) * 32) >> 4;
+                    mma_bf16_ss(tmem_base + C::TM_DP, ddo0 + o, dv + on, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar(L::B_DP_FULL));
                 mma_commit(bar(L::B_SLOT_EMPTY + vslot));  // V(j) consumed
@@ -327,11 +349,11 @@ thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 if (!ok) break;
                 tc_fence_after();
                 const int kslot = (2 * j) % C::NSLOT;
-                const uint64_t dkmn = dkmn0 + ((kslot * C::TILE_BYTES) >> 4);
+                const uint64_t dkmn = dkmn0 + ((kslot * C::NTILE_BYTES) >> 4);
                 const uint32_t ts = tmem_base + ((j & 1) ? C::TM_S2 : C::TM_S);
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; ++kk)  // dq += dS K
-                    mma_bf16_ts(tmem_base + C::TM_ACC0, ts + pcol(kk),
+                    mma_bf16_ts(tmem_base + C::TM_ACC0, ts + pcol<C::BN>(kk),
                                 dkmn + ((kk * 16 * 128) >> 4), idesc_acc, (j > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(bar(L::B_SLOT_EMPTY + kslot));  // K(j) consumed
                 // dP(j + 1) overwrites dP(j), read before dS(j) was signalled;
@@ -370,21 +392,25 @@ thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
             if (!ok) break;
             tc_fence_after();
             const uint32_t tm_s = (j & 1) ? C::TM_S2 : C::TM_S;
-            const int kh = it.kv_start + j * C::BN + 64 * h;  // first key of this half
-            const bool full = row_valid && kh >= s_doc && kh + 63 <= r_lo &&
+            constexpr int HALF = C::HALF;
+            const int kh = it.kv_start + j * C::BN + HALF * h;  // first key of this half
+            const bool full = row_valid && kh >= s_doc && kh + HALF - 1 <= r_lo &&
                               (W == 0 || kh >= r_hi - W + 1);
             const int c_lo = lo_i - kh, c_hi = i - kh;  // visible columns of the half
-            // P of this half (64 values) while the tensor core computes dP.
-            float pv[64];
+            // P of this half (HALF values) while the tensor core computes dP.
+            float pv[HALF];
             {
-                uint32_t sr[64];
-                tmem_ld32(lane_base + tm_s + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                tmem_ld32(lane_base + tm_s + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-                tmem_wait_ld();
-                reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                uint32_t sr[HALF];
 #pragma unroll
-                for (int c = 0; c < 64; ++c) {
+                for (int cc = 0; cc < HALF / 32; ++cc)
+                    tmem_ld32(lane_base + tm_s + HALF * h + 32 * cc,
+                              *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]));
+                tmem_wait_ld();
+#pragma unroll
+                for (int cc = 0; cc < HALF / 32; ++cc)
+                    reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]));
+#pragma unroll
+                for (int c = 0; c < HALF; ++c) {
                     const float x = ex2_approx(fmaf(__uint_as_float(sr[c]), sl2, -lse2));
                     pv[c] = (full || (c >= c_lo && c <= c_hi)) ? x : 0.0f;
                 }
@@ -393,9 +419,9 @@ thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
+            for (int cc = 0; cc < HALF / 32; ++cc) {
                 uint32_t dr[32];
-                tmem_ld32(lane_base + C::TM_DP + 64 * h + 32 * cc, dr);
+                tmem_ld32(lane_base + C::TM_DP + HALF * h + 32 * cc, dr);
                 tmem_wait_ld();
                 reg_fence32(dr);
                 uint32_t pk[16];
@@ -404,8 +430,8 @@ thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     pk[u] = pack_bf16x2(pv[32 * cc + 2 * u] * (__uint_as_float(dr[2 * u]) - Di),
                                         pv[32 * cc + 2 * u + 1] * (__uint_as_float(dr[2 * u + 1]) - Di));
                 // dS of this half's columns [32 cc, 32 cc + 32) goes to TMEM
-                // columns 64 h + [16 cc, 16 cc + 16) (S of this half, read).
-                tmem_st16(lane_base + tm_s + 64 * h + 16 * cc, pk);
+                // columns HALF h + [16 cc, 16 cc + 16) (S of this half, read).
+                tmem_st16(lane_base + tm_s + HALF * h + 16 * cc, pk);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -463,10 +489,12 @@ struct DkvLayout {
     static constexpr int NUM_BARS = B_DRAIN + 1;
     static constexpr int SMEM_K = 0;
     static constexpr int SMEM_V = SMEM_K + C::TILE_BYTES;
-    static constexpr int SMEM_PAIRS = SMEM_V + C::TILE_BYTES;  // [NPAIR][Q tile, dO tile]
-    static constexpr int PAIR_BYTES = 2 * C::TILE_BYTES;
-    static constexpr int SMEM_SIDE = SMEM_PAIRS + NPAIR * PAIR_BYTES;  // [NPAIR][lse2 128, delta 128]
-    static constexpr int SIDE_BYTES = 2 * 128 * 4;
+    static_assert(C::MODE != kDkDv || C::TM_ACC1 + C::D <= 512, "dk and dv together exceed TMEM");
+    static constexpr int V_BYTES = C::MODE == kDvOnly ? 0 : C::TILE_BYTES;  // dv alone needs no V
+    static constexpr int SMEM_PAIRS = SMEM_V + V_BYTES;  // [NPAIR][Q tile, dO tile] of BN rows
+    static constexpr int PAIR_BYTES = 2 * C::NTILE_BYTES;
+    static constexpr int SMEM_SIDE = SMEM_PAIRS + NPAIR * PAIR_BYTES;  // [NPAIR][lse2 BN, delta BN]
+    static constexpr int SIDE_BYTES = 2 * C::BN * 4;
     static constexpr int SMEM_BAR = SMEM_SIDE + NPAIR * SIDE_BYTES;
     static constexpr int SMEM_TMEM_SLOT = SMEM_BAR + NUM_BARS * 8;
     static constexpr int SMEM_ABORT = SMEM_TMEM_SLOT + 4;
@@ -489,7 +517,10 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
     const int lane = threadIdx.x & 31;
     const BwdKVItem it = prm.kv_items[blockIdx.x];
     const int G = prm.G;
-    const int n_steps = G * it.n_q;  // (query head, query tile) steps
+    const int nsub = it.n_q * (128 / C::BN);  // query tiles of BN rows per head
+    const int n_steps = G * nsub;             // (query head, query tile) steps
+    constexpr bool kDv = C::MODE != kDkOnly;  // accumulates dv
+    constexpr bool kDk = C::MODE != kDvOnly;  // accumulates dk
 
     auto bar = [&](int idx) -> uint32_t { return sbase + L::SMEM_BAR + 8u * idx; };
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::SMEM_ABORT);
@@ -531,37 +562,43 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
             tma_prefetch_desc(&tmap_do);
             tma_prefetch_desc(&tmap_k);
             tma_prefetch_desc(&tmap_v);
-            mbar_arrive_expect_tx(bar(L::B_KV_FULL), 2 * C::TILE_BYTES);
+            mbar_arrive_expect_tx(bar(L::B_KV_FULL), (kDk ? 2 : 1) * C::TILE_BYTES);
             for (int c = 0; c < C::KCH; ++c) {
                 tma_load_3d(sbase + L::SMEM_K + c * C::BOX_BYTES, &tmap_k, bar(L::B_KV_FULL), c * 64,
                             it.g, it.k0);
-                tma_load_3d(sbase + L::SMEM_V + c * C::BOX_BYTES, &tmap_v, bar(L::B_KV_FULL), c * 64,
-                            it.g, it.k0);
+                if (kDk)
+                    tma_load_3d(sbase + L::SMEM_V + c * C::BOX_BYTES, &tmap_v, bar(L::B_KV_FULL),
+                                c * 64, it.g, it.k0);
             }
         }
         for (int s = 0; ok && s < n_steps; ++s) {
             const int pr = s % L::NPAIR;
             ok = warp_wait(bar(L::B_PAIR_EMPTY + pr), ((s / L::NPAIR) & 1) ^ 1, abort_flag, prm.status);
             if (!ok) break;
-            const int h = it.g * G + s / it.n_q;
-            const int i0 = it.k0 + (s % it.n_q) * 128;
+            // Step s: query tile nsub - 1 - s / G (from the document end
+            // backward), query head g G + s % G.  The CTAs of one document
+            // start at its end together and walk the same Q / dO tiles at
+            // about the same time, so they share them in L2.
+            const int h = it.g * G + s % G;
+            const int i0 = it.k0 + (nsub - 1 - s / G) * C::BN;
             if (lane == 0) {
                 const uint32_t full = bar(L::B_PAIR_FULL + pr);
                 const uint32_t dst = sbase + L::SMEM_PAIRS + pr * L::PAIR_BYTES;
-                mbar_arrive_expect_tx(full, 2 * C::TILE_BYTES);
+                mbar_arrive_expect_tx(full, 2 * C::NTILE_BYTES);
                 for (int c = 0; c < C::KCH; ++c) {
-                    tma_load_3d(dst + c * C::BOX_BYTES, &tmap_q, full, c * 64, h, i0);
-                    tma_load_3d(dst + C::TILE_BYTES + c * C::BOX_BYTES, &tmap_do, full, c * 64, h, i0);
+                    tma_load_3d(dst + c * C::NBOX_BYTES, &tmap_q, full, c * 64, h, i0);
+                    tma_load_3d(dst + C::NTILE_BYTES + c * C::NBOX_BYTES, &tmap_do, full, c * 64, h,
+                                i0);
                 }
             }
-            float* sd = side + pr * 256;
+            float* sd = side + pr * 2 * C::BN;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int col = lane * 4 + u;
+            for (int u = 0; u < C::BN / 32; ++u) {
+                const int col = lane * (C::BN / 32) + u;
                 const int64_t i = static_cast<int64_t>(i0) + col;
                 const bool in = i < prm.T;
                 sd[col] = in ? prm.lse[i * prm.Hq + h] * kLog2e : 0.0f;
-                sd[128 + col] = in ? prm.delta[i * prm.Hq + h] : 0.0f;
+                sd[C::BN + col] = in ? prm.delta[i * prm.Hq + h] : 0.0f;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(L::B_PAIR_FULL + pr));
@@ -581,7 +618,7 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
             const uint64_t dk0 = smem_desc_sw128(sbase + L::SMEM_K, 16, 1024);
             const uint64_t dv0 = smem_desc_sw128(sbase + L::SMEM_V, 16, 1024);
             const uint64_t dpair0 = smem_desc_sw128(sbase + L::SMEM_PAIRS, 16, 1024);
-            const uint64_t dpairmn0 = smem_desc_sw128(sbase + L::SMEM_PAIRS, C::BOX_BYTES, 1024);
+            const uint64_t dpairmn0 = smem_desc_sw128(sbase + L::SMEM_PAIRS, C::NBOX_BYTES, 1024);
             auto wait = [&](int idx, uint32_t parity) -> bool {
                 return mbar_wait(bar(idx), parity, abort_flag, prm.status, kStatusTimeout);
             };
@@ -592,37 +629,45 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t qoff = (pr * L::PAIR_BYTES) >> 4;
-                const uint32_t dooff = (pr * L::PAIR_BYTES + C::TILE_BYTES) >> 4;
+                const uint32_t dooff = (pr * L::PAIR_BYTES + C::NTILE_BYTES) >> 4;
 #pragma unroll
                 for (int kk = 0; kk < C::D / 16; ++kk) {  // S^T = K Q^T
                     const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
-                    mma_bf16_ss(tmem_base + C::TM_S, dk0 + o, dpair0 + qoff + o, idesc_s,
+                    const uint32_t on = ((kk >> 2) * C::NBOX_BYTES + (kk & 3) * 32) >> 4;
+                    mma_bf16_ss(tmem_base + C::TM_S, dk0 + o, dpair0 + qoff + on, idesc_s,
                                 kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar(L::B_S_FULL));  // the exponentials start under dP^T
+                if constexpr (kDk) {
 #pragma unroll
-                for (int kk = 0; kk < C::D / 16; ++kk) {  // dP^T = V dO^T
-                    const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
-                    mma_bf16_ss(tmem_base + C::TM_DP, dv0 + o, dpair0 + dooff + o, idesc_s,
-                                kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < C::D / 16; ++kk) {  // dP^T = V dO^T
+                        const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
+                        const uint32_t on = ((kk >> 2) * C::NBOX_BYTES + (kk & 3) * 32) >> 4;
+                        mma_bf16_ss(tmem_base + C::TM_DP, dv0 + o, dpair0 + dooff + on, idesc_s,
+                                    kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar(L::B_DP_FULL));
                 }
-                mma_commit(bar(L::B_DP_FULL));
-                ok = wait(L::B_P_READY, s & 1);
-                if (!ok) break;
-                tc_fence_after();
+                if constexpr (kDv) {
+                    ok = wait(L::B_P_READY, s & 1);
+                    if (!ok) break;
+                    tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < C::BN / 16; ++kk)  // dv += P^T dO (16 query rows a step)
-                    mma_bf16_ts(tmem_base + C::TM_ACC0, tmem_base + C::TM_S + pcol(kk),
-                                dpairmn0 + dooff + ((kk * 16 * 128) >> 4), idesc_acc,
-                                (s > 0 || kk > 0) ? 1u : 0u);
-                ok = wait(L::B_DS_READY, s & 1);  // dS^T is computed under dv
-                if (!ok) break;
-                tc_fence_after();
+                    for (int kk = 0; kk < C::BN / 16; ++kk)  // dv += P^T dO (16 query rows a step)
+                        mma_bf16_ts(tmem_base + C::TM_ACC0, tmem_base + C::TM_S + pcol<C::BN>(kk),
+                                    dpairmn0 + dooff + ((kk * 16 * 128) >> 4), idesc_acc,
+                                    (s > 0 || kk > 0) ? 1u : 0u);
+                }
+                if constexpr (kDk) {
+                    ok = wait(L::B_DS_READY, s & 1);  // dS^T is computed under dv
+                    if (!ok) break;
+                    tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < C::BN / 16; ++kk)  // dk += dS^T Q
-                    mma_bf16_ts(tmem_base + C::TM_ACC1, tmem_base + C::TM_DP + pcol(kk),
-                                dpairmn0 + qoff + ((kk * 16 * 128) >> 4), idesc_acc,
-                                (s > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < C::BN / 16; ++kk)  // dk += dS^T Q
+                        mma_bf16_ts(tmem_base + C::TM_ACC1, tmem_base + C::TM_DP + pcol<C::BN>(kk),
+                                    dpairmn0 + qoff + ((kk * 16 * 128) >> 4), idesc_acc,
+                                    (s > 0 || kk > 0) ? 1u : 0u);
+                }
                 mma_commit(bar(L::B_PAIR_EMPTY + pr));
             }
             if (ok) mma_commit(bar(L::B_ACC_FULL));
@@ -647,32 +692,36 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
         if (!row_valid) i_hi = j - 1;
 
         bool ok = !skip;
+        constexpr int HALF = C::HALF;
         for (int s = 0; ok && s < n_steps; ++s) {
             const int pr = s % L::NPAIR;
-            const int ih = it.k0 + (s % it.n_q) * 128 + 64 * h;  // first query of this half
+            const int ih = it.k0 + (nsub - 1 - s / G) * C::BN + HALF * h;  // first query of this half
             // The side values of this step were stored before PAIR_FULL.
             ok = warp_wait(bar(L::B_PAIR_FULL + pr), (s / L::NPAIR) & 1, abort_flag, prm.status) &&
                  warp_wait(bar(L::B_S_FULL), s & 1, abort_flag, prm.status);
             if (!ok) break;
             tc_fence_after();
-            const float* lse2 = side + pr * 256 + 64 * h;
-            const float* dlt = side + pr * 256 + 128 + 64 * h;
+            const float* lse2 = side + pr * 2 * C::BN + HALF * h;
+            const float* dlt = side + pr * 2 * C::BN + C::BN + HALF * h;
             // Every (key, query) of this half visible: its queries after every
             // key, inside the document and inside every key's window.
-            const bool full = ih >= k_last && ih + 63 < e_doc && it.k0 + 127 < e_doc &&
-                              (W == 0 || ih + 63 - it.k0 < W);
+            const bool full = ih >= k_last && ih + HALF - 1 < e_doc && it.k0 + 127 < e_doc &&
+                              (W == 0 || ih + HALF - 1 - it.k0 < W);
             const int c_lo = j - ih, c_hi = i_hi - ih;  // visible columns of the half
             // P^T of this half (while the tensor core computes dP^T) ...
-            float pv[64];
+            float pv[HALF];
             {
-                uint32_t sr[64];
-                tmem_ld32(lane_base + C::TM_S + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                tmem_ld32(lane_base + C::TM_S + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-                tmem_wait_ld();
-                reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                uint32_t sr[HALF];
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
+                for (int cc = 0; cc < HALF / 32; ++cc)
+                    tmem_ld32(lane_base + C::TM_S + HALF * h + 32 * cc,
+                              *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]));
+                tmem_wait_ld();
+#pragma unroll
+                for (int cc = 0; cc < HALF / 32; ++cc)
+                    reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]));
+#pragma unroll
+                for (int u = 0; u < HALF / 4; ++u) {
                     const float4 l4 = *reinterpret_cast<const float4*>(lse2 + 4 * u);
                     const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
@@ -682,49 +731,83 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
                         pv[c] = (full || (c >= c_lo && c <= c_hi)) ? x : 0.0f;
                     }
                 }
-                uint32_t pp[32];
+                if constexpr (kDv) {
+                    uint32_t pp[HALF / 2];
 #pragma unroll
-                for (int u = 0; u < 32; ++u) pp[u] = pack_bf16x2(pv[2 * u], pv[2 * u + 1]);
-                // Over this half's own S^T columns [64 h, 64 h + 32), all read.
-                tmem_st16(lane_base + C::TM_S + 64 * h, *reinterpret_cast<uint32_t(*)[16]>(&pp[0]));
-                tmem_st16(lane_base + C::TM_S + 64 * h + 16, *reinterpret_cast<uint32_t(*)[16]>(&pp[16]));
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(L::B_P_READY));
-            // ... then dS^T = P^T (dP^T - delta) while it computes dv.
-            ok = warp_wait(bar(L::B_DP_FULL), s & 1, abort_flag, prm.status);
-            if (!ok) break;
-            tc_fence_after();
+                    for (int u = 0; u < HALF / 2; ++u) pp[u] = pack_bf16x2(pv[2 * u], pv[2 * u + 1]);
+                    // Over this half's own first S^T columns, all read.
 #pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                uint32_t dr[32];
-                tmem_ld32(lane_base + C::TM_DP + 64 * h + 32 * cc, dr);
-                tmem_wait_ld();
-                reg_fence32(dr);
-                uint32_t pd[16];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const float4 d4 = *reinterpret_cast<const float4*>(dlt + 32 * cc + 4 * u);
-                    const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
-                    float dsv[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        dsv[e] = pv[32 * cc + 4 * u + e] * (__uint_as_float(dr[4 * u + e]) - dv4[e]);
-                    pd[2 * u] = pack_bf16x2(dsv[0], dsv[1]);
-                    pd[2 * u + 1] = pack_bf16x2(dsv[2], dsv[3]);
+                    for (int cc = 0; cc < HALF / 32; ++cc)
+                        tmem_st16(lane_base + C::TM_S + HALF * h + 16 * cc,
+                                  *reinterpret_cast<uint32_t(*)[16]>(&pp[16 * cc]));
                 }
-                // Over dP^T columns 64 h + [16 cc, 16 cc + 16), already read.
-                tmem_st16(lane_base + C::TM_DP + 64 * h + 16 * cc, pd);
             }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(L::B_DS_READY));
+            if constexpr (kDv) {
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(L::B_P_READY));
+            }
+            if constexpr (kDk) {
+                // ... then dS^T = P^T (dP^T - delta) while it computes dv.
+                ok = warp_wait(bar(L::B_DP_FULL), s & 1, abort_flag, prm.status);
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll
+                for (int cc = 0; cc < HALF / 32; ++cc) {
+                    uint32_t dr[32];
+                    tmem_ld32(lane_base + C::TM_DP + HALF * h + 32 * cc, dr);
+                    tmem_wait_ld();
+                    reg_fence32(dr);
+                    uint32_t pd[16];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const float4 d4 = *reinterpret_cast<const float4*>(dlt + 32 * cc + 4 * u);
+                        const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+                        float dsv[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            dsv[e] = pv[32 * cc + 4 * u + e] * (__uint_as_float(dr[4 * u + e]) - dv4[e]);
+                        pd[2 * u] = pack_bf16x2(dsv[0], dsv[1]);
+                        pd[2 * u + 1] = pack_bf16x2(dsv[2], dsv[3]);
+                    }
+                    // Over dP^T columns HALF h + [16 cc, 16 cc + 16), already read.
+                    tmem_st16(lane_base + C::TM_DP + HALF * h + 16 * cc, pd);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(L::B_DS_READY));
+            }
         }
         if (ok) ok = warp_wait(bar(L::B_ACC_FULL), 0, abort_flag, prm.status);
-        if (ok) {
+        if (ok && C::MODE != kDkDv) {
+            // One accumulator (dv, or dk times the score scale); half h stores
+            // its columns [h D / 2, (h + 1) D / 2).
+            tc_fence_after();
+            constexpr int HC = C::D / 2;
+            __nv_bfloat16* dst_row = (kDv ? prm.dv : prm.dk) +
+                                     (static_cast<int64_t>(j) * prm.Hkv + it.g) * C::D + h * HC;
+            const float f = kDv ? 1.0f : prm.scale;
+            const uint32_t acc = lane_base + (kDv ? C::TM_ACC0 : C::TM_ACC1) + h * HC;
+#pragma unroll 1
+            for (int c = 0; c < HC / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(acc + c * 32, r);
+                tmem_wait_ld();
+                reg_fence32(r);
+                uint32_t w[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u)
+                    w[u] = pack_bf16x2(__uint_as_float(r[2 * u]) * f, __uint_as_float(r[2 * u + 1]) * f);
+                if (row_valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(dst_row + c * 32);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        dst[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+                }
+            }
+        } else if (ok) {
             tc_fence_after();
             // Half 0 stores dv, half 1 stores dk (times the score scale).
             __nv_bfloat16* dst_row = (h == 0 ? prm.dv : prm.dk) +

@@ -92,6 +92,11 @@ BWD_CASES = [
     ([333, 64], 6, 2, 128, 50, False),             # G = 3
     ([520, 3], 16, 1, 128, 0, True),               # MQA, G = 16
     ([500, 130], 16, 2, 128, 300, True),           # G = 8
+    ([520, 3], 16, 1, 256, 0, True),               # D = 256, MQA
+    ([300, 45, 1], 3, 1, 256, 0, True),            # D = 256, odd group
+    ([400, 77], 4, 2, 256, 65, False),             # D = 256, window
+    ([200, 1, 130], 2, 2, 256, 0, True),           # D = 256, MHA
+    ([700], 4, 1, 256, 129, True),                 # D = 256, several key and query tiles
 ]
 
 
@@ -127,13 +132,10 @@ def test_bwd_is_deterministic():
         assert torch.equal(x, y)
 
 
-def test_bwd_rejects_head_dim_256():
-    dev = torch.device("cuda:0")
-    p = workloads.random_pack(15, [64], 2, 1, 256, 0, 256 ** -0.5, False)
-    q, k, v = (p[n].to(dev) for n in "qkv")
-    out, lse = swa.thd_attn_fwd(q, k, v, p["cu_seqlens"], 0, p["scale"])
-    with pytest.raises(swa.ThdAttnError):
-        swa.thd_attn_bwd(q, k, v, out, lse, torch.zeros_like(out), p["cu_seqlens"], 0, p["scale"])
+def test_mid_pack_bwd_parity_d256():
+    # head dim 256: several 64-key and 64-query tiles per document, a sink
+    p = workloads.random_pack(15, [1100, 300, 2], 8, 2, 256, 0, 256 ** -0.5, True)
+    full_bwd_parity(p, 7, "mid pack D256")
 
 
 # ------------------------------------------------- full-size benchmark packs -
@@ -151,7 +153,7 @@ def sample_rows(cu, window, Hq, rng, n_random=256):
     return np.array(sorted(rows), dtype=np.int64)
 
 
-def kv_sample_rows(cu, window, Hkv, rng):
+def kv_sample_rows(cu, window, Hkv, rng, starts=True):
     """(key token, kv head) rows for the key-side check: keys at each
     document's end and its last tile edges (few queries see them, so the
     oracle stays cheap), every tile edge of the two shortest documents, and
@@ -168,7 +170,7 @@ def kv_sample_rows(cu, window, Hkv, rng):
         for t in (s, s + 1, s + 127, s + 128, s + 129):
             if s <= t < e:
                 rows.add((t, int(rng.integers(Hkv))))
-    if window > 0:
+    if window > 0 and starts:
         for s, e in sorted(docs, key=lambda d: d[0] - d[1])[:2]:
             rows.add((s, int(rng.integers(Hkv))))
             rows.add((s + (e - s) // 2, int(rng.integers(Hkv))))
@@ -183,7 +185,8 @@ def assert_sample_close(got, ref, what):
     assert err.mean() <= REL_MEAN * scale, f"{what}: mean err {err.mean():.3e} vs {scale:.3e}"
 
 
-@pytest.mark.parametrize("name", ["pack64k_gqa8_d128_causal_sink", "pack32k_gqa4_d128_w4096"])
+@pytest.mark.parametrize("name", ["pack64k_gqa8_d128_causal_sink", "pack32k_gqa4_d128_w4096",
+                                  "doc128k_mqa_d256_w8192_sink"])
 def test_full_size_pack_bwd(name):
     cfg = workloads.CONFIGS[name]
     p = workloads.make_pack(cfg, 0)
@@ -196,7 +199,10 @@ def test_full_size_pack_bwd(name):
                                       cfg.scale, rows, p["sinks"])
     assert_sample_close(dq[rows[:, 0], rows[:, 1]].double().numpy(), ref, f"{name} dq rows")
     # key side, element by element on sampled (key, kv head) rows
-    krows = kv_sample_rows(p["cu_seqlens"], cfg.window, cfg.Hkv, np.random.default_rng(2))
+    # (a key in the middle of the 128k document is seen by 8,192 queries of
+    # all 16 heads, too many for the oracle here: only its end-of-document keys)
+    krows = kv_sample_rows(p["cu_seqlens"], cfg.window, cfg.Hkv, np.random.default_rng(2),
+                           starts=cfg.D != 256)
     rk, rv = oracle.attention_bwd_kv_rows(p["q"], p["k"], p["v"], dout, p["cu_seqlens"],
                                           cfg.window, cfg.scale, krows, p["sinks"])
     assert_sample_close(dk[krows[:, 0], krows[:, 1]].double().numpy(), rk, f"{name} dk rows")

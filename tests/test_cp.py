@@ -101,3 +101,62 @@ def test_two_rank_gloo_kv_all_gather(tmp_path):
     port = _free_port()
     mp.spawn(_worker, args=(2, port, str(tmp_path)), nprocs=2, join=True)
     assert [open(tmp_path / f"r{r}.txt").read() for r in range(2)] == ["ok", "ok"]
+
+
+# ----------------------------------------------------------- head sharding --
+
+@pytest.mark.parametrize("Hq,Hkv,world", [(64, 8, 8), (64, 8, 2), (32, 8, 4), (16, 1, 8),
+                                          (16, 1, 2), (8, 2, 4), (4, 4, 4), (16, 2, 1)])
+def test_head_shard_partitions_the_heads(Hq, Hkv, world):
+    G = Hq // Hkv
+    seen = np.zeros(Hq, dtype=int)
+    for r in range(world):
+        q_lo, q_hi, kv_lo, kv_hi = cp.head_shard(Hq, Hkv, world, r)
+        assert q_hi - q_lo == Hq // world
+        seen[q_lo:q_hi] += 1
+        # every query head of the slice reads a kv head of the slice, and the
+        # slice's own GQA mapping (local head // local group) is the global one
+        for h in range(q_lo, q_hi):
+            assert kv_lo <= h // G < kv_hi
+            local_G = (q_hi - q_lo) // (kv_hi - kv_lo)
+            assert (h - q_lo) // local_G == h // G - kv_lo
+    assert (seen == 1).all()
+
+
+@pytest.mark.parametrize("Hq,Hkv,world", [(12, 4, 8), (6, 3, 4), (8, 2, 3)])
+def test_head_shard_rejects_uneven_splits(Hq, Hkv, world):
+    with pytest.raises(ValueError):
+        cp.head_shard(Hq, Hkv, world, 0)
+
+
+def _head_shard_worker(rank, world, port, Hq, Hkv, out_q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    torch.distributed.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        mine = torch.tensor(cp.head_shard(Hq, Hkv, world, rank), dtype=torch.int64)
+        got = [torch.zeros(4, dtype=torch.int64) for _ in range(world)]
+        torch.distributed.all_gather(got, mine)
+        if rank == 0:
+            out_q.put([g.tolist() for g in got])
+    finally:
+        torch.distributed.destroy_process_group()
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(64, 8), (16, 1)])
+def test_head_shard_over_two_gloo_ranks(Hq, Hkv):
+    # Each rank derives its own slice; together they cover every query head once.
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    out_q = ctx.Queue()
+    procs = [ctx.Process(target=_head_shard_worker, args=(r, 2, port, Hq, Hkv, out_q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    shards = out_q.get(timeout=120)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    heads = sorted(h for q_lo, q_hi, _, _ in shards for h in range(q_lo, q_hi))
+    assert heads == list(range(Hq))

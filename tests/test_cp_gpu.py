@@ -63,3 +63,38 @@ def test_single_process_cp_is_the_forward():
     a, la = cp.cp_attention_fwd(q, k, v, p["cu_seqlens"], 0, p["scale"], s)
     b, lb = swa.thd_attn_fwd(q, k, v, p["cu_seqlens"], 0, p["scale"], s)
     assert torch.equal(a, b) and torch.equal(la, lb)
+
+
+@pytest.mark.parametrize("lens,Hq,Hkv,D,window,sinks,world", [
+    ([390, 5, 128, 1, 200], 16, 4, 128, 0, True, 4),    # whole kv groups per rank
+    ([390, 5, 128, 1, 200], 16, 4, 128, 0, True, 2),
+    ([520, 3], 16, 1, 256, 300, True, 8),              # MQA: query heads split, K/V replicated
+    ([700, 45], 8, 2, 64, 0, False, 4),
+])
+def test_head_sharded_forward_equals_the_oracle(lens, Hq, Hkv, D, window, sinks, world):
+    """Every rank's head slice (cp.head_shard) run in turn on one GPU: the
+    slices side by side equal the oracle and, bit for bit, the whole-pack
+    forward (each row is computed the same way whichever heads share it)."""
+    p = workloads.random_pack(33, lens, Hq, Hkv, D, window, D ** -0.5, sinks)
+    dev = torch.device("cuda:0")
+    q, k, v = (p[n].to(dev) for n in "qkv")
+    s = p["sinks"].to(dev) if sinks else None
+    outs, lses = [], []
+    for r in range(world):
+        q_lo, q_hi, kv_lo, kv_hi = cp.head_shard(Hq, Hkv, world, r)
+        o, l = cp.head_sharded_attention_fwd(q[:, q_lo:q_hi].contiguous(), k[:, kv_lo:kv_hi].contiguous(),
+                                             v[:, kv_lo:kv_hi].contiguous(), p["cu_seqlens"], window,
+                                             p["scale"], s[q_lo:q_hi].contiguous() if sinks else None)
+        outs.append(o)
+        lses.append(l)
+    out, lse = torch.cat(outs, 1), torch.cat(lses, 1)
+    torch.cuda.synchronize()
+    assert swa.thd_attn_get_error() == 0
+    ref_o, ref_l = oracle.attention(p["q"], p["k"], p["v"], p["cu_seqlens"], window, p["scale"],
+                                    p["sinks"])
+    o = out.cpu().double().numpy()
+    assert np.abs(o - ref_o).max() <= 2e-2 and np.abs(o - ref_o).mean() <= 2e-3
+    assert np.abs(lse.cpu().double().numpy() - ref_l).max() <= 1e-3
+    full_o, full_l = swa.thd_attn_fwd(q, k, v, p["cu_seqlens"], window, p["scale"], s)
+    assert (full_o.float() - out.float()).abs().max() <= 1.6e-2
+    assert (full_l - lse).abs().max() <= 1e-3
