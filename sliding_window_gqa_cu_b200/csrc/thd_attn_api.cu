@@ -69,6 +69,7 @@ constexpr int kNumBwdVariants = 7;  // {dq, dkdv} x {D = 64, D = 128}, then dq, 
 
 struct DeviceState {
     int* d_status = nullptr;
+    int pair_clusters = 0;  // resident clusters of the head-dim-128 pair kernel
     bool attr_set[kNumVariants] = {};
     bool bwd_attr_set[kNumBwdVariants] = {};
     std::list<PlanEntry> plans;         // most recently used first
@@ -195,9 +196,10 @@ int launch_pair2(DeviceState* ds, int vidx, const PlanEntry& plan, const CUtenso
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::SMEM_ALLOC) != cudaSuccess)
             return THD_ERR_CUDA;
+        ds->pair_clusters = thd::pair_max_active_clusters<C>();
         ds->attr_set[vidx] = true;
     }
-    kern<<<static_cast<unsigned>(2 * plan.n_items), C::NUM_THREADS, C::SMEM_ALLOC, stream>>>(
+    kern<<<thd::pair_grid(plan.n_items, ds->pair_clusters), C::NUM_THREADS, C::SMEM_ALLOC, stream>>>(
         mq, mk, mv, prm);
     return cudaGetLastError() == cudaSuccess ? THD_OK : THD_ERR_CUDA;
 }
@@ -503,6 +505,7 @@ int thd_attn_fwd_range(const void* q, const void* k, const void* v, const int32_
     prm.window = window;
     prm.scale_log2 = scale * 1.4426950408889634f;
     prm.q_offset = static_cast<int>(q_begin);
+    prm.n_items = static_cast<int>(plan->n_items);
 
     switch (variant_index(ks)) {
         case 0: return launch<Cfg64x2>(ds, 0, *plan, mq, mk, mv, prm, stream);

@@ -58,6 +58,7 @@ struct NoAllocDevice {
     bool ready = false;
     unsigned char* scratch = nullptr;  // device address of g_noalloc_scratch
     bool attr_set[7] = {};
+    int pair_clusters = 0;  // resident clusters of the head-dim-128 pair kernel
     // arguments of the schedule now in the scratch (valid when have_plan)
     bool have_plan = false;
     int n_docs = 0, Hq = 0, Hkv = 0, D = 0, window = 0;
@@ -192,10 +193,11 @@ int launch_pair2(NoAllocDevice* st, int vidx, int64_t n_items, const CUtensorMap
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::SMEM_ALLOC) != cudaSuccess)
             return THD_ERR_CUDA;
+        st->pair_clusters = thd::pair_max_active_clusters<C>();
         st->attr_set[vidx] = true;
     }
-    kern<<<static_cast<unsigned>(2 * n_items), C::NUM_THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv,
-                                                                                      prm);
+    kern<<<thd::pair_grid(n_items, st->pair_clusters), C::NUM_THREADS, C::SMEM_ALLOC, stream>>>(
+        mq, mk, mv, prm);
     return cudaGetLastError() == cudaSuccess ? THD_OK : THD_ERR_CUDA;
 }
 
@@ -283,6 +285,7 @@ extern "C" int thd_attn_fwd_noalloc(const void* q, const void* k, const void* v,
     prm.window = window;
     prm.scale_log2 = scale * 1.4426950408889634f;
     prm.q_offset = 0;
+    prm.n_items = static_cast<int>(n_items);
     prm.plan_tag = reinterpret_cast<const unsigned long long*>(st->scratch + kTagOffset);
     prm.expected_tag = st->tag;
 

@@ -47,6 +47,13 @@
 #define THD_PAIR_EXP_EMU 1
 #endif
 
+// 1: a persistent grid of one cluster per SM pair loops over the work items
+// (the next item's Q load and first QK overlap the previous item's tail);
+// 0: one cluster per item.
+#ifndef THD_PAIR_PERSIST
+#define THD_PAIR_PERSIST 1
+#endif
+
 namespace thd {
 
 template <int D_, int NSLOT_, int EXP_EMU_>
@@ -87,12 +94,14 @@ struct PairConfig {
 
     // mbarrier indices
     static constexpr int B_Q_FULL = 0;                        // leader: all four Q tiles landed
-    static constexpr int B_SLOT_FULL = 1;                     // leader: both halves landed
+    static constexpr int B_Q_EMPTY = 1;                       // both: the item's last QK done
+    static constexpr int B_SLOT_FULL = 2;                     // leader: both halves landed
     static constexpr int B_SLOT_EMPTY = B_SLOT_FULL + NSLOT;  // both: slot may be refilled
     static constexpr int B_S_FULL = B_SLOT_EMPTY + NSLOT;     // both: S[q] ready (and PV(j-1) done)
     static constexpr int B_P_FULL = B_S_FULL + NQ;            // leader: P[q] written in both CTAs
     static constexpr int B_O_FULL = B_P_FULL + NQ;            // both: last PV of stream q done
-    static constexpr int B_DRAIN = B_O_FULL + NQ;
+    static constexpr int B_O_FREE = B_O_FULL + NQ;            // leader: O[q] read in both CTAs
+    static constexpr int B_DRAIN = B_O_FREE + NQ;
     static constexpr int NUM_BARS = B_DRAIN + 1;
 
     static constexpr int SMEM_Q = 0;
@@ -129,9 +138,13 @@ thd_attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmap_q,
     const int lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
-    const WorkItem it = p.items[blockIdx.x >> 1];
-    const int n = it.n_kv;
-    const int head_base = it.head0 + 2 * static_cast<int>(rank);  // this CTA's first head
+    // Cluster c runs items c, c + n_clusters, ... (one item per cluster when
+    // the grid has a cluster per item; a persistent grid of one cluster per
+    // SM pair otherwise).  Barrier phases run on across items: S and P once
+    // per key tile, Q, O and "O read" once per item.
+    const int cluster_id = static_cast<int>(blockIdx.x >> 1);
+    const int n_clusters = static_cast<int>(gridDim.x >> 1);
+    const int n_items = p.n_items;
 
     auto bar = [&](int idx) -> uint32_t { return sbase + C::SMEM_BAR + 8u * idx; };
     auto lead_bar = [&](int idx) -> uint32_t { return mapa_shared(bar(idx), 0); };
@@ -140,6 +153,7 @@ thd_attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmap_q,
 
     if (threadIdx.x == 0) {
         mbar_init(bar(C::B_Q_FULL), 1);
+        mbar_init(bar(C::B_Q_EMPTY), 1);
         for (int s = 0; s < C::NSLOT; ++s) {
             mbar_init(bar(C::B_SLOT_FULL + s), 1);
             mbar_init(bar(C::B_SLOT_EMPTY + s), 1);
@@ -148,6 +162,7 @@ thd_attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmap_q,
             mbar_init(bar(C::B_S_FULL + q), 1);
             mbar_init(bar(C::B_P_FULL + q), 8);  // 4 softmax warps of each CTA
             mbar_init(bar(C::B_O_FULL + q), 1);
+            mbar_init(bar(C::B_O_FREE + q), 8);  // 4 softmax warps of each CTA
         }
         mbar_init(bar(C::B_DRAIN), 1);
         *abort_flag = launch_should_skip(p);
@@ -172,33 +187,45 @@ thd_attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 tma_prefetch_desc(&tmap_q);
                 tma_prefetch_desc(&tmap_k);
                 tma_prefetch_desc(&tmap_v);
-                const int g = it.head0 / p.G;
-                if (leader) mbar_arrive_expect_tx(bar(C::B_Q_FULL), 2 * C::NQ * C::Q_TILE_BYTES);
-                for (int q = 0; q < C::NQ; ++q)
-                    for (int c = 0; c < C::KCH; ++c)
-                        tma_load_3d_pair(sbase + C::SMEM_Q + q * C::Q_TILE_BYTES + c * C::Q_BOX_BYTES,
-                                         &tmap_q, lead_bar(C::B_Q_FULL), c * 64, head_base + q,
-                                         it.q0 - p.q_offset);
-                // Ring positions: 2j holds K(j), 2j+1 holds V(j).  This CTA
-                // loads keys [rank*BN/2, (rank+1)*BN/2) of K(j) and head-dim
-                // columns [rank*D/2, (rank+1)*D/2) of V(j).
                 bool ok = true;
-                for (int pos = 0; pos < 2 * n && ok; ++pos) {
-                    const int slot = pos % C::NSLOT;
-                    ok = mbar_wait(bar(C::B_SLOT_EMPTY + slot), ((pos / C::NSLOT) & 1) ^ 1,
-                                   abort_flag, p.status, kStatusTimeout);
-                    if (!ok) break;
-                    if (leader) mbar_arrive_expect_tx(bar(C::B_SLOT_FULL + slot), 2 * C::SLOT_BYTES);
-                    const uint32_t full = lead_bar(C::B_SLOT_FULL + slot);
-                    const uint32_t dst = sbase + C::SMEM_SLOTS + slot * C::SLOT_BYTES;
-                    const int kt = it.kv_start + (pos >> 1) * C::BN;
-                    if ((pos & 1) == 0) {
+                int pos = 0;  // ring position, continued across items
+                int done = 0;  // items loaded so far
+                for (int w = cluster_id; ok && w < n_items; w += n_clusters, ++done) {
+                    const WorkItem it = p.items[w];
+                    const int head_base = it.head0 + 2 * static_cast<int>(rank);
+                    const int g = it.head0 / p.G;
+                    // The previous item's Q tiles stay until its last QK is done.
+                    if (done > 0) {
+                        ok = mbar_wait(bar(C::B_Q_EMPTY), (done - 1) & 1, abort_flag, p.status,
+                                       kStatusTimeout);
+                        if (!ok) break;
+                    }
+                    if (leader) mbar_arrive_expect_tx(bar(C::B_Q_FULL), 2 * C::NQ * C::Q_TILE_BYTES);
+                    for (int q = 0; q < C::NQ; ++q)
                         for (int c = 0; c < C::KCH; ++c)
-                            tma_load_3d_pair(dst + c * C::KH_BOX_BYTES, &tmap_k, full, c * 64, g,
-                                             kt + static_cast<int>(rank) * C::KH_ROWS);
-                    } else {
-                        tma_load_3d_pair(dst, &tmap_v, full, static_cast<int>(rank) * C::VH_COLS, g,
-                                         kt);
+                            tma_load_3d_pair(sbase + C::SMEM_Q + q * C::Q_TILE_BYTES + c * C::Q_BOX_BYTES,
+                                             &tmap_q, lead_bar(C::B_Q_FULL), c * 64, head_base + q,
+                                             it.q0 - p.q_offset);
+                    // Ring positions: K(j) then V(j) for each key tile.  This
+                    // CTA loads keys [rank*BN/2, (rank+1)*BN/2) of K(j) and
+                    // head-dim columns [rank*D/2, (rank+1)*D/2) of V(j).
+                    for (int jj = 0; jj < 2 * it.n_kv; ++jj, ++pos) {
+                        const int slot = pos % C::NSLOT;
+                        ok = mbar_wait(bar(C::B_SLOT_EMPTY + slot), ((pos / C::NSLOT) & 1) ^ 1,
+                                       abort_flag, p.status, kStatusTimeout);
+                        if (!ok) break;
+                        if (leader) mbar_arrive_expect_tx(bar(C::B_SLOT_FULL + slot), 2 * C::SLOT_BYTES);
+                        const uint32_t full = lead_bar(C::B_SLOT_FULL + slot);
+                        const uint32_t dst = sbase + C::SMEM_SLOTS + slot * C::SLOT_BYTES;
+                        const int kt = it.kv_start + (jj >> 1) * C::BN;
+                        if ((jj & 1) == 0) {
+                            for (int c = 0; c < C::KCH; ++c)
+                                tma_load_3d_pair(dst + c * C::KH_BOX_BYTES, &tmap_k, full, c * 64, g,
+                                                 kt + static_cast<int>(rank) * C::KH_ROWS);
+                        } else {
+                            tma_load_3d_pair(dst, &tmap_v, full, static_cast<int>(rank) * C::VH_COLS,
+                                             g, kt);
+                        }
                     }
                 }
                 // On an abort, loads still in flight (they complete on the
@@ -245,39 +272,54 @@ thd_attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     return wait(C::B_SLOT_FULL + pos % C::NSLOT, (pos / C::NSLOT) & 1);
                 };
 
-                bool ok = wait(C::B_Q_FULL, 0) && wait_slot(0);
-                if (ok) {
+                bool ok = true;
+                int pos = 0;   // ring position of the item's K(0)
+                int tile = 0;  // key tiles of earlier items (S / P phases)
+                int done = 0;  // earlier items (Q / O phases)
+                for (int w = cluster_id; ok && w < n_items; w += n_clusters, ++done) {
+                    const int n = p.items[w].n_kv;
+                    ok = wait(C::B_Q_FULL, done & 1) && wait_slot(pos);
+                    if (!ok) break;
                     tc_fence_after();
                     for (int q = 0; q < C::NQ; ++q) {
-                        issue_qk(q, 0);
+                        issue_qk(q, pos % C::NSLOT);
                         mma2_commit_both(bar(C::B_S_FULL + q));
                     }
-                    mma2_commit_both(bar(C::B_SLOT_EMPTY + 0));  // K(0) consumed
-                }
-                for (int j = 0; ok && j < n; ++j) {
-                    // PV(j) and QK(j+1) of a head stream go out as one run
-                    // with one commit: S(j+1) ready also means O holds PV(j),
-                    // so O gets its own commit only after the last tile.
-                    const int vslot = (2 * j + 1) % C::NSLOT;
-                    const bool has_next = j + 1 < n;
-                    const int kslot = (2 * j + 2) % C::NSLOT;
-                    ok = wait_slot(2 * j + 1) && (!has_next || wait_slot(2 * j + 2));
-                    if (!ok) break;
-                    for (int q = 0; q < C::NQ && ok; ++q) {
-                        ok = wait(C::B_P_FULL + q, j & 1);
+                    mma2_commit_both(bar(C::B_SLOT_EMPTY + pos % C::NSLOT));  // K(0) consumed
+                    if (n == 1) mma2_commit_both(bar(C::B_Q_EMPTY));           // last QK of the item
+                    for (int j = 0; ok && j < n; ++j) {
+                        // PV(j) and QK(j+1) of a head stream go out as one run
+                        // with one commit: S(j+1) ready also means O holds
+                        // PV(j), so O gets its own commit only after the last
+                        // tile.
+                        const int vpos = pos + 2 * j + 1;
+                        const int kpos = pos + 2 * j + 2;
+                        const bool has_next = j + 1 < n;
+                        ok = wait_slot(vpos) && (!has_next || wait_slot(kpos));
                         if (!ok) break;
-                        tc_fence_after();
-                        issue_pv(q, vslot, j > 0);
+                        for (int q = 0; q < C::NQ && ok; ++q) {
+                            ok = wait(C::B_P_FULL + q, (tile + j) & 1);
+                            // PV(0) overwrites O: the previous item's O must be read.
+                            if (ok && j == 0 && done > 0) ok = wait(C::B_O_FREE + q, (done - 1) & 1);
+                            if (!ok) break;
+                            tc_fence_after();
+                            issue_pv(q, vpos % C::NSLOT, j > 0);
+                            if (has_next) {
+                                issue_qk(q, kpos % C::NSLOT);
+                                mma2_commit_both(bar(C::B_S_FULL + q));
+                            } else {
+                                mma2_commit_both(bar(C::B_O_FULL + q));
+                            }
+                        }
+                        if (!ok) break;
+                        mma2_commit_both(bar(C::B_SLOT_EMPTY + vpos % C::NSLOT));  // V(j) done
                         if (has_next) {
-                            issue_qk(q, kslot);
-                            mma2_commit_both(bar(C::B_S_FULL + q));
-                        } else {
-                            mma2_commit_both(bar(C::B_O_FULL + q));
+                            mma2_commit_both(bar(C::B_SLOT_EMPTY + kpos % C::NSLOT));  // K(j+1) done
+                            if (j + 2 == n) mma2_commit_both(bar(C::B_Q_EMPTY));  // last QK of the item
                         }
                     }
-                    if (!ok) break;
-                    mma2_commit_both(bar(C::B_SLOT_EMPTY + vslot));                   // V(j) done
-                    if (has_next) mma2_commit_both(bar(C::B_SLOT_EMPTY + kslot));   // K(j+1) done
+                    pos += 2 * n;
+                    tile += n;
                 }
                 // Every MMA issued by this thread has completed once this lands.
                 mma2_commit_both(bar(C::B_DRAIN));
@@ -291,110 +333,117 @@ thd_attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmap_q,
         const int q = warp >> 2;
         const int wq = warp & 3;
         const int row = wq * 32 + lane;
-        const int h = head_base + q;
-        const int i = it.q0 + row;  // token of this row
-        const int s_doc = it.doc_start;
-        const int r_lo = it.q0 > s_doc ? it.q0 : s_doc;
-        const int r_hi = it.q1 - 1;
-        const bool row_valid = i >= r_lo && i <= r_hi;
         const int W = p.window;
-        const int lo_i = (W > 0 && i - W + 1 > s_doc) ? i - W + 1 : s_doc;
         const float sl2 = p.scale_log2;
         constexpr float kTau = 8.0f;  // rescale only when the max grows by > 2^8
-
-        float m_ref = -INFINITY;
-        float l = 0.0f;
-        if (p.sinks != nullptr) {
-            m_ref = p.sinks[h] * 1.4426950408889634f;
-            l = 1.0f;
-        }
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(wq * 32) << 16);
         const uint32_t s_tmem = lane_base + C::TMEM_S + q * C::BN;
         const uint32_t o_tmem = lane_base + C::TMEM_O + q * C::D;
         const uint32_t p_full_leader = lead_bar(C::B_P_FULL + q);
+        const uint32_t o_free_leader = lead_bar(C::B_O_FREE + q);
 
         bool ok = !skip;
-        for (int j = 0; ok && j < n; ++j) {
-            // S(j) ready; for j > 0 this also means PV(j-1) is in O.
-            ok = warp_wait(bar(C::B_S_FULL + q), j & 1, abort_flag, p.status);
-            if (!ok) break;
-            tc_fence_after();
-            uint32_t sr[C::BN];
-#pragma unroll
-            for (int c = 0; c < C::BN / 32; ++c)
-                tmem_ld32(s_tmem + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < C::BN / 32; ++c)
-                reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
-            float sv[C::BN];
-#pragma unroll
-            for (int c = 0; c < C::BN; ++c) sv[c] = __uint_as_float(sr[c]);
+        int tile = 0, done = 0;
+        for (int w = cluster_id; ok && w < n_items; w += n_clusters, ++done) {
+            const WorkItem it = p.items[w];
+            const int n = it.n_kv;
+            const int h = it.head0 + 2 * static_cast<int>(rank) + q;
+            const int i = it.q0 + row;  // token of this row
+            const int s_doc = it.doc_start;
+            const int r_lo = it.q0 > s_doc ? it.q0 : s_doc;
+            const int r_hi = it.q1 - 1;
+            const bool row_valid = i >= r_lo && i <= r_hi;
+            const int lo_i = (W > 0 && i - W + 1 > s_doc) ? i - W + 1 : s_doc;
 
-            const int kt = it.kv_start + j * C::BN;
-            const bool full_tile = kt >= s_doc && kt + C::BN - 1 <= r_lo &&
-                                   (W == 0 || kt >= r_hi - W + 1);
-            if (!full_tile) {
-                const int c_lo = lo_i - kt;
-                const int c_hi = i - kt;
-#pragma unroll
-                for (int c = 0; c < C::BN; ++c)
-                    if (c < c_lo || c > c_hi) sv[c] = -INFINITY;
+            float m_ref = -INFINITY;
+            float l = 0.0f;
+            if (p.sinks != nullptr) {
+                m_ref = p.sinks[h] * 1.4426950408889634f;
+                l = 1.0f;
             }
-            float mx[4] = {sv[0], sv[1], sv[2], sv[3]};
-#pragma unroll
-            for (int c = 4; c < C::BN; c += 2) mx[(c >> 1) & 3] = max3f(mx[(c >> 1) & 3], sv[c], sv[c + 1]);
-            const float smax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-            const float m_tile = smax * sl2;
 
-            float alpha = 1.0f;
-            bool rescale_o = false;
-            if (j == 0) {
-                if (m_tile > m_ref) {
+            for (int j = 0; ok && j < n; ++j) {
+                // S(j) ready; for j > 0 this also means PV(j-1) is in O.
+                ok = warp_wait(bar(C::B_S_FULL + q), (tile + j) & 1, abort_flag, p.status);
+                if (!ok) break;
+                tc_fence_after();
+                uint32_t sr[C::BN];
+#pragma unroll
+                for (int c = 0; c < C::BN / 32; ++c)
+                    tmem_ld32(s_tmem + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < C::BN / 32; ++c)
+                    reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+                float sv[C::BN];
+#pragma unroll
+                for (int c = 0; c < C::BN; ++c) sv[c] = __uint_as_float(sr[c]);
+
+                const int kt = it.kv_start + j * C::BN;
+                const bool full_tile = kt >= s_doc && kt + C::BN - 1 <= r_lo &&
+                                       (W == 0 || kt >= r_hi - W + 1);
+                if (!full_tile) {
+                    const int c_lo = lo_i - kt;
+                    const int c_hi = i - kt;
+#pragma unroll
+                    for (int c = 0; c < C::BN; ++c)
+                        if (c < c_lo || c > c_hi) sv[c] = -INFINITY;
+                }
+                float mx[4] = {sv[0], sv[1], sv[2], sv[3]};
+#pragma unroll
+                for (int c = 4; c < C::BN; c += 2)
+                    mx[(c >> 1) & 3] = max3f(mx[(c >> 1) & 3], sv[c], sv[c + 1]);
+                const float smax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+                const float m_tile = smax * sl2;
+
+                float alpha = 1.0f;
+                bool rescale_o = false;
+                if (j == 0) {
+                    if (m_tile > m_ref) {
+                        alpha = ex2_approx(m_ref - m_tile);
+                        m_ref = m_tile;
+                    }
+                } else if (m_tile > m_ref + kTau) {
                     alpha = ex2_approx(m_ref - m_tile);
                     m_ref = m_tile;
+                    rescale_o = true;
                 }
-            } else if (m_tile > m_ref + kTau) {
-                alpha = ex2_approx(m_ref - m_tile);
-                m_ref = m_tile;
-                rescale_o = true;
-            }
-            l *= alpha;
-            const float neg_m = (m_ref == -INFINITY) ? 0.0f : -m_ref;
+                l *= alpha;
+                const float neg_m = (m_ref == -INFINITY) ? 0.0f : -m_ref;
 
-            if (j > 0 && __any_sync(0xffffffffu, rescale_o)) {
+                if (j > 0 && __any_sync(0xffffffffu, rescale_o)) {
 #pragma unroll 1
-                for (int c = 0; c < C::D / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(o_tmem + c * 32, r);
-                    tmem_wait_ld();
-                    reg_fence32(r);
+                    for (int c = 0; c < C::D / 32; ++c) {
+                        uint32_t r[32];
+                        tmem_ld32(o_tmem + c * 32, r);
+                        tmem_wait_ld();
+                        reg_fence32(r);
 #pragma unroll
-                    for (int u = 0; u < 32; u += 2) {
-                        const float2 y = __fmul2_rn(
-                            make_float2(__uint_as_float(r[u]), __uint_as_float(r[u + 1])),
-                            make_float2(alpha, alpha));
-                        r[u] = __float_as_uint(y.x);
-                        r[u + 1] = __float_as_uint(y.y);
+                        for (int u = 0; u < 32; u += 2) {
+                            const float2 y = __fmul2_rn(
+                                make_float2(__uint_as_float(r[u]), __uint_as_float(r[u + 1])),
+                                make_float2(alpha, alpha));
+                            r[u] = __float_as_uint(y.x);
+                            r[u + 1] = __float_as_uint(y.y);
+                        }
+                        tmem_st32(o_tmem + c * 32, r);
                     }
-                    tmem_st32(o_tmem + c * 32, r);
+                    tmem_wait_st();
                 }
+
+                const float2 sl2x2 = make_float2(sl2, sl2);
+                const float2 negm2 = make_float2(neg_m, neg_m);
+                float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+                exp_and_store_p<0, C::BN / 32, C::BN, C::EXP_EMU>(sv, sl2x2, negm2, s_tmem, acc0, acc1);
                 tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(p_full_leader);
+                l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
             }
 
-            const float2 sl2x2 = make_float2(sl2, sl2);
-            const float2 negm2 = make_float2(neg_m, neg_m);
-            float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-            exp_and_store_p<0, C::BN / 32, C::BN, C::EXP_EMU>(sv, sl2x2, negm2, s_tmem, acc0, acc1);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(p_full_leader);
-            l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
-        }
-
-        if (ok) ok = warp_wait(bar(C::B_O_FULL + q), 0, abort_flag, p.status);
-        if (ok) {
+            if (ok) ok = warp_wait(bar(C::B_O_FULL + q), done & 1, abort_flag, p.status);
+            if (!ok) break;
             tc_fence_after();
             const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
             __nv_bfloat16* orow = p.out + (static_cast<int64_t>(i - p.q_offset) * p.Hq + h) * C::D;
@@ -404,21 +453,28 @@ thd_attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 tmem_ld32(o_tmem + c * 32, r);
                 tmem_wait_ld();
                 reg_fence32(r);
-                uint32_t w[16];
+                if (c == C::D / 32 - 1) {
+                    // O is read: the next item's PV(0) may overwrite it.
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(o_free_leader);
+                }
+                uint32_t wv[16];
 #pragma unroll
                 for (int u = 0; u < 16; ++u)
-                    w[u] = pack_bf16x2(__uint_as_float(r[2 * u]) * inv_l,
-                                       __uint_as_float(r[2 * u + 1]) * inv_l);
+                    wv[u] = pack_bf16x2(__uint_as_float(r[2 * u]) * inv_l,
+                                        __uint_as_float(r[2 * u + 1]) * inv_l);
                 if (row_valid) {
                     uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
-                        dst[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+                        dst[u] = make_uint4(wv[4 * u], wv[4 * u + 1], wv[4 * u + 2], wv[4 * u + 3]);
                 }
             }
             if (row_valid && p.lse != nullptr)
                 p.lse[static_cast<int64_t>(i - p.q_offset) * p.Hq + h] =
                     l > 0.0f ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
+            tile += n;
         }
     }
 
@@ -438,6 +494,35 @@ inline bool pair_launch_registers_ok() {
     cudaFuncAttributes a{};
     if (cudaFuncGetAttributes(&a, thd_attn_fwd_pair_kernel<C>) != cudaSuccess) return false;
     return a.numRegs >= C::LAUNCH_REGS;
+}
+
+// Clusters of the persistent grid: as many as can be resident at once (one
+// per SM pair), found once per device after the shared-memory attribute is
+// set.  Returns 0 on failure.
+template <class C>
+inline int pair_max_active_clusters() {
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(C::NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_ALLOC;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, thd_attn_fwd_pair_kernel<C>, &cfg) != cudaSuccess) return 0;
+    return n;
+}
+
+// Grid of a launch over n_items items: one cluster per item, or with the
+// persistent grid at most max_clusters clusters that loop over the items.
+inline unsigned pair_grid(int64_t n_items, int max_clusters) {
+    int64_t c = n_items;
+    if (THD_PAIR_PERSIST && max_clusters > 0 && c > max_clusters) c = max_clusters;
+    return static_cast<unsigned>(2 * c);
 }
 
 }  // namespace thd
