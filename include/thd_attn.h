@@ -57,8 +57,10 @@ enum thd_status {
     THD_ERR_TIMEOUT = -4,      /* a bounded wait inside the kernel ran out */
     THD_ERR_NO_MEMORY = -5,    /* the schedule cache could not be allocated */
     THD_ERR_TOO_LARGE = -6,    /* thd_attn_fwd_noalloc: the schedule exceeds its fixed scratch */
-    THD_ERR_STALE_SCRATCH = -7 /* thd_attn_fwd_noalloc: a launch found another call's schedule
-                                  in the shared scratch and did nothing */
+    THD_ERR_STALE_SCRATCH = -7, /* thd_attn_fwd_noalloc: a launch found another call's schedule
+                                   in the shared scratch and did nothing */
+    THD_ERR_BAD_ITEM = -8       /* debug builds (THD_DEBUG=1) only: a forward CTA found a work
+                                   item that breaks the schedule's invariants and did nothing */
 };
 
 /*

@@ -32,7 +32,7 @@ _lib = None
 
 STATUS = {0: "THD_OK", -1: "THD_ERR_INVALID_ARG", -2: "THD_ERR_UNSUPPORTED", -3: "THD_ERR_CUDA",
           -4: "THD_ERR_TIMEOUT", -5: "THD_ERR_NO_MEMORY", -6: "THD_ERR_TOO_LARGE",
-          -7: "THD_ERR_STALE_SCRATCH"}
+          -7: "THD_ERR_STALE_SCRATCH", -8: "THD_ERR_BAD_ITEM"}
 
 WORK_ITEM_FIELDS = ("q0", "q1", "doc_start", "head0", "kv_start", "n_kv", "n_heads", "block_n")
 
@@ -62,7 +62,13 @@ def load_library():
         raise ImportError(
             f"{path} is missing: build it with `python -m sliding_window_gqa_cu_b200.build` "
             "(there is no CPU fallback)")
-    lib = ctypes.CDLL(path)
+    _lib = bind(ctypes.CDLL(path))
+    return _lib
+
+
+def bind(lib):
+    """Declare the argument and result types of every entry point on a loaded
+    copy of the library (``load_library`` does this for the in-tree build)."""
     vp, i32p, c_int = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32), ctypes.c_int
     lib.thd_attn_fwd.argtypes = [vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int,
                                  ctypes.c_float, vp, vp, vp, vp]
@@ -109,7 +115,6 @@ def load_library():
     lib.thd_qk_norm_rope.restype = c_int
     lib.thd_attn_abi_version.argtypes = []
     lib.thd_attn_abi_version.restype = c_int
-    _lib = lib
     return lib
 
 

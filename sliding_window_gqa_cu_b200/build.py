@@ -37,17 +37,25 @@ def needs_build() -> bool:
     return any(os.path.getmtime(p) > t for p in DEPS if os.path.exists(p))
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if not force and not needs_build():
+def build(force: bool = False, verbose_ptxas: bool = False, out: str = LIB,
+          defines: tuple = ()) -> str:
+    """Build the library (if a source is newer) into ``out``; ``defines`` are
+    extra ``-D`` flags (e.g. ``("THD_DEBUG=1",)`` for the debug build, which a
+    different ``out`` keeps apart from the regular library)."""
+    if out == LIB and not defines and not force and not needs_build():
         return LIB
+    if out != LIB and not force and os.path.exists(out) and \
+            all(os.path.getmtime(p) <= os.path.getmtime(out) for p in DEPS if os.path.exists(p)):
+        return out
     cmd = [nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo",
            "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-shared", "--expt-relaxed-constexpr",
-           "-I", os.path.join(ROOT, "include"), "-o", LIB + ".tmp", *SOURCES]
+           *[f"-D{d}" for d in defines],
+           "-I", os.path.join(ROOT, "include"), "-o", out + ".tmp", *SOURCES]
     if verbose_ptxas:
         cmd[1:1] = ["-Xptxas", "-v"]
     subprocess.run(cmd, check=True)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(out + ".tmp", out)
+    return out
 
 
 def main(argv=None) -> int:

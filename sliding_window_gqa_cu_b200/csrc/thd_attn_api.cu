@@ -428,6 +428,7 @@ const char* thd_attn_status_string(int status) {
         case THD_ERR_NO_MEMORY: return "out of device memory for the schedule cache";
         case THD_ERR_TOO_LARGE: return "schedule larger than the allocation-free scratch (65,536 work items)";
         case THD_ERR_STALE_SCRATCH: return "the allocation-free scratch held another call's schedule; nothing was computed";
+        case THD_ERR_BAD_ITEM: return "debug build: a work item broke the schedule's invariants; nothing was computed";
         default: return "unknown status";
     }
 }

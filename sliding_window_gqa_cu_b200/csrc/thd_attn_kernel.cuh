@@ -35,6 +35,14 @@
 #define THD_EXP_EMU 0
 #endif
 
+// 1: debug build.  Every forward CTA checks the work items it will run
+// against the schedule's invariants before touching memory and, on a
+// violation, records kStatusBadItem in the status word and does nothing
+// (a status code instead of a trap or a fault).
+#ifndef THD_DEBUG
+#define THD_DEBUG 0
+#endif
+
 namespace thd {
 
 struct WorkItem {  // identical layout to thd_work_item in thd_attn.h
@@ -139,6 +147,32 @@ struct FwdParams {
 // allocation-free scratch (the launch then does nothing).
 constexpr int kStatusStaleScratch = -7;
 
+// Error code of the debug build's work-item checks.
+constexpr int kStatusBadItem = -8;
+
+// Debug build: the invariants every item of the host schedule satisfies
+// (see scheduler.cpp): 1..128 query rows ending in the document, key tiles
+// of block_n keys that end at the tile end, whole GQA head groups of
+// n_heads aligned heads inside [0, Hq).
+__device__ __forceinline__ bool item_ok(const WorkItem& it, const FwdParams& p, int n_heads,
+                                        int block_n) {
+    return it.n_kv >= 1 && it.block_n == block_n && it.n_heads == n_heads &&
+           it.q1 - it.q0 >= 1 && it.q1 - it.q0 <= 128 && it.doc_start < it.q1 &&
+           it.q0 - p.q_offset >= -128 && it.kv_start + it.n_kv * block_n == it.q1 &&
+           it.head0 >= 0 && it.head0 % n_heads == 0 && it.head0 + n_heads <= p.Hq &&
+           (it.head0 / p.G) == (it.head0 + n_heads - 1) / p.G;
+}
+
+// Debug build: record kStatusBadItem and return 1 if the item fails item_ok.
+__device__ __forceinline__ int debug_check_item(const WorkItem& it, const FwdParams& p, int n_heads,
+                                                int block_n) {
+    if (THD_DEBUG && !item_ok(it, p, n_heads, block_n)) {
+        atomicCAS(p.status, 0, kStatusBadItem);
+        return 1;
+    }
+    return 0;
+}
+
 // CTA start-up decision, taken by one thread: skip the work if an earlier
 // CTA or launch recorded an error that the host has not read yet, or if the
 // schedule this launch was enqueued for is no longer in place.
@@ -237,7 +271,7 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         mbar_init(bar(C::B_DRAIN), 1);
         // A timeout recorded by an earlier CTA (or launch) makes every later
         // CTA skip its work until the host reads and clears the status.
-        *abort_flag = launch_should_skip(p);
+        *abort_flag = launch_should_skip(p) | debug_check_item(it, p, C::NQ, C::BN);
         fence_barrier_init();
     }
     if (warp == C::MMA_WARP) {

@@ -165,7 +165,11 @@ thd_attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmap_q,
             mbar_init(bar(C::B_O_FREE + q), 8);  // 4 softmax warps of each CTA
         }
         mbar_init(bar(C::B_DRAIN), 1);
-        *abort_flag = launch_should_skip(p);
+        int bad = 0;
+        if (THD_DEBUG)
+            for (int w = cluster_id; w < n_items && !bad; w += n_clusters)
+                bad = debug_check_item(p.items[w], p, 2 * C::NQ, C::BN);
+        *abort_flag = launch_should_skip(p) | bad;
         fence_barrier_init();
     }
     if (warp == C::MMA_WARP) {

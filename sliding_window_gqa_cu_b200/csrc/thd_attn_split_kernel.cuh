@@ -146,7 +146,7 @@ thd_attn_fwd_split_kernel(const __grid_constant__ CUtensorMap tmap_q,
         mbar_init(bar(C::B_O_FULL), 1);
         mbar_init(bar(C::B_XCH), 8);  // the 8 softmax warps of this CTA
         mbar_init(bar(C::B_DRAIN), 1);
-        *abort_flag = launch_should_skip(p);
+        *abort_flag = launch_should_skip(p) | debug_check_item(it, p, 2, C::BN);
         fence_barrier_init();
     }
     if (warp == C::MMA_WARP) {
