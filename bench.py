@@ -60,13 +60,8 @@ DATASHEET_BF16_TFLOPS = 2250.0
 def kernel_name(D: int, group: int) -> str:
     """The kernel the library launches for this shape (label only): the
     CTA-pair kernel with the key-split softmax at head dim 256 with an even
-    GQA group, the CTA-pair kernel with two heads per CTA at head dim 128
-    with a group that is a multiple of four, else the one-CTA kernel."""
-    if D == 256 and group % 2 == 0:
-        return "thd_attn_fwd_split_kernel"
-    if D == 128 and group % 4 == 0:
-        return "thd_attn_fwd_pair_kernel"
-    return "thd_attn_fwd_kernel"
+    GQA group, else the one-CTA kernel."""
+    return "thd_attn_fwd_split_kernel" if D == 256 and group % 2 == 0 else "thd_attn_fwd_kernel"
 
 
 def log(*a):
@@ -115,7 +110,7 @@ def measured_peaks():
 E2E_CHUNKS = 16  # token ranges of the end-to-end call (copies overlap the attention)
 
 TRAFFIC_SOURCES = ("sm100_ptx.cuh", "thd_attn_kernel.cuh", "thd_attn_split_kernel.cuh",
-                   "thd_attn_pair_kernel.cuh", "scheduler.cpp", "scheduler.h")
+                   "scheduler.cpp", "scheduler.h")
 
 
 def kernel_source_hash() -> str:

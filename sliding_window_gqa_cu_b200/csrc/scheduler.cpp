@@ -7,22 +7,19 @@ namespace thd {
 
 bool choose_kernel_shape(int D, int group, KernelShape* out) {
     // One CTA per item with two heads of one kv group (even group) or one
-    // head; at D = 128 with a group that is a multiple of four, a CTA pair
-    // per item with two heads per CTA (M = 256 instructions, each CTA loading
-    // half of every K and V tile, whole score rows per CTA); at D = 256 with
-    // an even group, the CTA-pair kernel with the key-split softmax (one head
-    // per CTA, two per item), whose M = 256 instructions keep N = 256 PV and
-    // N = 128 QK at the tensor core's full rate.
+    // head; at D = 256 with an even group, the CTA-pair kernel with the
+    // key-split softmax (one head per CTA, two per item), whose M = 256
+    // instructions keep N = 256 PV and N = 128 QK at the tensor core's full
+    // rate.  (At D = 128 every CTA-pair design measured slower than the
+    // one-CTA kernel, including one with whole score rows and two heads per
+    // CTA: there the tensor core waits on the softmax, and the pair's
+    // cross-CTA signals lengthen that chain.)
     const bool two = (group % 2) == 0;
     switch (D) {
         case 64:
             *out = two ? KernelShape{64, 2, 1, 128, 8, false} : KernelShape{64, 1, 2, 128, 8, false};
             return true;
         case 128:
-            if (THD_PAIR128 && group % 4 == 0) {
-                *out = KernelShape{128, 4, 1, 128, 8, true};
-                return true;
-            }
             *out = two ? KernelShape{128, 2, 1, 128, 5, false} : KernelShape{128, 1, 2, 128, 6, false};
             return true;
         case 256:

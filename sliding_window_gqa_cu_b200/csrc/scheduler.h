@@ -13,19 +13,12 @@
 
 #include "../../include/thd_attn.h"
 
-// 1: head dim 128 with a GQA group that is a multiple of four runs on the
-// CTA-pair kernel with two heads per CTA (thd_attn_pair_kernel.cuh); 0: on
-// the one-CTA kernel with two heads per CTA.
-#ifndef THD_PAIR128
-#define THD_PAIR128 1
-#endif
-
 namespace thd {
 
 // Kernel shape chosen for a head dim and GQA group size.
 struct KernelShape {
     int D;
-    int nq;       // query heads per work item (1, 2 or 4)
+    int nq;       // query heads per work item (1 or 2)
     int nsb;      // S buffers per query tile
     int block_n;  // keys per key tile
     int nslot;    // K/V ring slots (one K or V tile each)

@@ -18,7 +18,6 @@
 #include "tma_map.h"
 #include "thd_attn_kernel.cuh"
 #include "thd_attn_split_kernel.cuh"
-#include "thd_attn_pair_kernel.cuh"
 #include "thd_attn_bwd_kernels.cuh"
 
 namespace {
@@ -33,12 +32,11 @@ using Cfg128x2 = thd::FwdConfig<128, 2, 1, 128, 5>;
 using Cfg128x1 = thd::FwdConfig<128, 1, 2, 128, 6>;
 using Cfg256x1 = thd::FwdConfig<256, 1, 2, 64, 5>;
 using SplitCfg256 = thd::SplitConfig<256, 2, 4>;  // 2 heads per item over a CTA pair
-using PairCfg128 = thd::PairConfig<128, 8, THD_PAIR_EXP_EMU>;  // 4 heads per item over a CTA pair
 
-constexpr int kNumVariants = 7;
+constexpr int kNumVariants = 6;
 
 int variant_index(const KernelShape& ks) {
-    if (ks.pair) return ks.D == 256 ? 5 : 6;
+    if (ks.pair) return 5;
     if (ks.D == 64) return ks.nq == 2 ? 0 : 1;
     if (ks.D == 128) return ks.nq == 2 ? 2 : 3;
     return 4;
@@ -69,7 +67,6 @@ constexpr int kNumBwdVariants = 7;  // {dq, dkdv} x {D = 64, D = 128}, then dq, 
 
 struct DeviceState {
     int* d_status = nullptr;
-    int pair_clusters = 0;  // resident clusters of the head-dim-128 pair kernel
     bool attr_set[kNumVariants] = {};
     bool bwd_attr_set[kNumBwdVariants] = {};
     std::list<PlanEntry> plans;         // most recently used first
@@ -181,25 +178,6 @@ int launch_pair(DeviceState* ds, int vidx, const PlanEntry& plan, const CUtensor
         ds->attr_set[vidx] = true;
     }
     kern<<<static_cast<unsigned>(2 * plan.n_items), C::NUM_THREADS, C::SMEM_ALLOC, stream>>>(
-        mq, mk, mv, prm);
-    return cudaGetLastError() == cudaSuccess ? THD_OK : THD_ERR_CUDA;
-}
-
-// CTA-pair shapes with two heads per CTA: two CTAs (one cluster) per item.
-template <class C>
-int launch_pair2(DeviceState* ds, int vidx, const PlanEntry& plan, const CUtensorMap& mq,
-                 const CUtensorMap& mk, const CUtensorMap& mv, const thd::FwdParams& prm,
-                 cudaStream_t stream) {
-    auto kern = thd::thd_attn_fwd_pair_kernel<C>;
-    if (!ds->attr_set[vidx]) {
-        if (!thd::pair_launch_registers_ok<C>()) return THD_ERR_UNSUPPORTED;
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM_ALLOC) != cudaSuccess)
-            return THD_ERR_CUDA;
-        ds->pair_clusters = thd::pair_max_active_clusters<C>();
-        ds->attr_set[vidx] = true;
-    }
-    kern<<<thd::pair_grid(plan.n_items, ds->pair_clusters), C::NUM_THREADS, C::SMEM_ALLOC, stream>>>(
         mq, mk, mv, prm);
     return cudaGetLastError() == cudaSuccess ? THD_OK : THD_ERR_CUDA;
 }
@@ -506,7 +484,6 @@ int thd_attn_fwd_range(const void* q, const void* k, const void* v, const int32_
     prm.window = window;
     prm.scale_log2 = scale * 1.4426950408889634f;
     prm.q_offset = static_cast<int>(q_begin);
-    prm.n_items = static_cast<int>(plan->n_items);
 
     switch (variant_index(ks)) {
         case 0: return launch<Cfg64x2>(ds, 0, *plan, mq, mk, mv, prm, stream);
@@ -514,8 +491,7 @@ int thd_attn_fwd_range(const void* q, const void* k, const void* v, const int32_
         case 2: return launch<Cfg128x2>(ds, 2, *plan, mq, mk, mv, prm, stream);
         case 3: return launch<Cfg128x1>(ds, 3, *plan, mq, mk, mv, prm, stream);
         case 4: return launch<Cfg256x1>(ds, 4, *plan, mq, mk, mv, prm, stream);
-        case 5: return launch_pair<SplitCfg256>(ds, 5, *plan, mq, mk, mv, prm, stream);
-        default: return launch_pair2<PairCfg128>(ds, 6, *plan, mq, mk, mv, prm, stream);
+        default: return launch_pair<SplitCfg256>(ds, 5, *plan, mq, mk, mv, prm, stream);
     }
 }
 

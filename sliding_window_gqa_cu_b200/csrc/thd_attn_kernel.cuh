@@ -135,7 +135,6 @@ struct FwdParams {
     int window;
     float scale_log2;    // scale * log2(e)
     int q_offset;        // pack row of row 0 of q / out / lse (0 unless a token range)
-    int n_items = 0;     // work items in the schedule (kernels that loop over items)
     // Optional schedule check (allocation-free entry point): when set, the
     // launch runs only if *plan_tag equals expected_tag, i.e. the shared
     // scratch still holds the schedule this launch was enqueued for.

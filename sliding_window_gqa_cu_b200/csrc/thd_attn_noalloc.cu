@@ -41,7 +41,6 @@
 #include "tma_map.h"
 #include "thd_attn_kernel.cuh"
 #include "thd_attn_split_kernel.cuh"
-#include "thd_attn_pair_kernel.cuh"
 
 namespace {
 
@@ -57,8 +56,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 struct NoAllocDevice {
     bool ready = false;
     unsigned char* scratch = nullptr;  // device address of g_noalloc_scratch
-    bool attr_set[7] = {};
-    int pair_clusters = 0;  // resident clusters of the head-dim-128 pair kernel
+    bool attr_set[6] = {};
     // arguments of the schedule now in the scratch (valid when have_plan)
     bool have_plan = false;
     int n_docs = 0, Hq = 0, Hkv = 0, D = 0, window = 0;
@@ -88,7 +86,6 @@ using NCfg128x2 = thd::FwdConfig<128, 2, 1, 128, 5>;
 using NCfg128x1 = thd::FwdConfig<128, 1, 2, 128, 6>;
 using NCfg256x1 = thd::FwdConfig<256, 1, 2, 64, 5>;
 using NSplitCfg256 = thd::SplitConfig<256, 2, 4>;  // 2 heads per item over a CTA pair
-using NPairCfg128 = thd::PairConfig<128, 8, THD_PAIR_EXP_EMU>;  // 4 heads per item over a CTA pair
 
 using thd::aligned16;
 using thd::make_map;
@@ -183,24 +180,6 @@ int launch_pair(NoAllocDevice* st, int vidx, int64_t n_items, const CUtensorMap&
     return cudaGetLastError() == cudaSuccess ? THD_OK : THD_ERR_CUDA;
 }
 
-template <class C>
-int launch_pair2(NoAllocDevice* st, int vidx, int64_t n_items, const CUtensorMap& mq,
-                 const CUtensorMap& mk, const CUtensorMap& mv, const thd::FwdParams& prm,
-                 cudaStream_t stream) {
-    auto kern = thd::thd_attn_fwd_pair_kernel<C>;
-    if (!st->attr_set[vidx]) {
-        if (!thd::pair_launch_registers_ok<C>()) return THD_ERR_UNSUPPORTED;
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM_ALLOC) != cudaSuccess)
-            return THD_ERR_CUDA;
-        st->pair_clusters = thd::pair_max_active_clusters<C>();
-        st->attr_set[vidx] = true;
-    }
-    kern<<<thd::pair_grid(n_items, st->pair_clusters), C::NUM_THREADS, C::SMEM_ALLOC, stream>>>(
-        mq, mk, mv, prm);
-    return cudaGetLastError() == cudaSuccess ? THD_OK : THD_ERR_CUDA;
-}
-
 }  // namespace
 
 extern "C" int thd_attn_fwd_noalloc(const void* q, const void* k, const void* v,
@@ -285,12 +264,10 @@ extern "C" int thd_attn_fwd_noalloc(const void* q, const void* k, const void* v,
     prm.window = window;
     prm.scale_log2 = scale * 1.4426950408889634f;
     prm.q_offset = 0;
-    prm.n_items = static_cast<int>(n_items);
     prm.plan_tag = reinterpret_cast<const unsigned long long*>(st->scratch + kTagOffset);
     prm.expected_tag = st->tag;
 
-    if (ks.pair && D == 256) return launch_pair<NSplitCfg256>(st, 5, n_items, mq, mk, mv, prm, stream);
-    if (ks.pair) return launch_pair2<NPairCfg128>(st, 6, n_items, mq, mk, mv, prm, stream);
+    if (ks.pair) return launch_pair<NSplitCfg256>(st, 5, n_items, mq, mk, mv, prm, stream);
     if (D == 64) {
         return ks.nq == 2 ? launch<NCfg64x2>(st, 0, n_items, mq, mk, mv, prm, stream)
                           : launch<NCfg64x1>(st, 1, n_items, mq, mk, mv, prm, stream);

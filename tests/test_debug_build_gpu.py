@@ -25,7 +25,7 @@ def debug_lib():
 
 @pytest.mark.parametrize("lens,Hq,Hkv,D,window,sinks", [
     ([300, 1, 0, 129, 77], 4, 2, 64, 100, True),   # one CTA, two heads
-    ([390, 5, 128, 1, 200], 8, 2, 128, 0, True),   # CTA pair, four heads per item
+    ([390, 5, 128, 1, 200], 8, 2, 128, 0, True),   # one CTA, two heads, G = 4
     ([400, 77], 4, 2, 128, 0, False),               # one CTA, two heads
     ([300, 9], 6, 2, 128, 50, True),                # one head per item
     ([520, 3], 16, 1, 256, 0, True),                # CTA pair, key-split softmax
