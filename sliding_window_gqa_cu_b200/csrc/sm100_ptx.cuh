@@ -77,11 +77,30 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // microseconds; two seconds means the pipeline is stuck.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
+// Non-blocking test of a phase (the thread is never suspended).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done) : "r"(bar), "r"(parity) : "memory");
+    return done != 0;
+}
+
 // Wait until the phase with the given parity has completed.  Returns false
 // (after recording `code` in *status and raising the CTA's abort flag) if
 // the limit runs out, or if another role of the CTA has already aborted.
+// With spin, the first polls never suspend the thread (for a thread whose
+// reaction time is on the critical path and whose polls cost little).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
-                                          volatile int* abort_flag, int* status, int code) {
+                                          volatile int* abort_flag, int* status, int code,
+                                          bool spin_first = false) {
+    if (spin_first) {
+#pragma unroll 1
+        for (int spin = 0; spin < 4096; ++spin)
+            if (mbar_test_wait(bar, parity)) return true;
+    }
     // Fast path: plain polling (try_wait itself suspends briefly in hardware).
 #pragma unroll 1
     for (int spin = 0; spin < 256; ++spin)

@@ -43,6 +43,12 @@
 #define THD_DEBUG 0
 #endif
 
+// 1: the MMA-issuing thread polls its barriers without suspending before it
+// falls back to the suspending wait.
+#ifndef THD_MMA_SPIN
+#define THD_MMA_SPIN 0
+#endif
+
 namespace thd {
 
 struct WorkItem {  // identical layout to thd_work_item in thd_attn.h
@@ -361,7 +367,7 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
 
             auto wait_slot = [&](int pos) -> bool {
                 return mbar_wait(bar(C::B_SLOT_FULL + pos % C::NSLOT), (pos / C::NSLOT) & 1,
-                                 abort_flag, p.status, kStatusTimeout);
+                                 abort_flag, p.status, kStatusTimeout, THD_MMA_SPIN != 0);
             };
             bool ok = mbar_wait(bar(C::B_Q_FULL), 0, abort_flag, p.status, kStatusTimeout);
             for (int jj = 0; ok && jj < C::NSB && jj < n; ++jj) {
@@ -387,7 +393,8 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 ok = wait_slot(2 * j + 1) && (!has_next || wait_slot(2 * j + 2));
                 if (!ok) break;
                 for (int q = 0; q < C::NQ && ok; ++q) {
-                    ok = mbar_wait(bar(C::B_P_FULL + q), j & 1, abort_flag, p.status, kStatusTimeout);
+                    ok = mbar_wait(bar(C::B_P_FULL + q), j & 1, abort_flag, p.status, kStatusTimeout,
+                                   THD_MMA_SPIN != 0);
                     if (!ok) break;
                     tc_fence_after();
                     issue_pv(q, 0, vslot, j > 0);
@@ -410,7 +417,8 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 const bool has_next = jn < n;
                 const int kslot = (2 * jn) % C::NSLOT;
                 for (int q = 0; q < C::NQ && ok; ++q) {
-                    ok = mbar_wait(bar(C::B_P_FULL + q), j & 1, abort_flag, p.status, kStatusTimeout);
+                    ok = mbar_wait(bar(C::B_P_FULL + q), j & 1, abort_flag, p.status, kStatusTimeout,
+                                   THD_MMA_SPIN != 0);
                     if (!ok) break;
                     tc_fence_after();
                     issue_pv(q, j % C::NSB, vslot, j > 0);
