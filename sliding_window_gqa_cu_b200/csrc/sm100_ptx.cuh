@@ -446,6 +446,21 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
     return make_float2(__int_as_float(ex), __int_as_float(ey));
 }
 
+// 2^x of two values on MUFU's half-precision path: x rounded to f16 (x <= 0
+// here; for |x| < 8 the rounding moves 2^x by at most 0.14 %, and larger |x|
+// give terms below 2^-8), two results from one ex2.approx.f16x2, widened to
+// fp32.
+__device__ __forceinline__ float2 exp2_f16x2(float2 x) {
+    uint32_t h, r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(x.y), "f"(x.x));
+    asm("ex2.approx.f16x2 %0, %1;" : "=r"(r) : "r"(h));
+    float lo, hi;
+    asm("{\n\t.reg .f16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+        "cvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
+        : "=f"(lo), "=f"(hi) : "r"(r));
+    return make_float2(lo, hi);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     // cvt packs its first source into the upper half.
     uint32_t r;

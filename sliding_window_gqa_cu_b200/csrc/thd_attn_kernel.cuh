@@ -49,6 +49,12 @@
 #define THD_MMA_SPIN 0
 #endif
 
+// 1: the softmax exponentials of the one-CTA kernel use MUFU's f16x2 path
+// (two exponentials per instruction).
+#ifndef THD_EXP_F16
+#define THD_EXP_F16 0
+#endif
+
 namespace thd {
 
 struct WorkItem {  // identical layout to thd_work_item in thd_attn.h
@@ -228,6 +234,10 @@ __device__ __forceinline__ void exp_and_store_p(const float (&sv)[BN], float2 sl
             float p0, p1;
             if ((u & 3) >= 4 - EMU) {
                 const float2 e = exp2_poly2(x);
+                p0 = e.x;
+                p1 = e.y;
+            } else if (THD_EXP_F16) {
+                const float2 e = exp2_f16x2(x);
                 p0 = e.x;
                 p1 = e.y;
             } else {
