@@ -20,8 +20,7 @@
 //     tensor core computes dq(j), dP(j + 1) and S(j + 2) while the
 //     elementwise warps exponentiate S(j + 1).
 //   * dkdv kernel: one CTA per (128-key tile, kv head), looping over the
-//     query tiles that see the keys (from the document end backward) and,
-//     for each, the query heads of the group:
+//     query heads of the group and the 128-query tiles that see the keys:
 //     S^T = K Q^T and dP^T = V dO^T (TMEM lane = key), P^T and dS^T written as
 //     bf16 over them, dv += P^T dO and dk += dS^T Q (TMEM operands, dO and Q
 //     as MN-major operands); dk and dv stay in TMEM for the whole group.
@@ -575,12 +574,8 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
             const int pr = s % L::NPAIR;
             ok = warp_wait(bar(L::B_PAIR_EMPTY + pr), ((s / L::NPAIR) & 1) ^ 1, abort_flag, prm.status);
             if (!ok) break;
-            // Step s: query tile nsub - 1 - s / G (from the document end
-            // backward), query head g G + s % G.  The CTAs of one document
-            // start at its end together and walk the same Q / dO tiles at
-            // about the same time, so they share them in L2.
-            const int h = it.g * G + s % G;
-            const int i0 = it.k0 + (nsub - 1 - s / G) * C::BN;
+            const int h = it.g * G + s / nsub;
+            const int i0 = it.k0 + (s % nsub) * C::BN;
             if (lane == 0) {
                 const uint32_t full = bar(L::B_PAIR_FULL + pr);
                 const uint32_t dst = sbase + L::SMEM_PAIRS + pr * L::PAIR_BYTES;
@@ -695,7 +690,7 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
         constexpr int HALF = C::HALF;
         for (int s = 0; ok && s < n_steps; ++s) {
             const int pr = s % L::NPAIR;
-            const int ih = it.k0 + (nsub - 1 - s / G) * C::BN + HALF * h;  // first query of this half
+            const int ih = it.k0 + (s % nsub) * C::BN + HALF * h;  // first query of this half
             // The side values of this step were stored before PAIR_FULL.
             ok = warp_wait(bar(L::B_PAIR_FULL + pr), (s / L::NPAIR) & 1, abort_flag, prm.status) &&
                  warp_wait(bar(L::B_S_FULL), s & 1, abort_flag, prm.status);
