@@ -55,6 +55,13 @@
 #define THD_EXP_F16 0
 #endif
 
+// 1: with one S buffer per head, the softmax publishes P in two halves (keys
+// [0, BN/2) and [BN/2, BN)), so PV starts on the first half while the second
+// half's exponentials are still running.
+#ifndef THD_P_SPLIT
+#define THD_P_SPLIT 0
+#endif
+
 namespace thd {
 
 struct WorkItem {  // identical layout to thd_work_item in thd_attn.h
@@ -111,8 +118,10 @@ struct FwdConfig {
     static constexpr int B_SLOT_FULL = 1;
     static constexpr int B_SLOT_EMPTY = B_SLOT_FULL + NSLOT;
     static constexpr int B_S_FULL = B_SLOT_EMPTY + NSLOT;  // [NQ][NSB]
-    static constexpr int B_P_FULL = B_S_FULL + NQ * NSB;   // P written, O rescaled
-    static constexpr int B_O_FULL = B_P_FULL + NQ;         // PV done
+    static constexpr int B_P_FULL = B_S_FULL + NQ * NSB;   // [NQ][2] P (half) written, O rescaled
+    static constexpr int B_O_FULL = B_P_FULL + 2 * NQ;     // PV done
+    // P published in two halves (one S buffer per head only).
+    static constexpr bool P_SPLIT = THD_P_SPLIT != 0 && NSB == 1;
     static constexpr int B_DRAIN = B_O_FULL + NQ;
     static constexpr int NUM_BARS = B_DRAIN + 1;
 
@@ -280,7 +289,8 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
         }
         for (int i = 0; i < C::NQ * C::NSB; ++i) mbar_init(bar(C::B_S_FULL + i), 1);
         for (int q = 0; q < C::NQ; ++q) {
-            mbar_init(bar(C::B_P_FULL + q), 4);
+            mbar_init(bar(C::B_P_FULL + 2 * q), 4);
+            mbar_init(bar(C::B_P_FULL + 2 * q + 1), 4);
             mbar_init(bar(C::B_O_FULL + q), 1);
         }
         mbar_init(bar(C::B_DRAIN), 1);
@@ -364,12 +374,12 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 }
             };
             // O += P V over the BN keys of one tile (K = 16 per instruction).
-            auto issue_pv = [&](int q, int b, int slot, bool acc) {
+            auto issue_pv = [&](int q, int b, int slot, bool acc, int kk0 = 0, int kk1 = C::BN / 16) {
                 const uint32_t d_tmem = tmem_base + C::TMEM_O + q * C::D;
                 const uint32_t p_tmem = tmem_base + C::TMEM_S + (q * C::NSB + b) * C::BN;
                 const uint64_t dv = dv0 + ((slot * C::KV_TILE_BYTES) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < C::BN / 16; ++kk) {
+                for (int kk = kk0; kk < kk1; ++kk) {
                     mma_bf16_ts(d_tmem, p_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_pv,
                                 (acc || kk > 0) ? 1u : 0u);
                 }
@@ -403,11 +413,20 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 ok = wait_slot(2 * j + 1) && (!has_next || wait_slot(2 * j + 2));
                 if (!ok) break;
                 for (int q = 0; q < C::NQ && ok; ++q) {
-                    ok = mbar_wait(bar(C::B_P_FULL + q), j & 1, abort_flag, p.status, kStatusTimeout,
+                    ok = mbar_wait(bar(C::B_P_FULL + 2 * q), j & 1, abort_flag, p.status, kStatusTimeout,
                                    THD_MMA_SPIN != 0);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_pv(q, 0, vslot, j > 0);
+                    if constexpr (C::P_SPLIT) {
+                        issue_pv(q, 0, vslot, j > 0, 0, C::BN / 32);
+                        ok = mbar_wait(bar(C::B_P_FULL + 2 * q + 1), j & 1, abort_flag, p.status,
+                                       kStatusTimeout, THD_MMA_SPIN != 0);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_pv(q, 0, vslot, true, C::BN / 32, C::BN / 16);
+                    } else {
+                        issue_pv(q, 0, vslot, j > 0);
+                    }
                     if (has_next) {
                         issue_qk(q, 0, kslot);
                         mma_commit(bar(C::B_S_FULL + q));
@@ -427,7 +446,7 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 const bool has_next = jn < n;
                 const int kslot = (2 * jn) % C::NSLOT;
                 for (int q = 0; q < C::NQ && ok; ++q) {
-                    ok = mbar_wait(bar(C::B_P_FULL + q), j & 1, abort_flag, p.status, kStatusTimeout,
+                    ok = mbar_wait(bar(C::B_P_FULL + 2 * q), j & 1, abort_flag, p.status, kStatusTimeout,
                                    THD_MMA_SPIN != 0);
                     if (!ok) break;
                     tc_fence_after();
@@ -566,15 +585,30 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
             const float2 sl2x2 = make_float2(sl2, sl2);
             const float2 negm2 = make_float2(neg_m, neg_m);
             float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-            exp_and_store_p<0, C::BN / 32, C::BN, C::EXP_EMU>(sv, sl2x2, negm2, s_tmem, acc0, acc1);
-            tmem_wait_st();
-            if (!o_ready) {
-                ok = warp_wait(bar(C::B_O_FULL + q), (j - 1) & 1, abort_flag, p.status);
-                if (!ok) break;
+            if constexpr (C::P_SPLIT) {
+                // (one S buffer: O already holds PV(j-1), o_ready is true)
+                exp_and_store_p<0, C::BN / 64, C::BN, C::EXP_EMU>(sv, sl2x2, negm2, s_tmem, acc0, acc1);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::B_P_FULL + 2 * q));
+                exp_and_store_p<C::BN / 2, C::BN / 64, C::BN, C::EXP_EMU>(sv, sl2x2, negm2, s_tmem,
+                                                                         acc0, acc1);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::B_P_FULL + 2 * q + 1));
+            } else {
+                exp_and_store_p<0, C::BN / 32, C::BN, C::EXP_EMU>(sv, sl2x2, negm2, s_tmem, acc0, acc1);
+                tmem_wait_st();
+                if (!o_ready) {
+                    ok = warp_wait(bar(C::B_O_FULL + q), (j - 1) & 1, abort_flag, p.status);
+                    if (!ok) break;
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::B_P_FULL + 2 * q));
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::B_P_FULL + q));
             l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
         }
 
