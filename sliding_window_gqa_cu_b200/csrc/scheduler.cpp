@@ -20,8 +20,7 @@ bool choose_kernel_shape(int D, int group, KernelShape* out) {
             *out = two ? KernelShape{64, 2, 1, 128, 8, false} : KernelShape{64, 1, 2, 128, 8, false};
             return true;
         case 128:
-            *out = two ? KernelShape{128, 2, kFwd128NSB, kFwd128BN, kFwd128Slots, false}
-                       : KernelShape{128, 1, 2, 128, 6, false};
+            *out = two ? KernelShape{128, 2, 1, 128, 5, false} : KernelShape{128, 1, 2, 128, 6, false};
             return true;
         case 256:
             *out = two ? KernelShape{256, 2, 2, 128, 4, true} : KernelShape{256, 1, 2, 64, 5, false};

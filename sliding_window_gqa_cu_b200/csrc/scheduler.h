@@ -13,19 +13,7 @@
 
 #include "../../include/thd_attn.h"
 
-// Head dim 128 with two heads per CTA: keys per key tile.  128: one S buffer
-// per head, PV(j) and QK(j+1) of a head issued as one run; 64: two S buffers
-// per head, so QK(j+1) runs while the softmax works on tile j (2 heads x
-// (2 x 64 + 128) = 512 TMEM columns).
-#ifndef THD_FWD128_BN
-#define THD_FWD128_BN 128
-#endif
-
 namespace thd {
-
-constexpr int kFwd128BN = THD_FWD128_BN;
-constexpr int kFwd128NSB = THD_FWD128_BN == 64 ? 2 : 1;
-constexpr int kFwd128Slots = THD_FWD128_BN == 64 ? 9 : 5;
 
 // Kernel shape chosen for a head dim and GQA group size.
 struct KernelShape {

@@ -77,30 +77,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // microseconds; two seconds means the pipeline is stuck.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-// Non-blocking test of a phase (the thread is never suspended).
-__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done) : "r"(bar), "r"(parity) : "memory");
-    return done != 0;
-}
-
 // Wait until the phase with the given parity has completed.  Returns false
 // (after recording `code` in *status and raising the CTA's abort flag) if
 // the limit runs out, or if another role of the CTA has already aborted.
-// With spin, the first polls never suspend the thread (for a thread whose
-// reaction time is on the critical path and whose polls cost little).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
-                                          volatile int* abort_flag, int* status, int code,
-                                          bool spin_first = false) {
-    if (spin_first) {
-#pragma unroll 1
-        for (int spin = 0; spin < 4096; ++spin)
-            if (mbar_test_wait(bar, parity)) return true;
-    }
+                                          volatile int* abort_flag, int* status, int code) {
     // Fast path: plain polling (try_wait itself suspends briefly in hardware).
 #pragma unroll 1
     for (int spin = 0; spin < 256; ++spin)
@@ -444,21 +425,6 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
     const int ex = __float_as_int(t.x) * (1 << 23) + __float_as_int(p.x);
     const int ey = __float_as_int(t.y) * (1 << 23) + __float_as_int(p.y);
     return make_float2(__int_as_float(ex), __int_as_float(ey));
-}
-
-// 2^x of two values on MUFU's half-precision path: x rounded to f16 (x <= 0
-// here; for |x| < 8 the rounding moves 2^x by at most 0.14 %, and larger |x|
-// give terms below 2^-8), two results from one ex2.approx.f16x2, widened to
-// fp32.
-__device__ __forceinline__ float2 exp2_f16x2(float2 x) {
-    uint32_t h, r;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(x.y), "f"(x.x));
-    asm("ex2.approx.f16x2 %0, %1;" : "=r"(r) : "r"(h));
-    float lo, hi;
-    asm("{\n\t.reg .f16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
-        "cvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
-        : "=f"(lo), "=f"(hi) : "r"(r));
-    return make_float2(lo, hi);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

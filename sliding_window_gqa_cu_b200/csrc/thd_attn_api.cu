@@ -28,7 +28,7 @@ using thd::KernelShape;
 
 using Cfg64x2 = thd::FwdConfig<64, 2, 1, 128, 8>;
 using Cfg64x1 = thd::FwdConfig<64, 1, 2, 128, 8>;
-using Cfg128x2 = thd::FwdConfig<128, 2, thd::kFwd128NSB, thd::kFwd128BN, thd::kFwd128Slots>;
+using Cfg128x2 = thd::FwdConfig<128, 2, 1, 128, 5>;
 using Cfg128x1 = thd::FwdConfig<128, 1, 2, 128, 6>;
 using Cfg256x1 = thd::FwdConfig<256, 1, 2, 64, 5>;
 using SplitCfg256 = thd::SplitConfig<256, 2, 4>;  // 2 heads per item over a CTA pair

@@ -43,24 +43,7 @@
 #define THD_DEBUG 0
 #endif
 
-// 1: the MMA-issuing thread polls its barriers without suspending before it
-// falls back to the suspending wait.
-#ifndef THD_MMA_SPIN
-#define THD_MMA_SPIN 0
-#endif
 
-// 1: the softmax exponentials of the one-CTA kernel use MUFU's f16x2 path
-// (two exponentials per instruction).
-#ifndef THD_EXP_F16
-#define THD_EXP_F16 0
-#endif
-
-// 1: with one S buffer per head, the softmax publishes P in two halves (keys
-// [0, BN/2) and [BN/2, BN)), so PV starts on the first half while the second
-// half's exponentials are still running.
-#ifndef THD_P_SPLIT
-#define THD_P_SPLIT 0
-#endif
 
 namespace thd {
 
@@ -120,8 +103,10 @@ struct FwdConfig {
     static constexpr int B_S_FULL = B_SLOT_EMPTY + NSLOT;  // [NQ][NSB]
     static constexpr int B_P_FULL = B_S_FULL + NQ * NSB;   // [NQ][2] P (half) written, O rescaled
     static constexpr int B_O_FULL = B_P_FULL + 2 * NQ;     // PV done
-    // P published in two halves (one S buffer per head only).
-    static constexpr bool P_SPLIT = THD_P_SPLIT != 0 && NSB == 1;
+    // With one S buffer per head the softmax publishes P in two halves (keys
+    // [0, BN/2), then [BN/2, BN)), so PV starts on the first half while the
+    // second half's exponentials still run (identical arithmetic).
+    static constexpr bool P_SPLIT = NSB == 1;
     static constexpr int B_DRAIN = B_O_FULL + NQ;
     static constexpr int NUM_BARS = B_DRAIN + 1;
 
@@ -243,10 +228,6 @@ __device__ __forceinline__ void exp_and_store_p(const float (&sv)[BN], float2 sl
             float p0, p1;
             if ((u & 3) >= 4 - EMU) {
                 const float2 e = exp2_poly2(x);
-                p0 = e.x;
-                p1 = e.y;
-            } else if (THD_EXP_F16) {
-                const float2 e = exp2_f16x2(x);
                 p0 = e.x;
                 p1 = e.y;
             } else {
@@ -387,7 +368,7 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
 
             auto wait_slot = [&](int pos) -> bool {
                 return mbar_wait(bar(C::B_SLOT_FULL + pos % C::NSLOT), (pos / C::NSLOT) & 1,
-                                 abort_flag, p.status, kStatusTimeout, THD_MMA_SPIN != 0);
+                                 abort_flag, p.status, kStatusTimeout);
             };
             bool ok = mbar_wait(bar(C::B_Q_FULL), 0, abort_flag, p.status, kStatusTimeout);
             for (int jj = 0; ok && jj < C::NSB && jj < n; ++jj) {
@@ -413,14 +394,13 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 ok = wait_slot(2 * j + 1) && (!has_next || wait_slot(2 * j + 2));
                 if (!ok) break;
                 for (int q = 0; q < C::NQ && ok; ++q) {
-                    ok = mbar_wait(bar(C::B_P_FULL + 2 * q), j & 1, abort_flag, p.status, kStatusTimeout,
-                                   THD_MMA_SPIN != 0);
+                    ok = mbar_wait(bar(C::B_P_FULL + 2 * q), j & 1, abort_flag, p.status, kStatusTimeout);
                     if (!ok) break;
                     tc_fence_after();
                     if constexpr (C::P_SPLIT) {
                         issue_pv(q, 0, vslot, j > 0, 0, C::BN / 32);
                         ok = mbar_wait(bar(C::B_P_FULL + 2 * q + 1), j & 1, abort_flag, p.status,
-                                       kStatusTimeout, THD_MMA_SPIN != 0);
+                                       kStatusTimeout);
                         if (!ok) break;
                         tc_fence_after();
                         issue_pv(q, 0, vslot, true, C::BN / 32, C::BN / 16);
@@ -446,8 +426,7 @@ thd_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 const bool has_next = jn < n;
                 const int kslot = (2 * jn) % C::NSLOT;
                 for (int q = 0; q < C::NQ && ok; ++q) {
-                    ok = mbar_wait(bar(C::B_P_FULL + 2 * q), j & 1, abort_flag, p.status, kStatusTimeout,
-                                   THD_MMA_SPIN != 0);
+                    ok = mbar_wait(bar(C::B_P_FULL + 2 * q), j & 1, abort_flag, p.status, kStatusTimeout);
                     if (!ok) break;
                     tc_fence_after();
                     issue_pv(q, j % C::NSB, vslot, j > 0);

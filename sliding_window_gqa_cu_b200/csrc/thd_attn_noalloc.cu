@@ -82,7 +82,7 @@ thd_work_item* const g_host_items = g_upload.items;
 
 using NCfg64x2 = thd::FwdConfig<64, 2, 1, 128, 8>;
 using NCfg64x1 = thd::FwdConfig<64, 1, 2, 128, 8>;
-using NCfg128x2 = thd::FwdConfig<128, 2, thd::kFwd128NSB, thd::kFwd128BN, thd::kFwd128Slots>;
+using NCfg128x2 = thd::FwdConfig<128, 2, 1, 128, 5>;
 using NCfg128x1 = thd::FwdConfig<128, 1, 2, 128, 6>;
 using NCfg256x1 = thd::FwdConfig<256, 1, 2, 64, 5>;
 using NSplitCfg256 = thd::SplitConfig<256, 2, 4>;  // 2 heads per item over a CTA pair
