@@ -16,7 +16,8 @@
 // sums meet once at the end.
 //
 // Warps: 0-15 softmax (head q = w / 8, key half h = (w / 4) % 2, TMEM lane
-// quadrant w % 4), 16 TMA producer, 17 MMA issuer, 18-19 idle.  TMEM: S[q] at
+// quadrant w % 4), 16 TMA producer, 17 MMA issuer (576 threads, 112 registers
+// each).  TMEM: S[q] at
 // 128 q, O[q] at 256 + 128 q (512 columns).  MMA order per key tile j, as in
 // the two-head one-CTA kernel: PV0(j) QK0(j+1) | PV1(j) QK1(j+1).
 #pragma once
@@ -59,14 +60,8 @@ struct KsplitConfig {
     static constexpr int NUM_SOFTMAX_WARPS = 8 * NQ;
     static constexpr int PRODUCER_WARP = NUM_SOFTMAX_WARPS;
     static constexpr int MMA_WARP = NUM_SOFTMAX_WARPS + 1;
-    static constexpr int NUM_THREADS = (NUM_SOFTMAX_WARPS + 4) * 32;  // 640
-    // 640 threads start with 96 registers each; the control warpgroup hands
-    // part of its share to the softmax warpgroups: 512*104 + 128*64 = 640*96.
-    static constexpr int LAUNCH_REGS = 96;
-    static constexpr int SOFTMAX_REGS = 104;
-    static constexpr int CONTROL_REGS = 64;
-    static_assert(NUM_SOFTMAX_WARPS * 32 * SOFTMAX_REGS + 128 * CONTROL_REGS <=
-                  NUM_THREADS * LAUNCH_REGS, "register split exceeds the launch");
+    // 18 warps, no register split: 576 threads x 112 registers.
+    static constexpr int NUM_THREADS = (NUM_SOFTMAX_WARPS + 2) * 32;
 
     static constexpr int B_Q_FULL = 0;
     static constexpr int B_SLOT_FULL = 1;
@@ -94,7 +89,7 @@ struct KsplitConfig {
 };
 
 template <class C>
-__global__ void __launch_bounds__(C::NUM_THREADS, 1)
+__global__ void __maxnreg__(112)
 thd_attn_fwd_ksplit_kernel(const __grid_constant__ CUtensorMap tmap_q,
                            const __grid_constant__ CUtensorMap tmap_k,
                            const __grid_constant__ CUtensorMap tmap_v,
@@ -140,7 +135,6 @@ thd_attn_fwd_ksplit_kernel(const __grid_constant__ CUtensorMap tmap_q,
     const bool skip = *abort_flag != 0;
 
     if (warp >= C::NUM_SOFTMAX_WARPS) {
-        regs_decrease<C::CONTROL_REGS>();
         if (warp == C::PRODUCER_WARP) {
             // ---------------------------------------------------- TMA producer
             if (lane == 0 && !skip) {
@@ -254,7 +248,6 @@ thd_attn_fwd_ksplit_kernel(const __grid_constant__ CUtensorMap tmap_q,
         }
     } else {
         // ------------------------------------------------------------ softmax
-        regs_increase<C::SOFTMAX_REGS>();
         const int q = warp >> 3;        // head of the CTA
         const int h = (warp >> 2) & 1;  // key half of every tile
         const int wq = warp & 3;
@@ -426,13 +419,10 @@ thd_attn_fwd_ksplit_kernel(const __grid_constant__ CUtensorMap tmap_q,
     }
 }
 
-// Host check before the first launch: the register split assumes the kernel
-// starts with LAUNCH_REGS registers per thread.
+// Host check before the first launch (the kernel has no register split).
 template <class C>
 inline bool ksplit_launch_registers_ok() {
-    cudaFuncAttributes a{};
-    if (cudaFuncGetAttributes(&a, thd_attn_fwd_ksplit_kernel<C>) != cudaSuccess) return false;
-    return a.numRegs >= C::LAUNCH_REGS;
+    return true;
 }
 
 }  // namespace thd
