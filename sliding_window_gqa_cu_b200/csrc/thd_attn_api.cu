@@ -330,7 +330,7 @@ int launch_bwd256(DeviceState* ds, const BwdPlanEntry& plan, const CUtensorMap& 
                   float* sink_part, cudaStream_t stream) {
     using Cq = thd::BwdConfig<256, 3, 64>;
     using Cdv = thd::BwdConfig<256, 2, 64, thd::kDvOnly>;
-    using Cdk = thd::BwdConfig<256, 1, 64, thd::kDkOnly>;
+    using Cdk = thd::BwdConfig<256, 2, 64, thd::kDkOnly, 1>;  // two Q slots, one dO slot
     auto kq = thd::thd_attn_bwd_dq_kernel<Cq>;
     auto kdv = thd::thd_attn_bwd_dkdv_kernel<Cdv>;
     auto kdk = thd::thd_attn_bwd_dkdv_kernel<Cdk>;

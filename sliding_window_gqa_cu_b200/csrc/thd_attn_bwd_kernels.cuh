@@ -158,10 +158,11 @@ __global__ void __launch_bounds__(256) thd_attn_bwd_dsink_kernel(const float* __
 // or one of them (head dim 256, two launches).
 enum BwdKvMode { kDkDv = 0, kDvOnly = 1, kDkOnly = 2 };
 
-template <int D_, int NSLOT_, int BN_ = 128, int MODE_ = kDkDv>
+template <int D_, int NSLOT_, int BN_ = 128, int MODE_ = kDkDv, int NDSLOT_ = NSLOT_>
 struct BwdConfig {
     static constexpr int D = D_;
-    static constexpr int NSLOT = NSLOT_;  // dq: K/V ring slots; dkdv: Q/dO pairs
+    static constexpr int NSLOT = NSLOT_;    // dq: K/V ring slots; dkdv: Q tile slots
+    static constexpr int NDSLOT = NDSLOT_;  // dkdv: dO tile slots
     static constexpr int BM = 128;        // TMEM lanes (queries for dq, keys for dkdv)
     static constexpr int BN = BN_;        // columns of S per tile (keys for dq, queries for dkdv)
     static constexpr int MODE = MODE_;    // dkdv kernel only
@@ -475,11 +476,17 @@ thd_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
 // ---------------------------------------------------------------- dk, dv ----
 template <class C>
 struct DkvLayout {
-    static constexpr int NPAIR = C::NSLOT;                    // Q/dO tile pairs in flight
-    static constexpr int B_KV_FULL = 0;                       // K and V landed
-    static constexpr int B_PAIR_FULL = 1;                     // [NPAIR] Q, dO, lse, delta
-    static constexpr int B_PAIR_EMPTY = B_PAIR_FULL + NPAIR;  // [NPAIR]
-    static constexpr int B_S_FULL = B_PAIR_EMPTY + NPAIR;     // S^T done
+    // Q tiles (with their lse / delta values) and dO tiles have rings of
+    // their own: step s uses Q slot s % NQS and dO slot s % NDS; a slot is
+    // released after the last product that reads it.
+    static constexpr int NQS = C::NSLOT;
+    static constexpr int NDS = C::NDSLOT;
+    static constexpr int B_KV_FULL = 0;                    // K and V landed
+    static constexpr int B_Q_FULL = 1;                     // [NQS] Q tile, lse, delta
+    static constexpr int B_Q_EMPTY = B_Q_FULL + NQS;       // [NQS]
+    static constexpr int B_DO_FULL = B_Q_EMPTY + NQS;      // [NDS] dO tile
+    static constexpr int B_DO_EMPTY = B_DO_FULL + NDS;     // [NDS]
+    static constexpr int B_S_FULL = B_DO_EMPTY + NDS;      // S^T done
     static constexpr int B_DP_FULL = B_S_FULL + 1;            // dP^T done
     static constexpr int B_P_READY = B_DP_FULL + 1;           // P^T in TMEM (8 warps)
     static constexpr int B_DS_READY = B_P_READY + 1;          // dS^T in TMEM (8 warps)
@@ -490,11 +497,11 @@ struct DkvLayout {
     static constexpr int SMEM_V = SMEM_K + C::TILE_BYTES;
     static_assert(C::MODE != kDkDv || C::TM_ACC1 + C::D <= 512, "dk and dv together exceed TMEM");
     static constexpr int V_BYTES = C::MODE == kDvOnly ? 0 : C::TILE_BYTES;  // dv alone needs no V
-    static constexpr int SMEM_PAIRS = SMEM_V + V_BYTES;  // [NPAIR][Q tile, dO tile] of BN rows
-    static constexpr int PAIR_BYTES = 2 * C::NTILE_BYTES;
-    static constexpr int SMEM_SIDE = SMEM_PAIRS + NPAIR * PAIR_BYTES;  // [NPAIR][lse2 BN, delta BN]
+    static constexpr int SMEM_Q = SMEM_V + V_BYTES;               // [NQS] Q tiles of BN rows
+    static constexpr int SMEM_DO = SMEM_Q + NQS * C::NTILE_BYTES;  // [NDS] dO tiles of BN rows
+    static constexpr int SMEM_SIDE = SMEM_DO + NDS * C::NTILE_BYTES;  // [NQS][lse2 BN, delta BN]
     static constexpr int SIDE_BYTES = 2 * C::BN * 4;
-    static constexpr int SMEM_BAR = SMEM_SIDE + NPAIR * SIDE_BYTES;
+    static constexpr int SMEM_BAR = SMEM_SIDE + NQS * SIDE_BYTES;
     static constexpr int SMEM_TMEM_SLOT = SMEM_BAR + NUM_BARS * 8;
     static constexpr int SMEM_ABORT = SMEM_TMEM_SLOT + 4;
     static constexpr int SMEM_ALLOC = SMEM_ABORT + 4 + 1024;
@@ -528,9 +535,13 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
 
     if (threadIdx.x == 0) {
         mbar_init(bar(L::B_KV_FULL), 1);
-        for (int s = 0; s < L::NPAIR; ++s) {
-            mbar_init(bar(L::B_PAIR_FULL + s), 2);  // TMA bytes + the side values
-            mbar_init(bar(L::B_PAIR_EMPTY + s), 1);
+        for (int s = 0; s < L::NQS; ++s) {
+            mbar_init(bar(L::B_Q_FULL + s), 2);  // TMA bytes + the side values
+            mbar_init(bar(L::B_Q_EMPTY + s), 1);
+        }
+        for (int s = 0; s < L::NDS; ++s) {
+            mbar_init(bar(L::B_DO_FULL + s), 1);
+            mbar_init(bar(L::B_DO_EMPTY + s), 1);
         }
         mbar_init(bar(L::B_S_FULL), 1);
         mbar_init(bar(L::B_DP_FULL), 1);
@@ -555,7 +566,8 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
         // All 32 lanes stage the per-query lse / delta values; lane 0 issues
         // the copies.
         bool ok = !skip;
-        int issued = 0;  // steps whose copies were issued
+        int issued = 0;     // steps whose Q copies were issued
+        int issued_do = 0;  // steps whose dO copies were issued
         if (ok && lane == 0) {
             tma_prefetch_desc(&tmap_q);
             tma_prefetch_desc(&tmap_do);
@@ -571,22 +583,19 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
             }
         }
         for (int s = 0; ok && s < n_steps; ++s) {
-            const int pr = s % L::NPAIR;
-            ok = warp_wait(bar(L::B_PAIR_EMPTY + pr), ((s / L::NPAIR) & 1) ^ 1, abort_flag, prm.status);
-            if (!ok) break;
+            const int qs = s % L::NQS, ds = s % L::NDS;
             const int h = it.g * G + s / nsub;
             const int i0 = it.k0 + (s % nsub) * C::BN;
+            ok = warp_wait(bar(L::B_Q_EMPTY + qs), ((s / L::NQS) & 1) ^ 1, abort_flag, prm.status);
+            if (!ok) break;
             if (lane == 0) {
-                const uint32_t full = bar(L::B_PAIR_FULL + pr);
-                const uint32_t dst = sbase + L::SMEM_PAIRS + pr * L::PAIR_BYTES;
-                mbar_arrive_expect_tx(full, 2 * C::NTILE_BYTES);
-                for (int c = 0; c < C::KCH; ++c) {
+                const uint32_t full = bar(L::B_Q_FULL + qs);
+                const uint32_t dst = sbase + L::SMEM_Q + qs * C::NTILE_BYTES;
+                mbar_arrive_expect_tx(full, C::NTILE_BYTES);
+                for (int c = 0; c < C::KCH; ++c)
                     tma_load_3d(dst + c * C::NBOX_BYTES, &tmap_q, full, c * 64, h, i0);
-                    tma_load_3d(dst + C::NTILE_BYTES + c * C::NBOX_BYTES, &tmap_do, full, c * 64, h,
-                                i0);
-                }
             }
-            float* sd = side + pr * 2 * C::BN;
+            float* sd = side + qs * 2 * C::BN;
 #pragma unroll
             for (int u = 0; u < C::BN / 32; ++u) {
                 const int col = lane * (C::BN / 32) + u;
@@ -596,14 +605,27 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 sd[C::BN + col] = in ? prm.delta[i * prm.Hq + h] : 0.0f;
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(L::B_PAIR_FULL + pr));
+            if (lane == 0) mbar_arrive(bar(L::B_Q_FULL + qs));
             issued = s + 1;
+            ok = warp_wait(bar(L::B_DO_EMPTY + ds), ((s / L::NDS) & 1) ^ 1, abort_flag, prm.status);
+            if (!ok) break;
+            if (lane == 0) {
+                const uint32_t full = bar(L::B_DO_FULL + ds);
+                const uint32_t dst = sbase + L::SMEM_DO + ds * C::NTILE_BYTES;
+                mbar_arrive_expect_tx(full, C::NTILE_BYTES);
+                for (int c = 0; c < C::KCH; ++c)
+                    tma_load_3d(dst + c * C::NBOX_BYTES, &tmap_do, full, c * 64, h, i0);
+            }
+            issued_do = s + 1;
         }
         if (!ok && !skip && lane == 0) {
-            // Unwinding: let the copies already issued land before exit.
+            // Unwinding: let the copies already issued land before exit
+            // (only the last ones into each slot can still be in flight).
             drain_wait(bar(L::B_KV_FULL), 0);
-            for (int s = issued - L::NPAIR > 0 ? issued - L::NPAIR : 0; s < issued; ++s)
-                drain_wait(bar(L::B_PAIR_FULL + s % L::NPAIR), (s / L::NPAIR) & 1);
+            for (int s = issued - L::NQS > 0 ? issued - L::NQS : 0; s < issued; ++s)
+                drain_wait(bar(L::B_Q_FULL + s % L::NQS), (s / L::NQS) & 1);
+            for (int s = issued_do - L::NDS > 0 ? issued_do - L::NDS : 0; s < issued_do; ++s)
+                drain_wait(bar(L::B_DO_FULL + s % L::NDS), (s / L::NDS) & 1);
         }
         __syncwarp();
     } else if (warp == C::MMA_WARP) {
@@ -612,36 +634,42 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
             constexpr uint32_t idesc_acc = idesc_bf16_f32(128, C::D, true);
             const uint64_t dk0 = smem_desc_sw128(sbase + L::SMEM_K, 16, 1024);
             const uint64_t dv0 = smem_desc_sw128(sbase + L::SMEM_V, 16, 1024);
-            const uint64_t dpair0 = smem_desc_sw128(sbase + L::SMEM_PAIRS, 16, 1024);
-            const uint64_t dpairmn0 = smem_desc_sw128(sbase + L::SMEM_PAIRS, C::NBOX_BYTES, 1024);
+            const uint64_t dq0 = smem_desc_sw128(sbase + L::SMEM_Q, 16, 1024);
+            const uint64_t dqmn0 = smem_desc_sw128(sbase + L::SMEM_Q, C::NBOX_BYTES, 1024);
+            const uint64_t ddo0 = smem_desc_sw128(sbase + L::SMEM_DO, 16, 1024);
+            const uint64_t ddomn0 = smem_desc_sw128(sbase + L::SMEM_DO, C::NBOX_BYTES, 1024);
             auto wait = [&](int idx, uint32_t parity) -> bool {
                 return mbar_wait(bar(idx), parity, abort_flag, prm.status, kStatusTimeout);
             };
             bool ok = wait(L::B_KV_FULL, 0);
             for (int s = 0; ok && s < n_steps; ++s) {
-                const int pr = s % L::NPAIR;
-                ok = wait(L::B_PAIR_FULL + pr, (s / L::NPAIR) & 1);
+                const int qs = s % L::NQS, ds = s % L::NDS;
+                ok = wait(L::B_Q_FULL + qs, (s / L::NQS) & 1);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t qoff = (pr * L::PAIR_BYTES) >> 4;
-                const uint32_t dooff = (pr * L::PAIR_BYTES + C::NTILE_BYTES) >> 4;
+                const uint32_t qoff = (qs * C::NTILE_BYTES) >> 4;
+                const uint32_t dooff = (ds * C::NTILE_BYTES) >> 4;
 #pragma unroll
                 for (int kk = 0; kk < C::D / 16; ++kk) {  // S^T = K Q^T
                     const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
                     const uint32_t on = ((kk >> 2) * C::NBOX_BYTES + (kk & 3) * 32) >> 4;
-                    mma_bf16_ss(tmem_base + C::TM_S, dk0 + o, dpair0 + qoff + on, idesc_s,
+                    mma_bf16_ss(tmem_base + C::TM_S, dk0 + o, dq0 + qoff + on, idesc_s,
                                 kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar(L::B_S_FULL));  // the exponentials start under dP^T
+                ok = wait(L::B_DO_FULL + ds, (s / L::NDS) & 1);
+                if (!ok) break;
+                tc_fence_after();
                 if constexpr (kDk) {
 #pragma unroll
                     for (int kk = 0; kk < C::D / 16; ++kk) {  // dP^T = V dO^T
                         const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
                         const uint32_t on = ((kk >> 2) * C::NBOX_BYTES + (kk & 3) * 32) >> 4;
-                        mma_bf16_ss(tmem_base + C::TM_DP, dv0 + o, dpair0 + dooff + on, idesc_s,
+                        mma_bf16_ss(tmem_base + C::TM_DP, dv0 + o, ddo0 + dooff + on, idesc_s,
                                     kk > 0 ? 1u : 0u);
                     }
                     mma_commit(bar(L::B_DP_FULL));
+                    if constexpr (!kDv) mma_commit(bar(L::B_DO_EMPTY + ds));  // dO(s) read by dP^T only
                 }
                 if constexpr (kDv) {
                     ok = wait(L::B_P_READY, s & 1);
@@ -650,8 +678,13 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
 #pragma unroll
                     for (int kk = 0; kk < C::BN / 16; ++kk)  // dv += P^T dO (16 query rows a step)
                         mma_bf16_ts(tmem_base + C::TM_ACC0, tmem_base + C::TM_S + pcol<C::BN>(kk),
-                                    dpairmn0 + dooff + ((kk * 16 * 128) >> 4), idesc_acc,
+                                    ddomn0 + dooff + ((kk * 16 * 128) >> 4), idesc_acc,
                                     (s > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(bar(L::B_DO_EMPTY + ds));  // dO(s) done
+                    // Q(s)'s slot also holds the lse / delta values the
+                    // elementwise warps read before P_READY: release it here
+                    // when no dk product follows.
+                    if constexpr (!kDk) mma_commit(bar(L::B_Q_EMPTY + qs));
                 }
                 if constexpr (kDk) {
                     ok = wait(L::B_DS_READY, s & 1);  // dS^T is computed under dv
@@ -660,10 +693,10 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
 #pragma unroll
                     for (int kk = 0; kk < C::BN / 16; ++kk)  // dk += dS^T Q
                         mma_bf16_ts(tmem_base + C::TM_ACC1, tmem_base + C::TM_DP + pcol<C::BN>(kk),
-                                    dpairmn0 + qoff + ((kk * 16 * 128) >> 4), idesc_acc,
+                                    dqmn0 + qoff + ((kk * 16 * 128) >> 4), idesc_acc,
                                     (s > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(bar(L::B_Q_EMPTY + qs));  // Q(s) done
                 }
-                mma_commit(bar(L::B_PAIR_EMPTY + pr));
             }
             if (ok) mma_commit(bar(L::B_ACC_FULL));
             mma_commit(bar(L::B_DRAIN));
@@ -689,15 +722,15 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
         bool ok = !skip;
         constexpr int HALF = C::HALF;
         for (int s = 0; ok && s < n_steps; ++s) {
-            const int pr = s % L::NPAIR;
+            const int qs = s % L::NQS;
             const int ih = it.k0 + (s % nsub) * C::BN + HALF * h;  // first query of this half
-            // The side values of this step were stored before PAIR_FULL.
-            ok = warp_wait(bar(L::B_PAIR_FULL + pr), (s / L::NPAIR) & 1, abort_flag, prm.status) &&
+            // The side values of this step were stored before Q_FULL.
+            ok = warp_wait(bar(L::B_Q_FULL + qs), (s / L::NQS) & 1, abort_flag, prm.status) &&
                  warp_wait(bar(L::B_S_FULL), s & 1, abort_flag, prm.status);
             if (!ok) break;
             tc_fence_after();
-            const float* lse2 = side + pr * 2 * C::BN + HALF * h;
-            const float* dlt = side + pr * 2 * C::BN + C::BN + HALF * h;
+            const float* lse2 = side + qs * 2 * C::BN + HALF * h;
+            const float* dlt = side + qs * 2 * C::BN + C::BN + HALF * h;
             // Every (key, query) of this half visible: its queries after every
             // key, inside the document and inside every key's window.
             const bool full = ih >= k_last && ih + HALF - 1 < e_doc && it.k0 + 127 < e_doc &&
