@@ -18,7 +18,7 @@ SOURCES = [os.path.join(CSRC, "thd_attn_api.cu"), os.path.join(CSRC, "thd_attn_n
            os.path.join(CSRC, "thd_prologue.cu"), os.path.join(CSRC, "thd_sparse_mla.cu"),
            os.path.join(CSRC, "thd_host_pipeline.cu"), os.path.join(CSRC, "scheduler.cpp")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("thd_attn_kernel.cuh", "thd_attn_split_kernel.cuh",
-                                                  "thd_attn_ksplit_kernel.cuh", "thd_attn_bwd_kernels.cuh",
+                                                  "thd_attn_bwd_kernels.cuh",
                                                   "sm100_ptx.cuh", "scheduler.h", "tma_map.h")] \
     + [os.path.join(ROOT, "include", "thd_attn.h")]
 

@@ -18,7 +18,6 @@
 #include "tma_map.h"
 #include "thd_attn_kernel.cuh"
 #include "thd_attn_split_kernel.cuh"
-#include "thd_attn_ksplit_kernel.cuh"
 #include "thd_attn_bwd_kernels.cuh"
 
 namespace {
@@ -30,7 +29,6 @@ using thd::KernelShape;
 using Cfg64x2 = thd::FwdConfig<64, 2, 1, 128, 8>;
 using Cfg64x1 = thd::FwdConfig<64, 1, 2, 128, 8>;
 using Cfg128x2 = thd::FwdConfig<128, 2, 1, 128, 5>;
-using KsplitCfg128 = thd::KsplitConfig<4>;
 using Cfg128x1 = thd::FwdConfig<128, 1, 2, 128, 6>;
 using Cfg256x1 = thd::FwdConfig<256, 1, 2, 64, 5>;
 using SplitCfg256 = thd::SplitConfig<256, 2, 4>;  // 2 heads per item over a CTA pair
@@ -148,24 +146,6 @@ int get_plan(DeviceState* ds, const int32_t* cu, int n_docs, int64_t q_begin, in
     ds->plans.push_front(std::move(e));
     *out = &ds->plans.front();
     return THD_OK;
-}
-
-// Head dim 128, two heads per CTA, key-split softmax (THD_KSPLIT128).
-template <class C>
-int launch_ksplit(DeviceState* ds, int vidx, const PlanEntry& plan, const CUtensorMap& mq,
-                  const CUtensorMap& mk, const CUtensorMap& mv, const thd::FwdParams& prm,
-                  cudaStream_t stream) {
-    auto kern = thd::thd_attn_fwd_ksplit_kernel<C>;
-    if (!ds->attr_set[vidx]) {
-        if (!thd::ksplit_launch_registers_ok<C>()) return THD_ERR_UNSUPPORTED;
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM_ALLOC) != cudaSuccess)
-            return THD_ERR_CUDA;
-        ds->attr_set[vidx] = true;
-    }
-    kern<<<static_cast<unsigned>(plan.n_items), C::NUM_THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv,
-                                                                                      prm);
-    return cudaGetLastError() == cudaSuccess ? THD_OK : THD_ERR_CUDA;
 }
 
 template <class C>
@@ -508,9 +488,7 @@ int thd_attn_fwd_range(const void* q, const void* k, const void* v, const int32_
     switch (variant_index(ks)) {
         case 0: return launch<Cfg64x2>(ds, 0, *plan, mq, mk, mv, prm, stream);
         case 1: return launch<Cfg64x1>(ds, 1, *plan, mq, mk, mv, prm, stream);
-        case 2:
-            if (THD_KSPLIT128) return launch_ksplit<KsplitCfg128>(ds, 2, *plan, mq, mk, mv, prm, stream);
-            return launch<Cfg128x2>(ds, 2, *plan, mq, mk, mv, prm, stream);
+        case 2: return launch<Cfg128x2>(ds, 2, *plan, mq, mk, mv, prm, stream);
         case 3: return launch<Cfg128x1>(ds, 3, *plan, mq, mk, mv, prm, stream);
         case 4: return launch<Cfg256x1>(ds, 4, *plan, mq, mk, mv, prm, stream);
         default: return launch_pair<SplitCfg256>(ds, 5, *plan, mq, mk, mv, prm, stream);

@@ -41,7 +41,6 @@
 #include "tma_map.h"
 #include "thd_attn_kernel.cuh"
 #include "thd_attn_split_kernel.cuh"
-#include "thd_attn_ksplit_kernel.cuh"
 
 namespace {
 
@@ -84,7 +83,6 @@ thd_work_item* const g_host_items = g_upload.items;
 using NCfg64x2 = thd::FwdConfig<64, 2, 1, 128, 8>;
 using NCfg64x1 = thd::FwdConfig<64, 1, 2, 128, 8>;
 using NCfg128x2 = thd::FwdConfig<128, 2, 1, 128, 5>;
-using NKsplitCfg128 = thd::KsplitConfig<4>;
 using NCfg128x1 = thd::FwdConfig<128, 1, 2, 128, 6>;
 using NCfg256x1 = thd::FwdConfig<256, 1, 2, 64, 5>;
 using NSplitCfg256 = thd::SplitConfig<256, 2, 4>;  // 2 heads per item over a CTA pair
@@ -147,23 +145,6 @@ int setup_device(int dev, NoAllocDevice* st) {
     st->scratch = static_cast<unsigned char*>(ptr);
     st->ready = true;
     return THD_OK;
-}
-
-template <class C>
-int launch_ksplit(NoAllocDevice* st, int vidx, int64_t n_items, const CUtensorMap& mq,
-                  const CUtensorMap& mk, const CUtensorMap& mv, const thd::FwdParams& prm,
-                  cudaStream_t stream) {
-    auto kern = thd::thd_attn_fwd_ksplit_kernel<C>;
-    if (!st->attr_set[vidx]) {
-        if (!thd::ksplit_launch_registers_ok<C>()) return THD_ERR_UNSUPPORTED;
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM_ALLOC) != cudaSuccess)
-            return THD_ERR_CUDA;
-        st->attr_set[vidx] = true;
-    }
-    kern<<<static_cast<unsigned>(n_items), C::NUM_THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv,
-                                                                                  prm);
-    return cudaGetLastError() == cudaSuccess ? THD_OK : THD_ERR_CUDA;
 }
 
 template <class C>
@@ -292,8 +273,6 @@ extern "C" int thd_attn_fwd_noalloc(const void* q, const void* k, const void* v,
                           : launch<NCfg64x1>(st, 1, n_items, mq, mk, mv, prm, stream);
     }
     if (D == 128) {
-        if (THD_KSPLIT128 && ks.nq == 2)
-            return launch_ksplit<NKsplitCfg128>(st, 2, n_items, mq, mk, mv, prm, stream);
         return ks.nq == 2 ? launch<NCfg128x2>(st, 2, n_items, mq, mk, mv, prm, stream)
                           : launch<NCfg128x1>(st, 3, n_items, mq, mk, mv, prm, stream);
     }
