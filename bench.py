@@ -260,7 +260,9 @@ def run_reference(args, info):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": workload_config(cfg, cu, pairs),
+        # the same config object as the GPU arm's line for this workload
+        "config": workload_config(cfg, cu, pairs, {"parallelism": f"pack-parallel x{info.world}",
+                                                   "per_rank_tflop": 4 * pairs * cfg.D * cfg.Hq / 1e12}),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": f"{tot_rows} random (token, head) rows of the pack over "
                                    f"{args.steps} steps (~{per_step:.2f} s each)"},
