@@ -11,17 +11,21 @@
 //    the attention processes ceil(count / 64) slot chunks, not K / 64.
 //
 // 1. Attention (thd_sparse_mla_attn_kernel): one CTA per (token, group of
-//    128 heads, quarter of the 512 latent columns).  The 128 query rows of
-//    the token (128 x 576 bf16) sit in TMEM as the A operand; the selected
-//    kv rows are gathered 64 at a time by a producer warpgroup (16-byte
-//    cp.async copies into the 128-byte-swizzled layout the tensor core
-//    reads), so one shared-memory tile serves S = Q kv^T (K-major operand)
-//    and latent += P kv[:, quarter] (MN-major operand).  TMEM: Q 288
-//    columns + S / P 64 + the latent quarter 128 = 480 of 512, which is why
-//    the latent is split over four CTAs (each recomputes S: QK^T runs four
-//    times per token).  Online softmax as in the
-//    attention forward (exp2 domain, lazy rescale).  Writes the normalised
-//    latent (bf16) to a workspace [T, H, 512].
+//    128 heads, half of the 512 latent columns).  The token's 128 query rows
+//    (128 x 576 bf16) are the A operand of S = Q kv^T: columns 0-255 in TMEM,
+//    columns 256-575 in shared memory (128-byte swizzled).  The selected kv
+//    rows are gathered 64 at a time by eight gather warps, four per stage
+//    (16-byte cp.async copies, one kv row per warp instruction, into the
+//    128-byte-swizzled layout the tensor core reads; two stages, each
+//    published as soon as its copies land), so one shared-memory tile
+//    serves S (K-major
+//    operand) and latent += P kv[:, half] (MN-major operand, N = 256).
+//    TMEM: Q 128 columns + two S / P buffers of 64 + the latent half 256 =
+//    512, so S of the next chunk is computed while the softmax works on this
+//    one; the two CTAs of a token each compute S (QK^T runs twice per
+//    token).  Online softmax as in the attention forward (exp2 domain, lazy
+//    rescale).  Writes the normalised latent (bf16) to a workspace
+//    [T, H, 512].
 // 2. Projection (thd_sparse_mla_proj_kernel): per head a GEMM
 //    out[:, h, :] = latent[:, h, :] @ value_weight[h]^T, one CTA per
 //    (128-token tile, head), TMA-fed tcgen05 MMAs with K = 512.
@@ -44,8 +48,11 @@ using thd::kStatusTimeout;
 
 // --------------------------------------------------------- cp.async gather --
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+// One 16-byte global-to-shared copy.  No compiler memory barrier, so that
+// the loads that compute the next copies' addresses may move ahead of it
+// (the copied data is read only after cp_async_wait, which keeps one).
+__device__ __forceinline__ void cp_async16_nc(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src));
 }
 __device__ __forceinline__ void cp_async_commit() {
     asm volatile("cp.async.commit_group;" ::: "memory");
@@ -68,21 +75,36 @@ struct SmlaParams {
 };
 
 constexpr int kQDim = 576, kLat = 512;
-constexpr int kBN = 64;             // selected keys per chunk
-constexpr int kNST = 3;             // chunk stages
+constexpr int kHalf = kLat / 2;                  // latent columns per CTA
+constexpr int kBN = 64;                          // selected keys per chunk
+constexpr int kNST = 2;                          // chunk stages
 constexpr int kChunkBytes = kBN * 128;           // one 64-column chunk of a 64-row tile
 constexpr int kStageBytes = 9 * kChunkBytes;     // 64 rows x 576 columns
-constexpr int kTmQ = 0, kTmS = 288, kTmO = 352;  // TMEM columns
-constexpr int B_Q_READY = 0, B_FULL = 1, B_EMPTY = B_FULL + kNST, B_S_FULL = B_EMPTY + kNST,
-              B_P_FULL = B_S_FULL + 1, B_O_FULL = B_P_FULL + 1, B_DRAIN = B_O_FULL + 1,
+constexpr int kQT = 256;                         // query columns held in TMEM
+constexpr int kQSChunks = (kQDim - kQT) / 64;    // query chunks of 64 columns in shared memory
+constexpr int kQSChunkBytes = 128 * 128;         // 128 rows x 64 columns
+// TMEM columns: Q[:, :256] (bf16 pairs) 128, two S / P buffers of 64, the
+// latent half 256: all 512.
+constexpr int kTmQ = 0, kTmS = kQT / 2, kTmO = kTmS + 2 * kBN;
+constexpr int B_Q_READY = 0, B_QS_FULL = 1, B_FULL = 2, B_EMPTY = B_FULL + kNST, B_S_FULL = B_EMPTY + kNST,
+              B_P_FULL = B_S_FULL + 2, B_O_FULL = B_P_FULL + 2, B_DRAIN = B_O_FULL + 1,
               kNumBars = B_DRAIN + 1;
-constexpr int kSmemBias = kNST * kStageBytes;               // float [kNST][64]
+constexpr int kSmemQ = kNST * kStageBytes;                  // 1024-aligned
+constexpr int kSmemBias = kSmemQ + kQSChunks * kQSChunkBytes;  // float [kNST][64]
 constexpr int kSmemBar = kSmemBias + kNST * kBN * 4;
 constexpr int kSmemTmem = kSmemBar + kNumBars * 8;
 constexpr int kSmemAbort = kSmemTmem + 4;
 constexpr int kSmemAlloc = kSmemAbort + 4 + 1024;
 static_assert(kSmemAlloc <= 232448, "shared memory budget exceeded");
-static_assert(kTmO + 128 <= 512, "TMEM budget exceeded");
+static_assert(kSmemQ % 1024 == 0 && kQSChunkBytes % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+static_assert(kTmO + kHalf <= 512, "TMEM budget exceeded");
+// Warps: 0-3 softmax (thread = head), then kPW gather warps per stage, then
+// the MMA issuer.
+constexpr int kPW = 4;
+constexpr int kMmaWarp = 4 + kNST * kPW;
+constexpr int kThreads = (kMmaWarp + 1) * 32;
+static_assert(kBN % kPW == 0 && kBN / kPW <= 32, "gather rows per warp");
+static_assert((kQDim - kQT) % 64 == 0 && kQT % 64 == 0, "query split on 64-column chunks");
 
 __global__ void __launch_bounds__(256) thd_sparse_mla_compact_kernel(const int32_t* __restrict__ idx,
                                                                       int64_t T, int K, int64_t Tg,
@@ -106,18 +128,18 @@ __global__ void __launch_bounds__(256) thd_sparse_mla_compact_kernel(const int32
     if (lane == 0) count[t] = n;
 }
 
-__global__ void __launch_bounds__(288, 1) thd_sparse_mla_attn_kernel(const SmlaParams p) {
+__global__ void __launch_bounds__(kThreads, 1) thd_sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                                                                          const SmlaParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = thd::smem_addr(smem_raw);
     uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
     const uint32_t sbase = thd::smem_addr(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int quarter = blockIdx.x & 3;
+    const int half = blockIdx.x & 1;
     const int hgroups = p.H / 128;
-    const int hg = (blockIdx.x >> 2) % hgroups;
-    const int64_t t = (blockIdx.x >> 2) / hgroups;
+    const int hg = (blockIdx.x >> 1) % hgroups;
+    const int64_t t = (blockIdx.x >> 1) / hgroups;
     const int nch = (p.count[t] + kBN - 1) / kBN;  // chunks holding valid slots
-
     auto bar = [&](int i) -> uint32_t { return sbase + kSmemBar + 8u * i; };
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSmemAbort);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kSmemTmem);
@@ -125,18 +147,21 @@ __global__ void __launch_bounds__(288, 1) thd_sparse_mla_attn_kernel(const SmlaP
 
     if (threadIdx.x == 0) {
         thd::mbar_init(bar(B_Q_READY), 4);
+        thd::mbar_init(bar(B_QS_FULL), 1);
         for (int s = 0; s < kNST; ++s) {
-            thd::mbar_init(bar(B_FULL + s), 4);  // the four producer warps
+            thd::mbar_init(bar(B_FULL + s), kPW);  // the stage's gather warps
             thd::mbar_init(bar(B_EMPTY + s), 1);
         }
-        thd::mbar_init(bar(B_S_FULL), 1);
-        thd::mbar_init(bar(B_P_FULL), 4);
+        for (int b = 0; b < 2; ++b) {
+            thd::mbar_init(bar(B_S_FULL + b), 1);
+            thd::mbar_init(bar(B_P_FULL + b), 4);
+        }
         thd::mbar_init(bar(B_O_FULL), 1);
         thd::mbar_init(bar(B_DRAIN), 1);
         *abort_flag = *reinterpret_cast<volatile int*>(p.status) != 0 ? 1 : 0;
         thd::fence_barrier_init();
     }
-    if (warp == 8) {
+    if (warp == kMmaWarp) {
         thd::tmem_alloc(thd::smem_addr(tmem_slot), 512);
         thd::tmem_relinquish();
     }
@@ -146,74 +171,140 @@ __global__ void __launch_bounds__(288, 1) thd_sparse_mla_attn_kernel(const SmlaP
     const uint32_t tmem_base = *tmem_slot;
     const bool skip = *abort_flag != 0;
 
-    if (warp >= 4 && warp < 8) {
-        // ---------------------------------------------- gather producer (128)
-        const int pt = threadIdx.x - 128;
+    if (warp >= 4 && warp < kMmaWarp) {
+        // ------------------------------------------------- gather producers
+        // kPW warps per stage: stage 0 takes the even chunks, stage 1 the
+        // odd ones.  Chunk c goes to its stage once the products of chunk
+        // c - kNST have read it, and is published as soon as its own copies
+        // have landed, independently of the other stage.
+        const int pw = warp - 4;
+        const int s = pw / kPW;                 // this warp's stage
+        const int wi = pw % kPW;
         const int32_t* irow = p.idx + t * p.K;
         bool ok = !skip;
-        for (int c = 0; ok && c <= nch; ++c) {
-            if (c < nch) {
-                const int s = c % kNST;
-                ok = thd::warp_wait(bar(B_EMPTY + s), ((c / kNST) & 1) ^ 1, abort_flag, p.status);
-                if (!ok) break;
-                const uint32_t stage = sbase + s * kStageBytes;
-                for (int u = pt; u < kBN * 72; u += 128) {
-                    const int r = u / 72, uu = u % 72;
-                    const int gi = irow[c * kBN + r];
-                    const int64_t row = (gi >= 0 && gi < p.Tg) ? gi : 0;
-                    const uint32_t dst = stage + (uu >> 3) * kChunkBytes + r * 128 +
-                                         ((static_cast<uint32_t>(uu & 7) ^ static_cast<uint32_t>(r & 7)) << 4);
-                    cp_async16(dst, p.kv + row * kQDim + uu * 8);
-                }
-                if (pt < kBN) {
-                    const int gi = irow[c * kBN + pt];
-                    bias[s * kBN + pt] = (gi >= 0 && gi < p.Tg) ? 0.0f : -INFINITY;
-                }
-                cp_async_commit();
+        for (int c = s; ok && c < nch; c += kNST) {
+            ok = thd::warp_wait(bar(B_EMPTY + s), ((c / kNST) & 1) ^ 1, abort_flag, p.status);
+            if (!ok) break;
+            const uint32_t stage = sbase + s * kStageBytes;
+            // Warp wi of the stage copies rows [wi * kBN / kPW, +kBN / kPW)
+            // of the chunk, one row (72 units of 16 bytes) at a time, lane =
+            // unit: each copy instruction moves 512 contiguous bytes of a
+            // row.  An invalid slot reads row 0 and gets a -inf bias.
+            const int r0 = wi * (kBN / kPW);
+            if (lane < kBN / kPW) {
+                const int gi = irow[c * kBN + r0 + lane];
+                bias[s * kBN + r0 + lane] = (gi >= 0 && gi < p.Tg) ? 0.0f : -INFINITY;
             }
-            // Chunk c - 1 (this thread's copies) complete: publish it.
-            if (c >= 1) {
-                if (c < nch) cp_async_wait<1>(); else cp_async_wait<0>();
-                thd::fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) thd::mbar_arrive(bar(B_FULL + (c - 1) % kNST));
+#pragma unroll 4
+            for (int rr = 0; rr < kBN / kPW; ++rr) {
+                const int r = r0 + rr;
+                const int gi = irow[c * kBN + r];
+                const __nv_bfloat16* src = p.kv + static_cast<int64_t>((gi >= 0 && gi < p.Tg) ? gi : 0) * kQDim;
+                const uint32_t drow = stage + r * 128;
+                const uint32_t sw = static_cast<uint32_t>(r & 7);
+#pragma unroll
+                for (int k = 0; k < 3; ++k) {
+                    const int uu = lane + 32 * k;
+                    if (uu < 72)
+                        cp_async16_nc(drow + (uu >> 3) * kChunkBytes + ((static_cast<uint32_t>(uu & 7) ^ sw) << 4),
+                                      src + uu * 8);
+                }
             }
+            cp_async_commit();
+            cp_async_wait<0>();
+            thd::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) thd::mbar_arrive(bar(B_FULL + s));
         }
         if (!ok) cp_async_wait<0>();
         __syncwarp();
-    } else if (warp == 8) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------- MMA issuer
+        // Order S(0) S(1) PV(0) S(2) PV(1) ...: S(c + 1) runs while the
+        // softmax works on chunk c (two S / P buffers; S(c + 2) reuses the
+        // buffer of P(c) only after PV(c), which the in-order tensor pipe
+        // guarantees).
         if (lane == 0 && !skip) {
             constexpr uint32_t idesc_s = thd::idesc_bf16_f32(128, kBN, false);
-            constexpr uint32_t idesc_o = thd::idesc_bf16_f32(128, 128, true);
+            constexpr uint32_t idesc_o = thd::idesc_bf16_f32(128, kHalf, true);
             auto wait = [&](int i, uint32_t par) -> bool {
                 return thd::mbar_wait(bar(i), par, abort_flag, p.status, kStatusTimeout);
             };
-            bool ok = wait(B_Q_READY, 0);
-            for (int c = 0; ok && c < nch; ++c) {
-                const int s = c % kNST;
-                ok = wait(B_FULL + s, (c / kNST) & 1);
-                if (!ok) break;
-                thd::tc_fence_after();
-                const uint32_t stage = sbase + s * kStageBytes;
-                const uint64_t dk = thd::smem_desc_sw128(stage, 16, 1024);
+            const uint64_t dq0 = thd::smem_desc_sw128(sbase + kSmemQ, 16, 1024);
+            // S(c) = Q kv^T: the first kQT columns of Q from TMEM, the rest
+            // from shared memory (K steps of 16 columns = 32 bytes).
+            auto issue_s = [&](int c) {
+                const uint64_t dk = thd::smem_desc_sw128(sbase + (c % kNST) * kStageBytes, 16, 1024);
+                const uint32_t d = tmem_base + kTmS + kBN * (c & 1);
 #pragma unroll
-                for (int kk = 0; kk < kQDim / 16; ++kk)  // S = Q kv^T
-                    thd::mma_bf16_ts(tmem_base + kTmS, tmem_base + kTmQ + kk * 8,
+                for (int kk = 0; kk < kQT / 16; ++kk)
+                    thd::mma_bf16_ts(d, tmem_base + kTmQ + kk * 8,
                                      dk + (((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4), idesc_s,
                                      kk > 0 ? 1u : 0u);
-                thd::mma_commit(bar(B_S_FULL));
-                ok = wait(B_P_FULL, c & 1);
-                if (!ok) break;
-                thd::tc_fence_after();
-                const uint64_t dv =
-                    thd::smem_desc_sw128(stage + 2 * quarter * kChunkBytes, kChunkBytes, 1024);
 #pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk)  // latent quarter += P kv
-                    thd::mma_bf16_ts(tmem_base + kTmO, tmem_base + kTmS + kk * 8,
-                                     dv + ((kk * 16 * 128) >> 4), idesc_o, (c > 0 || kk > 0) ? 1u : 0u);
-                thd::mma_commit(bar(B_O_FULL));
-                thd::mma_commit(bar(B_EMPTY + s));
+                for (int kk = kQT / 16; kk < kQDim / 16; ++kk) {
+                    const int qk = kk - kQT / 16;
+                    thd::mma_bf16_ss(d, dq0 + (((qk >> 2) * kQSChunkBytes + (qk & 3) * 32) >> 4),
+                                     dk + (((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4), idesc_s, 1u);
+                }
+            };
+            // Issue whichever of the next S and the next PV can go first
+            // (non-blocking tests): S(k) needs chunk k gathered and PV(k - 2)
+            // issued (its S / P buffer), PV(k) needs P(k).  A PV that can go
+            // is issued first: it frees the chunk's stage for the gather of
+            // chunk k + 2.
+            // Q[:, kQT:] of the token's 128 heads: five 64-column boxes
+            // straight into the swizzled layout.
+            thd::tma_prefetch_desc(&tmap_q);
+            thd::mbar_arrive_expect_tx(bar(B_QS_FULL), kQSChunks * kQSChunkBytes);
+            for (int i = 0; i < kQSChunks; ++i)
+                thd::tma_load_3d(sbase + kSmemQ + i * kQSChunkBytes, &tmap_q, bar(B_QS_FULL), kQT + 64 * i,
+                                 hg * 128, static_cast<int>(t));
+            bool ok = wait(B_QS_FULL, 0);
+            if (!ok) thd::drain_wait(bar(B_QS_FULL), 0);
+            ok = ok && wait(B_Q_READY, 0);
+            int next_s = 0, next_pv = 0;
+            uint64_t t_wait = 0;
+            while (ok && next_pv < nch) {
+                if (next_pv < next_s &&
+                    thd::mbar_test(bar(B_P_FULL + (next_pv & 1)), (next_pv >> 1) & 1)) {
+                    const int c = next_pv;
+                    thd::tc_fence_after();
+                    // latent half += P kv[:, half]: N = 256, the MN-major
+                    // operand spans four 64-column chunks of the stage.
+                    const uint64_t dv = thd::smem_desc_sw128(
+                        sbase + (c % kNST) * kStageBytes + 4 * half * kChunkBytes, kChunkBytes, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk)
+                        thd::mma_bf16_ts(tmem_base + kTmO, tmem_base + kTmS + kBN * (c & 1) + kk * 8,
+                                         dv + ((kk * 16 * 128) >> 4), idesc_o, (c > 0 || kk > 0) ? 1u : 0u);
+                    thd::mma_commit(bar(B_O_FULL));
+                    thd::mma_commit(bar(B_EMPTY + c % kNST));
+                    ++next_pv;
+                    t_wait = 0;
+                    continue;
+                }
+                if (next_s < nch && next_s <= next_pv + 1 &&
+                    thd::mbar_test(bar(B_FULL + next_s % kNST), (next_s / kNST) & 1)) {
+                    thd::tc_fence_after();
+                    issue_s(next_s);
+                    thd::mma_commit(bar(B_S_FULL + (next_s & 1)));
+                    ++next_s;
+                    t_wait = 0;
+                    continue;
+                }
+                // Neither can go yet: bounded wait.
+                const uint64_t now = thd::global_timer_ns();
+                if (t_wait == 0) {
+                    t_wait = now;
+                } else if (now - t_wait > thd::kWaitLimitNs) {
+                    atomicCAS(p.status, 0, kStatusTimeout);
+                    *abort_flag = 1;
+                    ok = false;
+                } else if (*abort_flag || *reinterpret_cast<volatile int*>(p.status) != 0) {
+                    *abort_flag = 1;
+                    ok = false;
+                }
             }
             thd::mma_commit(bar(B_DRAIN));
             thd::drain_wait(bar(B_DRAIN), 0);
@@ -226,14 +317,24 @@ __global__ void __launch_bounds__(288, 1) thd_sparse_mla_attn_kernel(const SmlaP
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
         bool ok = !skip;
         if (ok) {
+            // Q row h, columns [0, kQT), into TMEM (bf16 pairs): rounds of 64
+            // columns, the next round's loads in flight while this one is
+            // stored.  (Columns kQT and up arrive by TMA.)
             const uint4* src = reinterpret_cast<const uint4*>(p.q + (t * p.H + h) * kQDim);
-#pragma unroll 1
-            for (int i = 0; i < 9; ++i) {  // 64 elements (32 columns) at a time
+            uint4 x[2][8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) x[0][u] = src[u];
+#pragma unroll
+            for (int i = 0; i < kQT / 64; ++i) {
+                if (i + 1 < kQT / 64) {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) x[(i + 1) & 1][u] = src[(i + 1) * 8 + u];
+                }
                 uint32_t w[32];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    const uint4 x = src[i * 8 + u];
-                    w[4 * u] = x.x; w[4 * u + 1] = x.y; w[4 * u + 2] = x.z; w[4 * u + 3] = x.w;
+                    w[4 * u] = x[i & 1][u].x; w[4 * u + 1] = x[i & 1][u].y;
+                    w[4 * u + 2] = x[i & 1][u].z; w[4 * u + 3] = x[i & 1][u].w;
                 }
                 thd::tmem_st32(lane_base + kTmQ + 32 * i, w);
             }
@@ -247,13 +348,14 @@ __global__ void __launch_bounds__(288, 1) thd_sparse_mla_attn_kernel(const SmlaP
         const float sl2 = p.scale_log2;
         for (int c = 0; ok && c < nch; ++c) {
             const int s = c % kNST;
+            const uint32_t ts = lane_base + kTmS + kBN * (c & 1);
             ok = thd::warp_wait(bar(B_FULL + s), (c / kNST) & 1, abort_flag, p.status) &&
-                 thd::warp_wait(bar(B_S_FULL), c & 1, abort_flag, p.status);
+                 thd::warp_wait(bar(B_S_FULL + (c & 1)), (c >> 1) & 1, abort_flag, p.status);
             if (!ok) break;
             thd::tc_fence_after();
             uint32_t sr[64];
-            thd::tmem_ld32(lane_base + kTmS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-            thd::tmem_ld32(lane_base + kTmS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+            thd::tmem_ld32(ts, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+            thd::tmem_ld32(ts + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
             thd::tmem_wait_ld();
             thd::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
             thd::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
@@ -294,17 +396,19 @@ __global__ void __launch_bounds__(288, 1) thd_sparse_mla_attn_kernel(const SmlaP
                 l += p0 + p1;
                 pk[u] = thd::pack_bf16x2(p0, p1);
             }
-            thd::tmem_st16(lane_base + kTmS, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
-            thd::tmem_st16(lane_base + kTmS + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
+            thd::tmem_st16(ts, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+            thd::tmem_st16(ts + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
             if (c > 0) {
                 // The previous chunk's product must be done before O is
-                // rescaled (and before this chunk's is issued).
+                // rescaled (and before this chunk's is issued); waiting every
+                // chunk also keeps the P barriers within one phase of the
+                // MMA issuer.
                 ok = thd::warp_wait(bar(B_O_FULL), (c - 1) & 1, abort_flag, p.status);
                 if (!ok) break;
                 thd::tc_fence_after();
                 if (__any_sync(0xffffffffu, rescale_o)) {
 #pragma unroll 1
-                    for (int cc = 0; cc < 4; ++cc) {
+                    for (int cc = 0; cc < kHalf / 32; ++cc) {
                         uint32_t r[32];
                         thd::tmem_ld32(lane_base + kTmO + 32 * cc, r);
                         thd::tmem_wait_ld();
@@ -318,15 +422,15 @@ __global__ void __launch_bounds__(288, 1) thd_sparse_mla_attn_kernel(const SmlaP
             thd::tmem_wait_st();
             thd::tc_fence_before();
             __syncwarp();
-            if (lane == 0) thd::mbar_arrive(bar(B_P_FULL));
+            if (lane == 0) thd::mbar_arrive(bar(B_P_FULL + (c & 1)));
         }
         if (ok && nch > 0) ok = thd::warp_wait(bar(B_O_FULL), (nch - 1) & 1, abort_flag, p.status);
         if (ok) {
             thd::tc_fence_after();
             const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
-            __nv_bfloat16* dst = p.latent + (t * p.H + h) * kLat + 128 * quarter;
+            __nv_bfloat16* dst = p.latent + (t * p.H + h) * kLat + kHalf * half;
 #pragma unroll 1
-            for (int cc = 0; cc < 4; ++cc) {
+            for (int cc = 0; cc < kHalf / 32; ++cc) {
                 uint32_t r[32];
                 if (nch > 0) {
                     thd::tmem_ld32(lane_base + kTmO + 32 * cc, r);
@@ -349,7 +453,7 @@ __global__ void __launch_bounds__(288, 1) thd_sparse_mla_attn_kernel(const SmlaP
     }
     thd::tc_fence_before();
     __syncthreads();
-    if (warp == 8) {
+    if (warp == kMmaWarp) {
         thd::tc_fence_after();
         thd::tmem_dealloc(tmem_base, 512);
     }
@@ -487,6 +591,21 @@ constexpr int proj_smem() {
     return kPNST * (kPA + VD * 128) + 8 * (2 * kPNST + 2) + 8 + 1024;
 }
 
+// 3-D map over q [T, H, 576]: dims (576, H, T), box (64, 128, 1): one token's
+// 128 heads, 64 columns.
+bool make_q_map(CUtensorMap* map, const void* base, int64_t T, int H) {
+    auto fn = thd::encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(kQDim), static_cast<cuuint64_t>(H),
+                          static_cast<cuuint64_t>(T)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(kQDim) * 2, static_cast<cuuint64_t>(H) * kQDim * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 3-D map over value_weight [H, VD, 512]: dims (512, VD, H), box (64, VD, 1).
 bool make_w_map(CUtensorMap* map, const void* base, int H, int vd) {
     auto fn = thd::encode_fn();
@@ -541,7 +660,7 @@ extern "C" int thd_sparse_mla_fwd(const void* q, const void* kv, const int32_t* 
     if (value_dim != 64 && value_dim != 128 && value_dim != 256) return THD_ERR_UNSUPPORTED;
     if (!(std::isfinite(scale) && scale >= 0.0f)) return THD_ERR_INVALID_ARG;
     if (T == 0) return THD_OK;
-    if (T * (H / 128) * 4 > 0x7fffffffLL || Tg > 0x7fffffffLL) return THD_ERR_INVALID_ARG;
+    if (T * (H / 128) * 2 > 0x7fffffffLL || Tg > 0x7fffffffLL) return THD_ERR_INVALID_ARG;
     if (!q || !kv || (!indices && K > 0) || !value_weight || !out || !workspace)
         return THD_ERR_INVALID_ARG;
     if (!thd::aligned16(q) || !thd::aligned16(kv) || !thd::aligned16(value_weight) ||
@@ -582,7 +701,10 @@ extern "C" int thd_sparse_mla_fwd(const void* q, const void* kv, const int32_t* 
     p.H = H;
     p.K = Keff;
     p.scale_log2 = scale * 1.4426950408889634f;
-    thd_sparse_mla_attn_kernel<<<static_cast<unsigned>(T * (H / 128) * 4), 288, kSmemAlloc, stream>>>(p);
+    CUtensorMap mq;
+    if (!make_q_map(&mq, q, T, H)) return THD_ERR_CUDA;
+    thd_sparse_mla_attn_kernel<<<static_cast<unsigned>(T * (H / 128) * 2), kThreads, kSmemAlloc, stream>>>(
+        mq, p);
     if (cudaGetLastError() != cudaSuccess) return THD_ERR_CUDA;
 
     CUtensorMap ml, mw;
