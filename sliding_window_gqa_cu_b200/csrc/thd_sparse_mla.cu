@@ -17,9 +17,11 @@
 //    rows are gathered 64 at a time by eight gather warps, four per stage
 //    (16-byte cp.async copies, one kv row per warp instruction, into the
 //    128-byte-swizzled layout the tensor core reads; two stages, each
-//    published as soon as its copies land), so one shared-memory tile
-//    serves S (K-major
-//    operand) and latent += P kv[:, half] (MN-major operand, N = 256).
+//    refilled in two parts -- the columns PV does not read once S of the
+//    stage's previous chunk is done, this CTA's latent half once its PV is
+//    -- and published as soon as its copies land), so one shared-memory
+//    tile serves S (K-major operand) and latent += P kv[:, half] (MN-major
+//    operand, N = 256).
 //    TMEM: Q 128 columns + two S / P buffers of 64 + the latent half 256 =
 //    512, so S of the next chunk is computed while the softmax works on this
 //    one; the two CTAs of a token each compute S (QK^T runs twice per
@@ -86,7 +88,10 @@ constexpr int kQSChunkBytes = 128 * 128;         // 128 rows x 64 columns
 // TMEM columns: Q[:, :256] (bf16 pairs) 128, two S / P buffers of 64, the
 // latent half 256: all 512.
 constexpr int kTmQ = 0, kTmS = kQT / 2, kTmO = kTmS + 2 * kBN;
-constexpr int B_Q_READY = 0, B_QS_FULL = 1, B_FULL = 2, B_EMPTY = B_FULL + kNST, B_S_FULL = B_EMPTY + kNST,
+// Per stage: FULL (gathered), SFREE (S of its chunk done: the columns that
+// PV does not read may be refilled), EMPTY (PV done: all of it).
+constexpr int B_Q_READY = 0, B_QS_FULL = 1, B_FULL = 2, B_SFREE = B_FULL + kNST, B_EMPTY = B_SFREE + kNST,
+              B_S_FULL = B_EMPTY + kNST,
               B_P_FULL = B_S_FULL + 2, B_O_FULL = B_P_FULL + 2, B_DRAIN = B_O_FULL + 1,
               kNumBars = B_DRAIN + 1;
 constexpr int kSmemQ = kNST * kStageBytes;                  // 1024-aligned
@@ -150,6 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1) thd_sparse_mla_attn_kernel(const 
         thd::mbar_init(bar(B_QS_FULL), 1);
         for (int s = 0; s < kNST; ++s) {
             thd::mbar_init(bar(B_FULL + s), kPW);  // the stage's gather warps
+            thd::mbar_init(bar(B_SFREE + s), 1);
             thd::mbar_init(bar(B_EMPTY + s), 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -174,49 +180,62 @@ __global__ void __launch_bounds__(kThreads, 1) thd_sparse_mla_attn_kernel(const 
     if (warp >= 4 && warp < kMmaWarp) {
         // ------------------------------------------------- gather producers
         // kPW warps per stage: stage 0 takes the even chunks, stage 1 the
-        // odd ones.  Chunk c goes to its stage once the products of chunk
-        // c - kNST have read it, and is published as soon as its own copies
-        // have landed, independently of the other stage.
+        // odd ones.  Chunk c refills its stage in two parts: the columns that
+        // PV does not read (the other latent half and the rotary part) once
+        // S of chunk c - kNST is done, then this CTA's latent half once PV of
+        // chunk c - kNST is done; it is published as soon as its copies have
+        // landed, independently of the other stage.  Warp wi copies rows
+        // [wi * kBN / kPW, +kBN / kPW) of the chunk, lane = 16-byte unit of a
+        // row (units [32 k, 32 k + 32) of a row in copy k; this CTA's latent
+        // half is exactly copy k = half), so each copy instruction moves 512
+        // contiguous bytes of one kv row.  An invalid slot reads row 0 and
+        // gets a -inf bias.
+        constexpr int kRows = kBN / kPW;
         const int pw = warp - 4;
         const int s = pw / kPW;                 // this warp's stage
-        const int wi = pw % kPW;
+        const int r0 = (pw % kPW) * kRows;
         const int32_t* irow = p.idx + t * p.K;
         bool ok = !skip;
         for (int c = s; ok && c < nch; c += kNST) {
-            ok = thd::warp_wait(bar(B_EMPTY + s), ((c / kNST) & 1) ^ 1, abort_flag, p.status);
+            const uint32_t par = ((c / kNST) & 1) ^ 1;
+            ok = thd::warp_wait(bar(B_SFREE + s), par, abort_flag, p.status);
             if (!ok) break;
             const uint32_t stage = sbase + s * kStageBytes;
-            // Warp wi of the stage copies rows [wi * kBN / kPW, +kBN / kPW)
-            // of the chunk, one row (72 units of 16 bytes) at a time, lane =
-            // unit: each copy instruction moves 512 contiguous bytes of a
-            // row.  An invalid slot reads row 0 and gets a -inf bias.
-            const int r0 = wi * (kBN / kPW);
-            if (lane < kBN / kPW) {
+            const __nv_bfloat16* src[kRows];
+#pragma unroll
+            for (int rr = 0; rr < kRows; ++rr) {
+                const int gi = irow[c * kBN + r0 + rr];
+                src[rr] = p.kv + static_cast<int64_t>((gi >= 0 && gi < p.Tg) ? gi : 0) * kQDim;
+            }
+            auto copy = [&](int rr, int k) {
+                const int r = r0 + rr;
+                const int uu = lane + 32 * k;
+                if (uu < 72)
+                    cp_async16_nc(stage + r * 128 + (uu >> 3) * kChunkBytes +
+                                      ((static_cast<uint32_t>(uu & 7) ^ static_cast<uint32_t>(r & 7)) << 4),
+                                  src[rr] + uu * 8);
+            };
+#pragma unroll
+            for (int rr = 0; rr < kRows; ++rr) {
+#pragma unroll
+                for (int k = 0; k < 3; ++k)
+                    if (k != half) copy(rr, k);
+            }
+            ok = thd::warp_wait(bar(B_EMPTY + s), par, abort_flag, p.status);
+            if (!ok) break;
+            if (lane < kRows) {
                 const int gi = irow[c * kBN + r0 + lane];
                 bias[s * kBN + r0 + lane] = (gi >= 0 && gi < p.Tg) ? 0.0f : -INFINITY;
             }
-#pragma unroll 4
-            for (int rr = 0; rr < kBN / kPW; ++rr) {
-                const int r = r0 + rr;
-                const int gi = irow[c * kBN + r];
-                const __nv_bfloat16* src = p.kv + static_cast<int64_t>((gi >= 0 && gi < p.Tg) ? gi : 0) * kQDim;
-                const uint32_t drow = stage + r * 128;
-                const uint32_t sw = static_cast<uint32_t>(r & 7);
 #pragma unroll
-                for (int k = 0; k < 3; ++k) {
-                    const int uu = lane + 32 * k;
-                    if (uu < 72)
-                        cp_async16_nc(drow + (uu >> 3) * kChunkBytes + ((static_cast<uint32_t>(uu & 7) ^ sw) << 4),
-                                      src + uu * 8);
-                }
-            }
+            for (int rr = 0; rr < kRows; ++rr) copy(rr, half);
             cp_async_commit();
             cp_async_wait<0>();
             thd::fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) thd::mbar_arrive(bar(B_FULL + s));
         }
-        if (!ok) cp_async_wait<0>();
+        cp_async_wait<0>();
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------- MMA issuer
@@ -289,6 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) thd_sparse_mla_attn_kernel(const 
                     thd::tc_fence_after();
                     issue_s(next_s);
                     thd::mma_commit(bar(B_S_FULL + (next_s & 1)));
+                    thd::mma_commit(bar(B_SFREE + next_s % kNST));
                     ++next_s;
                     t_wait = 0;
                     continue;
