@@ -123,13 +123,22 @@ std::vector<thd_bwd_kv_item> build_bwd_kv_plan(const int32_t* cu, int n_docs, in
                 items.push_back(thd_bwd_kv_item{k0, s, e, g, n_q, 0, 0, 0});
         }
     }
-    const int c = kv_groups_per_chunk(cu[n_docs], D, Hkv);
+    // A dk/dv item streams the Q and dO rows of its group's G query heads,
+    // G times the bytes of the group's K and V: chunk the groups by that
+    // footprint, so that the CTAs in flight share the query tiles they read
+    // in L2.
+    const int64_t G = Hkv > 0 ? Hq / Hkv : 1;
+    const int64_t per_group = static_cast<int64_t>(cu[n_docs]) * G * D * 2 * 2;
+    constexpr int64_t kL2Budget = 48ll << 20;  // as for the forward's K / V
+    int64_t cc = per_group > 0 ? kL2Budget / per_group : Hkv;
+    if (cc < 1) cc = 1;
+    if (cc > Hkv) cc = Hkv;
+    const int c = static_cast<int>(cc);
     std::stable_sort(items.begin(), items.end(),
                      [c](const thd_bwd_kv_item& a, const thd_bwd_kv_item& b) {
                          if (a.g / c != b.g / c) return a.g / c < b.g / c;
                          return a.n_q > b.n_q;
                      });
-    (void)Hq;
     return items;
 }
 
