@@ -642,7 +642,85 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 return mbar_wait(bar(idx), parity, abort_flag, prm.status, kStatusTimeout);
             };
             bool ok = wait(L::B_KV_FULL, 0);
-            for (int s = 0; ok && s < n_steps; ++s) {
+            auto issue_st = [&](int s) {  // S^T(s) = K Q(s)^T
+                const uint32_t qoff = ((s % L::NQS) * C::NTILE_BYTES) >> 4;
+#pragma unroll
+                for (int kk = 0; kk < C::D / 16; ++kk) {
+                    const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
+                    const uint32_t on = ((kk >> 2) * C::NBOX_BYTES + (kk & 3) * 32) >> 4;
+                    mma_bf16_ss(tmem_base + C::TM_S, dk0 + o, dq0 + qoff + on, idesc_s, kk > 0 ? 1u : 0u);
+                }
+            };
+            auto issue_dpt = [&](int s) {  // dP^T(s) = V dO(s)^T
+                const uint32_t dooff = ((s % L::NDS) * C::NTILE_BYTES) >> 4;
+#pragma unroll
+                for (int kk = 0; kk < C::D / 16; ++kk) {
+                    const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
+                    const uint32_t on = ((kk >> 2) * C::NBOX_BYTES + (kk & 3) * 32) >> 4;
+                    mma_bf16_ss(tmem_base + C::TM_DP, dv0 + o, ddo0 + dooff + on, idesc_s, kk > 0 ? 1u : 0u);
+                }
+            };
+            if constexpr (C::MODE == kDkDv) {
+                // Order dv(s) S^T(s+1) dk(s) dP^T(s+1): S^T(s+1) overwrites
+                // P^T(s) only after dv(s) and dP^T(s+1) overwrites dS^T(s)
+                // only after dk(s) (in-order tensor pipe), so the tensor core
+                // works on S^T(s+1) while dS^T(s) is formed and on dk(s) and
+                // dP^T(s+1) while P^T(s+1) is: each elementwise phase runs
+                // under two products instead of one.
+                if (ok && n_steps > 0) {
+                    ok = wait(L::B_Q_FULL + 0, 0);
+                    if (ok) {
+                        tc_fence_after();
+                        issue_st(0);
+                        mma_commit(bar(L::B_S_FULL));
+                        ok = wait(L::B_DO_FULL + 0, 0);
+                    }
+                    if (ok) {
+                        tc_fence_after();
+                        issue_dpt(0);
+                        mma_commit(bar(L::B_DP_FULL));
+                    }
+                }
+                for (int s = 0; ok && s < n_steps; ++s) {
+                    const int qs = s % L::NQS, ds = s % L::NDS;
+                    const uint32_t qoff = (qs * C::NTILE_BYTES) >> 4;
+                    const uint32_t dooff = (ds * C::NTILE_BYTES) >> 4;
+                    const bool more = s + 1 < n_steps;
+                    ok = wait(L::B_P_READY, s & 1);
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < C::BN / 16; ++kk)  // dv += P^T dO
+                        mma_bf16_ts(tmem_base + C::TM_ACC0, tmem_base + C::TM_S + pcol<C::BN>(kk),
+                                    ddomn0 + dooff + ((kk * 16 * 128) >> 4), idesc_acc,
+                                    (s > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(bar(L::B_DO_EMPTY + ds));  // dO(s) done
+                    if (more) {
+                        ok = wait(L::B_Q_FULL + (s + 1) % L::NQS, ((s + 1) / L::NQS) & 1);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_st(s + 1);
+                        mma_commit(bar(L::B_S_FULL));
+                    }
+                    ok = wait(L::B_DS_READY, s & 1);
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < C::BN / 16; ++kk)  // dk += dS^T Q
+                        mma_bf16_ts(tmem_base + C::TM_ACC1, tmem_base + C::TM_DP + pcol<C::BN>(kk),
+                                    dqmn0 + qoff + ((kk * 16 * 128) >> 4), idesc_acc,
+                                    (s > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(bar(L::B_Q_EMPTY + qs));  // Q(s) done
+                    if (more) {
+                        ok = wait(L::B_DO_FULL + (s + 1) % L::NDS, ((s + 1) / L::NDS) & 1);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_dpt(s + 1);
+                        mma_commit(bar(L::B_DP_FULL));
+                    }
+                }
+            }
+            for (int s = 0; ok && s < n_steps && C::MODE != kDkDv; ++s) {
                 const int qs = s % L::NQS, ds = s % L::NDS;
                 ok = wait(L::B_Q_FULL + qs, (s / L::NQS) & 1);
                 if (!ok) break;
