@@ -309,7 +309,7 @@ int launch_bwd256(DeviceState* ds, const BwdPlanEntry& plan, const CUtensorMap& 
                   const void* dout, const float* sinks, float* dsinks, float* delta,
                   float* sink_part, cudaStream_t stream) {
     using Cq = thd::BwdConfig<256, 3, 64>;
-    using Cdv = thd::BwdConfig<256, 2, 64, thd::kDvOnly>;
+    using Cdv = thd::BwdConfig<256, 3, 64, thd::kDvOnly, 2, 2>;  // three Q slots, two dO, two S^T buffers
     using Cdk = thd::BwdConfig<256, 2, 64, thd::kDkOnly, 1>;  // two Q slots, one dO slot
     auto kq = thd::thd_attn_bwd_dq_kernel<Cq>;
     auto kdv = thd::thd_attn_bwd_dkdv_kernel<Cdv>;

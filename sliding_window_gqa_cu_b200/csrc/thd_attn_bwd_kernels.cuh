@@ -158,11 +158,12 @@ __global__ void __launch_bounds__(256) thd_attn_bwd_dsink_kernel(const float* __
 // or one of them (head dim 256, two launches).
 enum BwdKvMode { kDkDv = 0, kDvOnly = 1, kDkOnly = 2 };
 
-template <int D_, int NSLOT_, int BN_ = 128, int MODE_ = kDkDv, int NDSLOT_ = NSLOT_>
+template <int D_, int NSLOT_, int BN_ = 128, int MODE_ = kDkDv, int NDSLOT_ = NSLOT_, int NBUF_ = 1>
 struct BwdConfig {
     static constexpr int D = D_;
     static constexpr int NSLOT = NSLOT_;    // dq: K/V ring slots; dkdv: Q tile slots
     static constexpr int NDSLOT = NDSLOT_;  // dkdv: dO tile slots
+    static constexpr int NBUF = NBUF_;      // dkdv: S^T / dP^T buffers (2: one accumulator, BN = 64)
     static constexpr int BM = 128;        // TMEM lanes (queries for dq, keys for dkdv)
     static constexpr int BN = BN_;        // columns of S per tile (keys for dq, queries for dkdv)
     static constexpr int MODE = MODE_;    // dkdv kernel only
@@ -486,11 +487,20 @@ struct DkvLayout {
     static constexpr int B_Q_EMPTY = B_Q_FULL + NQS;       // [NQS]
     static constexpr int B_DO_FULL = B_Q_EMPTY + NQS;      // [NDS] dO tile
     static constexpr int B_DO_EMPTY = B_DO_FULL + NDS;     // [NDS]
-    static constexpr int B_S_FULL = B_DO_EMPTY + NDS;      // S^T done
-    static constexpr int B_DP_FULL = B_S_FULL + 1;            // dP^T done
-    static constexpr int B_P_READY = B_DP_FULL + 1;           // P^T in TMEM (8 warps)
-    static constexpr int B_DS_READY = B_P_READY + 1;          // dS^T in TMEM (8 warps)
-    static constexpr int B_ACC_FULL = B_DS_READY + 1;         // dk, dv accumulated
+    // Score buffers: with one accumulator and 64-column score tiles, two
+    // S^T (and two dP^T) buffers fit in TMEM beside it; step s uses buffer
+    // s % NB.  The scores of step s + NB need Q(s + NB) while Q(s) is still
+    // in use, so two buffers want a third Q slot.
+    static constexpr int NB = C::NBUF;
+    static_assert(NB == 1 || (NB == 2 && C::MODE != kDkDv && C::BN == 64 && NQS >= 3),
+                  "two score buffers: one accumulator, 64-column tiles, three Q slots");
+    static_assert(C::TM_S + NB * C::BN <= C::TM_DP && C::TM_DP + NB * C::BN <= C::TM_ACC0,
+                  "score buffers overlap");
+    static constexpr int B_S_FULL = B_DO_EMPTY + NDS;      // [NB] S^T done
+    static constexpr int B_DP_FULL = B_S_FULL + NB;           // [NB] dP^T done
+    static constexpr int B_P_READY = B_DP_FULL + NB;          // [NB] P^T in TMEM (8 warps)
+    static constexpr int B_DS_READY = B_P_READY + NB;         // [NB] dS^T in TMEM (8 warps)
+    static constexpr int B_ACC_FULL = B_DS_READY + NB;        // dk, dv accumulated
     static constexpr int B_DRAIN = B_ACC_FULL + 1;
     static constexpr int NUM_BARS = B_DRAIN + 1;
     static constexpr int SMEM_K = 0;
@@ -543,10 +553,12 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
             mbar_init(bar(L::B_DO_FULL + s), 1);
             mbar_init(bar(L::B_DO_EMPTY + s), 1);
         }
-        mbar_init(bar(L::B_S_FULL), 1);
-        mbar_init(bar(L::B_DP_FULL), 1);
-        mbar_init(bar(L::B_P_READY), 8);
-        mbar_init(bar(L::B_DS_READY), 8);
+        for (int b = 0; b < L::NB; ++b) {
+            mbar_init(bar(L::B_S_FULL + b), 1);
+            mbar_init(bar(L::B_DP_FULL + b), 1);
+            mbar_init(bar(L::B_P_READY + b), 8);
+            mbar_init(bar(L::B_DS_READY + b), 8);
+        }
         mbar_init(bar(L::B_ACC_FULL), 1);
         mbar_init(bar(L::B_DRAIN), 1);
         *abort_flag = *reinterpret_cast<volatile int*>(prm.status) != 0 ? 1 : 0;
@@ -648,7 +660,8 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 for (int kk = 0; kk < C::D / 16; ++kk) {
                     const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
                     const uint32_t on = ((kk >> 2) * C::NBOX_BYTES + (kk & 3) * 32) >> 4;
-                    mma_bf16_ss(tmem_base + C::TM_S, dk0 + o, dq0 + qoff + on, idesc_s, kk > 0 ? 1u : 0u);
+                    mma_bf16_ss(tmem_base + C::TM_S + C::BN * (s % L::NB), dk0 + o, dq0 + qoff + on, idesc_s,
+                                kk > 0 ? 1u : 0u);
                 }
             };
             auto issue_dpt = [&](int s) {  // dP^T(s) = V dO(s)^T
@@ -657,7 +670,8 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 for (int kk = 0; kk < C::D / 16; ++kk) {
                     const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
                     const uint32_t on = ((kk >> 2) * C::NBOX_BYTES + (kk & 3) * 32) >> 4;
-                    mma_bf16_ss(tmem_base + C::TM_DP, dv0 + o, ddo0 + dooff + on, idesc_s, kk > 0 ? 1u : 0u);
+                    mma_bf16_ss(tmem_base + C::TM_DP + C::BN * (s % L::NB), dv0 + o, ddo0 + dooff + on, idesc_s,
+                                kk > 0 ? 1u : 0u);
                 }
             };
             if constexpr (C::MODE == kDkDv) {
@@ -720,60 +734,58 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     }
                 }
             }
-            for (int s = 0; ok && s < n_steps && C::MODE != kDkDv; ++s) {
-                const int qs = s % L::NQS, ds = s % L::NDS;
-                ok = wait(L::B_Q_FULL + qs, (s / L::NQS) & 1);
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t qoff = (qs * C::NTILE_BYTES) >> 4;
-                const uint32_t dooff = (ds * C::NTILE_BYTES) >> 4;
-#pragma unroll
-                for (int kk = 0; kk < C::D / 16; ++kk) {  // S^T = K Q^T
-                    const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
-                    const uint32_t on = ((kk >> 2) * C::NBOX_BYTES + (kk & 3) * 32) >> 4;
-                    mma_bf16_ss(tmem_base + C::TM_S, dk0 + o, dq0 + qoff + on, idesc_s,
-                                kk > 0 ? 1u : 0u);
-                }
-                mma_commit(bar(L::B_S_FULL));  // the exponentials start under dP^T
-                ok = wait(L::B_DO_FULL + ds, (s / L::NDS) & 1);
-                if (!ok) break;
-                tc_fence_after();
-                if constexpr (kDk) {
-#pragma unroll
-                    for (int kk = 0; kk < C::D / 16; ++kk) {  // dP^T = V dO^T
-                        const uint32_t o = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
-                        const uint32_t on = ((kk >> 2) * C::NBOX_BYTES + (kk & 3) * 32) >> 4;
-                        mma_bf16_ss(tmem_base + C::TM_DP, dv0 + o, ddo0 + dooff + on, idesc_s,
-                                    kk > 0 ? 1u : 0u);
+            if constexpr (C::MODE != kDkDv) {
+                // One accumulator: S^T(s + NB) (and dP^T(s + NB)) go out after
+                // the product of step s that reads the buffer they
+                // overwrite, so with two buffers the next step's scores are
+                // computed while this step's elementwise work runs.
+                auto issue_scores = [&](int s) -> bool {
+                    if (!wait(L::B_Q_FULL + s % L::NQS, (s / L::NQS) & 1)) return false;
+                    tc_fence_after();
+                    issue_st(s);
+                    mma_commit(bar(L::B_S_FULL + s % L::NB));
+                    if constexpr (kDk) {
+                        if (!wait(L::B_DO_FULL + s % L::NDS, (s / L::NDS) & 1)) return false;
+                        tc_fence_after();
+                        issue_dpt(s);
+                        mma_commit(bar(L::B_DP_FULL + s % L::NB));
+                        mma_commit(bar(L::B_DO_EMPTY + s % L::NDS));  // dO(s) read by dP^T only
                     }
-                    mma_commit(bar(L::B_DP_FULL));
-                    if constexpr (!kDv) mma_commit(bar(L::B_DO_EMPTY + ds));  // dO(s) read by dP^T only
-                }
-                if constexpr (kDv) {
-                    ok = wait(L::B_P_READY, s & 1);
-                    if (!ok) break;
-                    tc_fence_after();
+                    return true;
+                };
+                for (int j = 0; ok && j < L::NB && j < n_steps; ++j) ok = issue_scores(j);
+                for (int s = 0; ok && s < n_steps; ++s) {
+                    const int qs = s % L::NQS, ds = s % L::NDS, b = s % L::NB;
+                    const uint32_t ph = (s / L::NB) & 1;
+                    if constexpr (kDv) {
+                        ok = wait(L::B_DO_FULL + ds, (s / L::NDS) & 1) && wait(L::B_P_READY + b, ph);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint32_t dooff = (ds * C::NTILE_BYTES) >> 4;
 #pragma unroll
-                    for (int kk = 0; kk < C::BN / 16; ++kk)  // dv += P^T dO (16 query rows a step)
-                        mma_bf16_ts(tmem_base + C::TM_ACC0, tmem_base + C::TM_S + pcol<C::BN>(kk),
-                                    ddomn0 + dooff + ((kk * 16 * 128) >> 4), idesc_acc,
-                                    (s > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(bar(L::B_DO_EMPTY + ds));  // dO(s) done
-                    // Q(s)'s slot also holds the lse / delta values the
-                    // elementwise warps read before P_READY: release it here
-                    // when no dk product follows.
-                    if constexpr (!kDk) mma_commit(bar(L::B_Q_EMPTY + qs));
-                }
-                if constexpr (kDk) {
-                    ok = wait(L::B_DS_READY, s & 1);  // dS^T is computed under dv
-                    if (!ok) break;
-                    tc_fence_after();
+                        for (int kk = 0; kk < C::BN / 16; ++kk)  // dv += P^T dO
+                            mma_bf16_ts(tmem_base + C::TM_ACC0,
+                                        tmem_base + C::TM_S + C::BN * b + pcol<C::BN>(kk),
+                                        ddomn0 + dooff + ((kk * 16 * 128) >> 4), idesc_acc,
+                                        (s > 0 || kk > 0) ? 1u : 0u);
+                        mma_commit(bar(L::B_DO_EMPTY + ds));  // dO(s) done
+                        // Q(s)'s slot also holds the lse / delta values the
+                        // elementwise warps read before P_READY.
+                        mma_commit(bar(L::B_Q_EMPTY + qs));
+                    } else {
+                        ok = wait(L::B_DS_READY + b, ph);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint32_t qoff = (qs * C::NTILE_BYTES) >> 4;
 #pragma unroll
-                    for (int kk = 0; kk < C::BN / 16; ++kk)  // dk += dS^T Q
-                        mma_bf16_ts(tmem_base + C::TM_ACC1, tmem_base + C::TM_DP + pcol<C::BN>(kk),
-                                    dqmn0 + qoff + ((kk * 16 * 128) >> 4), idesc_acc,
-                                    (s > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(bar(L::B_Q_EMPTY + qs));  // Q(s) done
+                        for (int kk = 0; kk < C::BN / 16; ++kk)  // dk += dS^T Q
+                            mma_bf16_ts(tmem_base + C::TM_ACC1,
+                                        tmem_base + C::TM_DP + C::BN * b + pcol<C::BN>(kk),
+                                        dqmn0 + qoff + ((kk * 16 * 128) >> 4), idesc_acc,
+                                        (s > 0 || kk > 0) ? 1u : 0u);
+                        mma_commit(bar(L::B_Q_EMPTY + qs));  // Q(s) done
+                    }
+                    if (s + L::NB < n_steps) ok = issue_scores(s + L::NB);
                 }
             }
             if (ok) mma_commit(bar(L::B_ACC_FULL));
@@ -803,8 +815,11 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
             const int qs = s % L::NQS;
             const int ih = it.k0 + (s % nsub) * C::BN + HALF * h;  // first query of this half
             // The side values of this step were stored before Q_FULL.
+            const int b = s % L::NB;
+            const uint32_t ph = (s / L::NB) & 1;
+            const uint32_t tm_s = C::TM_S + C::BN * b, tm_dp = C::TM_DP + C::BN * b;
             ok = warp_wait(bar(L::B_Q_FULL + qs), (s / L::NQS) & 1, abort_flag, prm.status) &&
-                 warp_wait(bar(L::B_S_FULL), s & 1, abort_flag, prm.status);
+                 warp_wait(bar(L::B_S_FULL + b), ph, abort_flag, prm.status);
             if (!ok) break;
             tc_fence_after();
             const float* lse2 = side + qs * 2 * C::BN + HALF * h;
@@ -820,7 +835,7 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 uint32_t sr[HALF];
 #pragma unroll
                 for (int cc = 0; cc < HALF / 32; ++cc)
-                    tmem_ld32(lane_base + C::TM_S + HALF * h + 32 * cc,
+                    tmem_ld32(lane_base + tm_s + HALF * h + 32 * cc,
                               *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]));
                 tmem_wait_ld();
 #pragma unroll
@@ -844,7 +859,7 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     // Over this half's own first S^T columns, all read.
 #pragma unroll
                     for (int cc = 0; cc < HALF / 32; ++cc)
-                        tmem_st16(lane_base + C::TM_S + HALF * h + 16 * cc,
+                        tmem_st16(lane_base + tm_s + HALF * h + 16 * cc,
                                   *reinterpret_cast<uint32_t(*)[16]>(&pp[16 * cc]));
                 }
             }
@@ -852,17 +867,17 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar(L::B_P_READY));
+                if (lane == 0) mbar_arrive(bar(L::B_P_READY + b));
             }
             if constexpr (kDk) {
                 // ... then dS^T = P^T (dP^T - delta) while it computes dv.
-                ok = warp_wait(bar(L::B_DP_FULL), s & 1, abort_flag, prm.status);
+                ok = warp_wait(bar(L::B_DP_FULL + b), ph, abort_flag, prm.status);
                 if (!ok) break;
                 tc_fence_after();
 #pragma unroll
                 for (int cc = 0; cc < HALF / 32; ++cc) {
                     uint32_t dr[32];
-                    tmem_ld32(lane_base + C::TM_DP + HALF * h + 32 * cc, dr);
+                    tmem_ld32(lane_base + tm_dp + HALF * h + 32 * cc, dr);
                     tmem_wait_ld();
                     reg_fence32(dr);
                     uint32_t pd[16];
@@ -878,12 +893,12 @@ thd_attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
                         pd[2 * u + 1] = pack_bf16x2(dsv[2], dsv[3]);
                     }
                     // Over dP^T columns HALF h + [16 cc, 16 cc + 16), already read.
-                    tmem_st16(lane_base + C::TM_DP + HALF * h + 16 * cc, pd);
+                    tmem_st16(lane_base + tm_dp + HALF * h + 16 * cc, pd);
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar(L::B_DS_READY));
+                if (lane == 0) mbar_arrive(bar(L::B_DS_READY + b));
             }
         }
         if (ok) ok = warp_wait(bar(L::B_ACC_FULL), 0, abort_flag, prm.status);
