@@ -337,8 +337,8 @@ __global__ void __launch_bounds__(kThreads, 1) thd_sparse_mla_attn_kernel(const 
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
         bool ok = !skip;
         if (ok) {
-            // Q row h, columns [0, kQT), into TMEM (bf16 pairs): rounds of 64
-            // columns, the next round's loads in flight while this one is
+            // Q row h, columns [0, kQT), into TMEM (bf16 pairs): batches of
+            // 64 columns, the next batch's loads in flight while this one is
             // stored.  (Columns kQT and up arrive by TMA.)
             const uint4* src = reinterpret_cast<const uint4*>(p.q + (t * p.H + h) * kQDim);
             uint4 x[2][8];
