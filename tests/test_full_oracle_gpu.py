@@ -56,3 +56,40 @@ def test_full_size_pack_every_row_full_oracle(name):
     print("FULL_ORACLE " + json.dumps(rec), flush=True)
     assert np.isfinite(out.float().numpy()).all()
     assert err.max() <= OUT_MAX and err.mean() <= OUT_MEAN and lerr.max() <= LSE_MAX
+
+
+@pytest.mark.parametrize("name", ["pack8k_gqa4_d128_causal", "pack32k_gqa4_d128_w4096"])
+def test_full_size_pack_bwd_every_element_full_oracle(name):
+    """dq, dk and dv of the 8k and 32k packs on every element against the
+    full fp64 backward oracle (the derivative of the same definition), with
+    the backward tolerances: max error 2e-2 and mean error 2e-3 of max|ref|
+    per tensor.  The default GPU suite checks these packs' gradients on
+    sampled rows."""
+    cfg = workloads.CONFIGS[name]
+    p = workloads.make_pack(cfg, 0)
+    dev = torch.device("cuda:0")
+    g = torch.Generator().manual_seed(5)
+    dout = torch.randn(p["q"].shape, generator=g).to(torch.bfloat16)
+    q, k, v = (p[n].to(dev) for n in "qkv")
+    sinks = p["sinks"].to(dev) if p["sinks"] is not None else None
+    out, lse = swa.thd_attn_fwd(q, k, v, p["cu_seqlens"], cfg.window, cfg.scale, sinks)
+    dq, dk, dv, ds = swa.thd_attn_bwd(q, k, v, out, lse, dout.to(dev), p["cu_seqlens"], cfg.window,
+                                      cfg.scale, sinks)
+    torch.cuda.synchronize()
+    assert swa.thd_attn_get_error() == 0
+    got = {"dq": dq.cpu(), "dk": dk.cpu(), "dv": dv.cpu()}
+    del q, k, v, out, lse, dq, dk, dv
+    t0 = time.time()
+    rq, rk, rv, rs = oracle.attention_bwd(p["q"], p["k"], p["v"], dout, p["cu_seqlens"], cfg.window,
+                                          cfg.scale, p["sinks"])
+    secs = time.time() - t0
+    rec = {"workload": name, "oracle_seconds": round(secs, 1), "oracle_threads": oracle.num_threads()}
+    ok = True
+    for key, ref in (("dq", rq), ("dk", rk), ("dv", rv)):
+        gv = got[key].double().numpy().reshape(ref.shape)
+        scale = max(float(np.abs(ref).max()), 1e-3)
+        err = np.abs(gv - ref)
+        rec[key] = {"max_abs": float(err.max()), "mean_abs": float(err.mean()), "max_ref": scale}
+        ok = ok and np.isfinite(gv).all() and err.max() <= REL_MAX * scale and err.mean() <= REL_MEAN * scale
+    print("FULL_ORACLE_BWD " + json.dumps(rec), flush=True)
+    assert ok, rec
