@@ -395,7 +395,8 @@ def measure_bwd(swa, name, args, info, device, stream, clocks, peaks):
     return summarise(tot, per, args, work * info.world, UNIT, peak * info.world, peaks,
                      clocks.summary(h0, h1), "thd_attn_bwd_dq_kernel + thd_attn_bwd_dkdv_kernel",
                      {"workload": name, "valid_pairs": int(pairs), "tokens": T,
-                      "launches_per_step": 4 if t["sinks"] is not None else 3,
+                      # preprocess, dq, dk/dv (dv and dk apart at D = 256), dsink with sinks
+                      "launches_per_step": (4 if cfg.D == 256 else 3) + (1 if t["sinks"] is not None else 0),
                       "metric": "THD varlen attention bwd TFLOP/s (valid pairs, 2.5x forward FLOP)"})
 
 
@@ -444,7 +445,8 @@ def measure_sparse_mla(swa, args, info, device, stream, clocks, peaks):
     return summarise(tot, per, args, flop * info.world, UNIT, peak * info.world, peaks,
                      clocks.summary(h0, h1), "thd_sparse_mla_attn_kernel + thd_sparse_mla_proj_kernel",
                      {"workload": w["name"], "tokens": T, "heads": H, "selected_keys": w["K"],
-                      "value_dim": vd, "valid_slots": valid, "launches_per_step": 2,
+                      "value_dim": vd, "valid_slots": valid,
+                      "launches_per_step": 3,  # slot compaction, attention, projection
                       "metric": "sparse MLA fwd TFLOP/s (valid slots, incl. value projection)"})
 
 
