@@ -161,6 +161,48 @@ int thd_attn_fwd_range(const void* q, const void* k, const void* v,
                        void* stream);
 
 /*
+ * thd_attn_fwd_range with the keys restricted to j < k_end: each row sees the
+ * keys its causal / document / window rule allows AND below k_end.  This is
+ * the part of a context-parallel row that lies on earlier ranks (the Magi
+ * plans of the "muse_spark.magi_cp" page exchange keys between the ranks of
+ * MuseMagiPlan.attention; a rank owning rows [b, e) can compute the keys at
+ * or after b from its own slice and add the keys before b once they have
+ * arrived, merging the two with thd_attn_merge).
+ *   k, v       bf16 device [T, Hkv, D]; only rows j < k_end are read (rows
+ *              below a document start may be read and are masked)
+ *   k_end      0 <= k_end <= T, else THD_ERR_INVALID_ARG; k_end = T is
+ *              thd_attn_fwd_range
+ *   other arguments as thd_attn_fwd_range.  A row with no key below k_end
+ *   gets out = 0 and lse = -inf (or, with sinks, lse = the sink logit).
+ */
+int thd_attn_fwd_range_keys(const void* q, const void* k, const void* v,
+                            const int32_t* cu_seqlens, int n_docs,
+                            int64_t q_begin, int64_t q_end, int64_t k_end,
+                            int Hq, int Hkv, int D, int window, float scale,
+                            const float* sinks_or_null,
+                            void* out, float* lse,
+                            void* stream);
+
+/*
+ * Merges two partial results of the same rows computed over disjoint key
+ * sets (for example thd_attn_fwd on a rank's own slice of the pack and
+ * thd_attn_fwd_range_keys on the keys before it).  The pages print no such
+ * step: it is the log-sum-exp combination of two softmax parts, with
+ * m = max(lse_a, lse_b), w = exp(lse - m):
+ *   lse = m + log(w_a + w_b),  out = (w_a out_a + w_b out_b) / (w_a + w_b);
+ * a part with lse = -inf has weight 0 (both -inf: out = 0, lse = -inf).
+ * Sinks belong to exactly one of the parts.
+ *   out_a, out_b   bf16 device [rows, Hq, D], 16-byte aligned
+ *   lse_a, lse_b   fp32 device [rows, Hq] (natural log, as thd_attn_fwd)
+ *   out, lse       results, same shapes; may be out_a / lse_a (in place)
+ * D in {64, 128, 256} else THD_ERR_UNSUPPORTED; a NULL or misaligned buffer
+ * (rows > 0) THD_ERR_INVALID_ARG; rows = 0 is a no-op.  Asynchronous on
+ * `stream`.
+ */
+int thd_attn_merge(const void* out_a, const float* lse_a, const void* out_b, const float* lse_b,
+                   int64_t rows, int Hq, int D, void* out, float* lse, void* stream);
+
+/*
  * The forward from HOST buffers, with the copies overlapped with the
  * attention.  The pages have no counterpart of this entry point: it computes
  * the same packed-THD forward as thd_attn_fwd (MuseMagiPlan.attention,
@@ -209,6 +251,13 @@ int thd_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host
 int thd_attn_plan_range(const int32_t* cu_seqlens, int n_docs, int64_t q_begin, int64_t q_end,
                         int Hq, int Hkv, int D, int window,
                         thd_work_item* items, int64_t capacity, int64_t* n_items);
+
+/* Host-only: the schedule thd_attn_fwd_range_keys uses (key tiles end at
+ * min(tile end, k_end); a tile whose rows see no key below k_end keeps one
+ * wholly masked key tile).  Same conventions as thd_attn_plan. */
+int thd_attn_plan_range_keys(const int32_t* cu_seqlens, int n_docs, int64_t q_begin,
+                             int64_t q_end, int64_t k_end, int Hq, int Hkv, int D, int window,
+                             thd_work_item* items, int64_t capacity, int64_t* n_items);
 
 /*
  * Allocation-free variant of thd_attn_fwd.  The pages have no counterpart of

@@ -20,11 +20,12 @@ from typing import Optional
 
 import numpy as np
 
-__all__ = ["thd_attn_fwd", "thd_attn_fwd_noalloc", "thd_attn_fwd_range", "thd_attn_fwd_host",
+__all__ = ["thd_attn_fwd", "thd_attn_fwd_noalloc", "thd_attn_fwd_range", "thd_attn_merge",
+           "thd_attn_fwd_host",
            "thd_attn_bwd", "thd_attn_bwd_workspace_bytes", "thd_qk_norm_rope",
            "thd_sparse_mla_fwd", "thd_sparse_mla_workspace_bytes", "thd_sparse_mla_get_error",
            "thd_attn_get_error", "thd_attn_noalloc_get_error", "thd_attn_selftest_stall", "thd_attn_plan", "thd_attn_plan_range",
-           "ThdAttnError", "library_path", "load_library", "STATUS"]
+           "thd_attn_plan_range_keys", "ThdAttnError", "library_path", "load_library", "STATUS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_NAME = "libthdattn.so"
@@ -94,6 +95,12 @@ def bind(lib):
     lib.thd_attn_fwd_range.argtypes = [vp, vp, vp, i32p, c_int, ctypes.c_int64, ctypes.c_int64,
                                        c_int, c_int, c_int, c_int, ctypes.c_float, vp, vp, vp, vp]
     lib.thd_attn_fwd_range.restype = c_int
+    lib.thd_attn_fwd_range_keys.argtypes = [vp, vp, vp, i32p, c_int, ctypes.c_int64, ctypes.c_int64,
+                                            ctypes.c_int64, c_int, c_int, c_int, c_int, ctypes.c_float,
+                                            vp, vp, vp, vp]
+    lib.thd_attn_fwd_range_keys.restype = c_int
+    lib.thd_attn_merge.argtypes = [vp, vp, vp, vp, ctypes.c_int64, c_int, c_int, vp, vp, vp]
+    lib.thd_attn_merge.restype = c_int
     lib.thd_attn_fwd_host.argtypes = [vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int,
                                       ctypes.c_float, vp, vp, vp, vp, vp, vp, vp, vp, vp, c_int, vp]
     lib.thd_attn_fwd_host.restype = c_int
@@ -103,6 +110,10 @@ def bind(lib):
                                         c_int, c_int, vp, ctypes.c_int64,
                                         ctypes.POINTER(ctypes.c_int64)]
     lib.thd_attn_plan_range.restype = c_int
+    lib.thd_attn_plan_range_keys.argtypes = [i32p, c_int, ctypes.c_int64, ctypes.c_int64,
+                                             ctypes.c_int64, c_int, c_int, c_int, c_int, vp,
+                                             ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)]
+    lib.thd_attn_plan_range_keys.restype = c_int
     lib.thd_sparse_mla_workspace_bytes.argtypes = [ctypes.c_int64, c_int, c_int]
     lib.thd_sparse_mla_workspace_bytes.restype = ctypes.c_size_t
     lib.thd_sparse_mla_fwd.argtypes = [vp, vp, vp, vp, ctypes.c_int64, ctypes.c_int64, c_int, c_int,
@@ -309,13 +320,14 @@ def thd_qk_norm_rope(q, k, cu_seqlens, eps: float = 1e-5, theta: float = 500000.
 
 def thd_attn_fwd_range(q, k, v, cu_seqlens, q_begin: int, q_end: int, window: int = 0,
                        scale: Optional[float] = None, sinks=None, out=None, lse=None,
-                       return_lse: bool = True, stream=None):
+                       return_lse: bool = True, stream=None, k_end: Optional[int] = None):
     """Forward of the query rows [q_begin, q_end) of the pack against K/V of
     the whole pack (the local step of a context-parallel forward).
 
     q: bf16 CUDA [q_end - q_begin, Hq, D]; k, v: bf16 CUDA [T, Hkv, D];
-    cu_seqlens: host boundaries of the whole pack.  Returns ``(out, lse)`` for
-    those rows.
+    cu_seqlens: host boundaries of the whole pack.  ``k_end`` (default T)
+    restricts the keys to j < k_end (``thd_attn_fwd_range_keys``; only those
+    rows of k and v are read).  Returns ``(out, lse)`` for those rows.
     """
     import torch
 
@@ -332,6 +344,10 @@ def thd_attn_fwd_range(q, k, v, cu_seqlens, q_begin: int, q_end: int, window: in
         raise ValueError(f"cu_seqlens[-1]={int(cu[-1])} does not match {T} key tokens")
     if not (0 <= q_begin <= q_end <= T) or q_end - q_begin != Tq:
         raise ValueError("q must hold exactly the rows [q_begin, q_end) of the pack")
+    if k_end is None:
+        k_end = T
+    if not (0 <= k_end <= T):
+        raise ValueError(f"k_end={k_end} outside [0, {T}]")
     if scale is None:
         scale = D ** -0.5
     if sinks is not None:
@@ -345,15 +361,45 @@ def thd_attn_fwd_range(q, k, v, cu_seqlens, q_begin: int, q_end: int, window: in
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     with torch.cuda.device(q.device):
-        rc = lib.thd_attn_fwd_range(
+        rc = lib.thd_attn_fwd_range_keys(
             q.data_ptr(), k.data_ptr(), v.data_ptr(),
             cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), cu.size - 1,
-            int(q_begin), int(q_end), Hq, Hkv, D, int(window), float(scale),
+            int(q_begin), int(q_end), int(k_end), Hq, Hkv, D, int(window), float(scale),
             sinks.data_ptr() if sinks is not None else None,
             out.data_ptr(), lse.data_ptr() if lse is not None else None,
             ctypes.c_void_p(stream.cuda_stream))
     if rc != 0:
         raise ThdAttnError(rc, "thd_attn_fwd_range")
+    return out, lse
+
+
+def thd_attn_merge(out_a, lse_a, out_b, lse_b, out=None, lse=None, stream=None):
+    """Merge two partial results of the same rows over disjoint key sets
+    (log-sum-exp combination, ``thd_attn_merge``).  out_*: bf16 CUDA
+    [rows, Hq, D]; lse_*: fp32 CUDA [rows, Hq].  ``out`` / ``lse`` default to
+    new tensors and may be ``out_a`` / ``lse_a``.  Returns ``(out, lse)``."""
+    import torch
+
+    lib = load_library()
+    rows, Hq, D = out_a.shape
+    for name, t, dt, shape in (("out_a", out_a, torch.bfloat16, (rows, Hq, D)),
+                               ("out_b", out_b, torch.bfloat16, (rows, Hq, D)),
+                               ("lse_a", lse_a, torch.float32, (rows, Hq)),
+                               ("lse_b", lse_b, torch.float32, (rows, Hq))):
+        if t.dtype != dt or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != shape:
+            raise ValueError(f"{name} must be a contiguous {dt} CUDA tensor of shape {shape}")
+    if out is None:
+        out = torch.empty_like(out_a)
+    if lse is None:
+        lse = torch.empty_like(lse_a)
+    if stream is None:
+        stream = torch.cuda.current_stream(out_a.device)
+    with torch.cuda.device(out_a.device):
+        rc = lib.thd_attn_merge(out_a.data_ptr(), lse_a.data_ptr(), out_b.data_ptr(), lse_b.data_ptr(),
+                                rows, Hq, D, out.data_ptr(), lse.data_ptr(),
+                                ctypes.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise ThdAttnError(rc, "thd_attn_merge")
     return out, lse
 
 
@@ -419,6 +465,26 @@ def thd_attn_fwd_host(q_host, k_host, v_host, cu_seqlens, window: int = 0,
     if rc != 0:
         raise ThdAttnError(rc, "thd_attn_fwd_host")
     return out_host, lse_host
+
+
+def thd_attn_plan_range_keys(cu_seqlens, q_begin: int, q_end: int, k_end: int, Hq: int, Hkv: int,
+                             D: int, window: int) -> np.ndarray:
+    """Host-only: the work list of :func:`thd_attn_fwd_range` with keys below
+    ``k_end`` only (structured array)."""
+    lib = load_library()
+    cu = _cu_array(cu_seqlens)
+    n = ctypes.c_int64(0)
+    args = (cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), cu.size - 1, int(q_begin), int(q_end),
+            int(k_end), Hq, Hkv, D, int(window))
+    rc = lib.thd_attn_plan_range_keys(*args, None, 0, ctypes.byref(n))
+    if rc != 0:
+        raise ThdAttnError(rc, "thd_attn_plan_range_keys")
+    dt = np.dtype([(f, np.int32) for f in WORK_ITEM_FIELDS])
+    items = np.zeros(max(1, n.value), dtype=dt)
+    rc = lib.thd_attn_plan_range_keys(*args, items.ctypes.data, n.value, ctypes.byref(n))
+    if rc != 0:
+        raise ThdAttnError(rc, "thd_attn_plan_range_keys")
+    return items[:n.value].copy()
 
 
 def thd_attn_plan_range(cu_seqlens, q_begin: int, q_end: int, Hq: int, Hkv: int, D: int,

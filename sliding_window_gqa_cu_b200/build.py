@@ -16,7 +16,8 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libthdattn.so")
 SOURCES = [os.path.join(CSRC, "thd_attn_api.cu"), os.path.join(CSRC, "thd_attn_noalloc.cu"),
            os.path.join(CSRC, "thd_prologue.cu"), os.path.join(CSRC, "thd_sparse_mla.cu"),
-           os.path.join(CSRC, "thd_host_pipeline.cu"), os.path.join(CSRC, "scheduler.cpp")]
+           os.path.join(CSRC, "thd_host_pipeline.cu"), os.path.join(CSRC, "thd_attn_merge.cu"),
+           os.path.join(CSRC, "scheduler.cpp")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("thd_attn_kernel.cuh", "thd_attn_split_kernel.cuh",
                                                   "thd_attn_bwd_kernels.cuh",
                                                   "sm100_ptx.cuh", "scheduler.h", "tma_map.h")] \

@@ -58,7 +58,7 @@ std::vector<thd_work_item> build_plan(const int32_t* cu, int n_docs, int Hq, int
 
 std::vector<thd_work_item> build_plan_range(const int32_t* cu, int n_docs, int64_t q_begin,
                                             int64_t q_end, int Hq, int Hkv, int window,
-                                            const KernelShape& ks) {
+                                            const KernelShape& ks, int64_t k_end) {
     constexpr int BM = 128;
     const int G = Hq / Hkv;
     const int BN = ks.block_n;
@@ -82,10 +82,13 @@ std::vector<thd_work_item> build_plan_range(const int32_t* cu, int n_docs, int64
             const int r_lo = q0 > s ? q0 : s;
             int k_lo = s;  // lowest key any row of the tile can see
             if (window > 0 && r_lo - window + 1 > k_lo) k_lo = r_lo - window + 1;
-            const int n_kv = (q1 - k_lo + BN - 1) / BN;
-            // Key tiles are aligned to the tile end: the last one sits on the
-            // causal diagonal, keys below k_lo in the first one are masked.
-            const int kv_start = q1 - n_kv * BN;
+            // Key tiles are aligned to the end of the keys the tile may read
+            // (its end, or k_end before it): the last one sits on the causal
+            // diagonal, keys below k_lo in the first one are masked.
+            const int kv_end = static_cast<int>(q1 < k_end ? q1 : k_end);
+            int n_kv = (kv_end - k_lo + BN - 1) / BN;
+            if (n_kv < 1) n_kv = 1;  // no key below k_end: one wholly masked tile
+            const int kv_start = kv_end - n_kv * BN;
             for (int g = 0; g < Hkv; ++g)
                 for (int hp = 0; hp < G / ks.nq; ++hp)
                     items.push_back(thd_work_item{q0, q1, s, g * G + hp * ks.nq, kv_start, n_kv,

@@ -43,10 +43,13 @@ std::vector<thd_work_item> build_plan(const int32_t* cu_seqlens, int n_docs, int
 
 // The same for the query rows [q_begin, q_end) of the pack only (keys from
 // the whole pack): the local step of a context-parallel forward whose rank
-// owns those rows.  build_plan is the range [0, T).
+// owns those rows.  build_plan is the range [0, T).  With k_end < T the rows
+// see only keys j < k_end (the part of a context-parallel row that lies on
+// earlier ranks): a tile's key range then ends at min(tile end, k_end), and a
+// tile whose rows see no such key keeps one key tile, wholly masked.
 std::vector<thd_work_item> build_plan_range(const int32_t* cu_seqlens, int n_docs, int64_t q_begin,
                                             int64_t q_end, int Hq, int Hkv, int window,
-                                            const KernelShape& ks);
+                                            const KernelShape& ks, int64_t k_end = INT64_MAX);
 
 // Key-side work list of the backward (dk, dv): one item per (128-key tile of
 // a document, kv head), with the query tiles that see any of its keys; same

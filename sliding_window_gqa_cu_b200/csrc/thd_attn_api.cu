@@ -48,6 +48,7 @@ struct PlanEntry {
     std::vector<int32_t> cu;
     int Hq, Hkv, D, window;
     int64_t q_begin, q_end;  // query rows of the pack the plan covers
+    int64_t k_end;           // keys j < k_end only (T: all)
     thd::WorkItem* d_items = nullptr;
     int64_t n_items = 0;
 };
@@ -104,12 +105,12 @@ int device_state(DeviceState** out, int* dev_out) {
 }
 
 // Finds or builds (and uploads) the plan for these arguments.  Caller holds g_mu.
-int get_plan(DeviceState* ds, const int32_t* cu, int n_docs, int64_t q_begin, int64_t q_end, int Hq,
-             int Hkv, int D, int window, const KernelShape& ks, cudaStream_t stream,
-             const PlanEntry** out) {
+int get_plan(DeviceState* ds, const int32_t* cu, int n_docs, int64_t q_begin, int64_t q_end,
+             int64_t k_end, int Hq, int Hkv, int D, int window, const KernelShape& ks,
+             cudaStream_t stream, const PlanEntry** out) {
     for (auto it = ds->plans.begin(); it != ds->plans.end(); ++it) {
         if (it->Hq == Hq && it->Hkv == Hkv && it->D == D && it->window == window &&
-            it->q_begin == q_begin && it->q_end == q_end &&
+            it->q_begin == q_begin && it->q_end == q_end && it->k_end == k_end &&
             it->cu.size() == static_cast<size_t>(n_docs) + 1 &&
             std::memcmp(it->cu.data(), cu, sizeof(int32_t) * (n_docs + 1)) == 0) {
             ds->plans.splice(ds->plans.begin(), ds->plans, it);
@@ -118,11 +119,12 @@ int get_plan(DeviceState* ds, const int32_t* cu, int n_docs, int64_t q_begin, in
         }
     }
     std::vector<thd_work_item> items =
-        thd::build_plan_range(cu, n_docs, q_begin, q_end, Hq, Hkv, window, ks);
+        thd::build_plan_range(cu, n_docs, q_begin, q_end, Hq, Hkv, window, ks, k_end);
     PlanEntry e;
     e.cu.assign(cu, cu + n_docs + 1);
     e.q_begin = q_begin;
     e.q_end = q_end;
+    e.k_end = k_end;
     e.Hq = Hq;
     e.Hkv = Hkv;
     e.D = D;
@@ -421,14 +423,24 @@ int thd_attn_plan(const int32_t* cu_seqlens, int n_docs, int Hq, int Hkv, int D,
 int thd_attn_plan_range(const int32_t* cu_seqlens, int n_docs, int64_t q_begin, int64_t q_end,
                         int Hq, int Hkv, int D, int window, thd_work_item* items,
                         int64_t capacity, int64_t* n_items) {
+    if (n_docs < 0 || cu_seqlens == nullptr) return THD_ERR_INVALID_ARG;
+    return thd_attn_plan_range_keys(cu_seqlens, n_docs, q_begin, q_end, cu_seqlens[n_docs], Hq, Hkv,
+                                    D, window, items, capacity, n_items);
+}
+
+int thd_attn_plan_range_keys(const int32_t* cu_seqlens, int n_docs, int64_t q_begin,
+                             int64_t q_end, int64_t k_end, int Hq, int Hkv, int D, int window,
+                             thd_work_item* items, int64_t capacity, int64_t* n_items) {
     if (n_items == nullptr || capacity < 0) return THD_ERR_INVALID_ARG;
     int rc = thd::validate_args(cu_seqlens, n_docs, Hq, Hkv, D, window);
     if (rc != THD_OK) return rc;
-    if (q_begin < 0 || q_end < q_begin || q_end > cu_seqlens[n_docs]) return THD_ERR_INVALID_ARG;
+    if (q_begin < 0 || q_end < q_begin || q_end > cu_seqlens[n_docs] || k_end < 0 ||
+        k_end > cu_seqlens[n_docs])
+        return THD_ERR_INVALID_ARG;
     KernelShape ks;
     if (!thd::choose_kernel_shape(D, Hq / Hkv, &ks)) return THD_ERR_UNSUPPORTED;
     std::vector<thd_work_item> v =
-        thd::build_plan_range(cu_seqlens, n_docs, q_begin, q_end, Hq, Hkv, window, ks);
+        thd::build_plan_range(cu_seqlens, n_docs, q_begin, q_end, Hq, Hkv, window, ks, k_end);
     *n_items = static_cast<int64_t>(v.size());
     if (items != nullptr) {
         const int64_t n = std::min<int64_t>(capacity, static_cast<int64_t>(v.size()));
@@ -441,11 +453,21 @@ int thd_attn_fwd_range(const void* q, const void* k, const void* v, const int32_
                        int n_docs, int64_t q_begin, int64_t q_end, int Hq, int Hkv, int D,
                        int window, float scale, const float* sinks_or_null, void* out, float* lse,
                        void* stream_ptr) {
+    if (n_docs < 0 || cu_seqlens == nullptr) return THD_ERR_INVALID_ARG;
+    return thd_attn_fwd_range_keys(q, k, v, cu_seqlens, n_docs, q_begin, q_end, cu_seqlens[n_docs],
+                                   Hq, Hkv, D, window, scale, sinks_or_null, out, lse, stream_ptr);
+}
+
+int thd_attn_fwd_range_keys(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                            int n_docs, int64_t q_begin, int64_t q_end, int64_t k_end, int Hq,
+                            int Hkv, int D, int window, float scale, const float* sinks_or_null,
+                            void* out, float* lse, void* stream_ptr) {
     int rc = thd::validate_args(cu_seqlens, n_docs, Hq, Hkv, D, window);
     if (rc != THD_OK) return rc;
     if (!(std::isfinite(scale) && scale > 0.0f)) return THD_ERR_INVALID_ARG;
     const int64_t T = cu_seqlens[n_docs];
-    if (q_begin < 0 || q_end < q_begin || q_end > T) return THD_ERR_INVALID_ARG;
+    if (q_begin < 0 || q_end < q_begin || q_end > T || k_end < 0 || k_end > T)
+        return THD_ERR_INVALID_ARG;
     if (T == 0 || q_end == q_begin) return THD_OK;
     if (!q || !k || !v || !out) return THD_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
@@ -462,7 +484,8 @@ int thd_attn_fwd_range(const void* q, const void* k, const void* v, const int32_
     rc = device_state(&ds, nullptr);
     if (rc != THD_OK) return rc;
     const PlanEntry* plan = nullptr;
-    rc = get_plan(ds, cu_seqlens, n_docs, q_begin, q_end, Hq, Hkv, D, window, ks, stream, &plan);
+    rc = get_plan(ds, cu_seqlens, n_docs, q_begin, q_end, k_end, Hq, Hkv, D, window, ks, stream,
+                  &plan);
     if (rc != THD_OK) return rc;
     if (plan->n_items == 0) return THD_OK;
 

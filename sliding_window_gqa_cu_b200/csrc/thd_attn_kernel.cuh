@@ -157,13 +157,13 @@ constexpr int kStatusBadItem = -8;
 
 // Debug build: the invariants every item of the host schedule satisfies
 // (see scheduler.cpp): 1..128 query rows ending in the document, key tiles
-// of block_n keys that end at the tile end, whole GQA head groups of
-// n_heads aligned heads inside [0, Hq).
+// of block_n keys that end at the tile end (or before it, for a key-bounded
+// range), whole GQA head groups of n_heads aligned heads inside [0, Hq).
 __device__ __forceinline__ bool item_ok(const WorkItem& it, const FwdParams& p, int n_heads,
                                         int block_n) {
     return it.n_kv >= 1 && it.block_n == block_n && it.n_heads == n_heads &&
            it.q1 - it.q0 >= 1 && it.q1 - it.q0 <= 128 && it.doc_start < it.q1 &&
-           it.q0 - p.q_offset >= -128 && it.kv_start + it.n_kv * block_n == it.q1 &&
+           it.q0 - p.q_offset >= -128 && it.kv_start + it.n_kv * block_n <= it.q1 &&
            it.head0 >= 0 && it.head0 % n_heads == 0 && it.head0 + n_heads <= p.Hq &&
            (it.head0 / p.G) == (it.head0 + n_heads - 1) / p.G;
 }

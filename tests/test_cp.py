@@ -1,8 +1,10 @@
 """Context-parallel forward, host side (CPU): the token shards, the K/V
-all-gather over a world-size-2 gloo group, and the range schedule of each
-rank's local step (every row of the shard owned exactly once, no row outside
-it, every visible key in its items' key tiles), checked by brute force
-against the window definition of FlintMagiPlan.attention ("flint.magi"
+all-gather over a world-size-2 gloo group (blocking and asynchronous), the
+range schedule of each rank's local step (every row of the shard owned
+exactly once, no row outside it, every visible key in its items' key tiles)
+and its key-bounded form, and the overlapped forward's split of a shard into
+its own-slice pack and the rows with keys on earlier ranks, checked by brute
+force against the window definition of FlintMagiPlan.attention ("flint.magi"
 page)."""
 import os
 import socket
@@ -69,6 +71,78 @@ def test_range_plans_cover_each_shard_exactly(lens, Hq, Hkv, D, window, world):
         check_range_plan(cu, qb, qe, Hq, Hkv, D, window)
 
 
+def check_key_bounded_plan(cu, qb, qe, k_end, Hq, Hkv, D, window):
+    """Every row of [qb, qe) exactly once; an item's key tiles end at
+    min(q1, k_end) (at least one tile); each row's keys below k_end inside
+    them."""
+    plan = swa.thd_attn_plan_range_keys(cu, qb, qe, k_end, Hq, Hkv, D, window)
+    cu = np.asarray(cu)
+    T = int(cu[-1])
+    owner = np.zeros((T, Hq), dtype=int)
+    for it in plan:
+        q0, q1, s, h0 = int(it["q0"]), int(it["q1"]), int(it["doc_start"]), int(it["head0"])
+        ks, nkv, nh, bn = int(it["kv_start"]), int(it["n_kv"]), int(it["n_heads"]), int(it["block_n"])
+        assert nkv >= 1 and ks + nkv * bn == min(q1, k_end)
+        rows = range(max(q0, s, qb), q1)
+        owner[rows.start:rows.stop, h0:h0 + nh] += 1
+        for i in rows:
+            lo = s if window == 0 else max(s, i - window + 1)
+            hi = min(i, k_end - 1)
+            if lo <= hi:
+                assert ks <= lo and hi < ks + nkv * bn
+    assert (owner[qb:qe] == 1).all() and (owner[:qb] == 0).all() and (owner[qe:] == 0).all()
+
+
+@pytest.mark.parametrize("lens,Hq,Hkv,D,window", [
+    ([300, 1, 0, 129, 77], 4, 2, 128, 0),
+    ([300, 1, 0, 129, 77], 4, 2, 128, 100),
+    ([700, 256, 3], 6, 2, 128, 128),
+    ([1000, 33], 16, 1, 256, 129),
+    ([513], 2, 2, 64, 1),
+])
+def test_key_bounded_range_plans(lens, Hq, Hkv, D, window):
+    """The schedule of the keys-before-the-rank part of an overlapped
+    context-parallel row (thd_attn_fwd_range with k_end = the rank's first
+    row), and k_end = T, which is the plain range plan."""
+    cu = workloads.cu_seqlens_from_lengths(lens)
+    T = int(cu[-1])
+    for world in (2, 3, 5):
+        for qb, qe in cp.shard_bounds(T, world):
+            check_key_bounded_plan(cu, qb, qe, qb, Hq, Hkv, D, window)
+            check_key_bounded_plan(cu, qb, qe, T, Hq, Hkv, D, window)
+            assert np.array_equal(swa.thd_attn_plan_range_keys(cu, qb, qe, T, Hq, Hkv, D, window),
+                                  swa.thd_attn_plan_range(cu, qb, qe, Hq, Hkv, D, window))
+    with pytest.raises(swa.ThdAttnError):
+        swa.thd_attn_plan_range_keys(cu, 0, T, T + 1, Hq, Hkv, D, window)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_overlap_split_of_a_shard_by_brute_force(seed):
+    """local_cu_seqlens cuts the pack's documents at the range start (row i
+    of [b, e) keeps the keys of its document at or after b, from the pack's
+    boundaries), and crossing_rows ends the rows whose document started
+    before b -- the only rows with keys on earlier ranks."""
+    rng = np.random.default_rng(seed)
+    lens = [int(x) for x in rng.integers(0, 90, size=int(rng.integers(1, 7)))]
+    cu = workloads.cu_seqlens_from_lengths(lens)
+    T = int(cu[-1])
+    doc_start = np.zeros(T, dtype=int)
+    for d in range(len(lens)):
+        doc_start[cu[d]:cu[d + 1]] = cu[d]
+    for world in (1, 2, 3, 7):
+        for b, e in cp.shard_bounds(T, world):
+            lc = cp.local_cu_seqlens(cu, b, e)
+            assert lc[0] == 0 and lc[-1] == e - b and (np.diff(lc) >= 0).all()
+            x = cp.crossing_rows(cu, b, e)
+            assert b <= x <= e
+            for i in range(b, e):
+                j = int(np.searchsorted(lc, i - b, side="right")) - 1
+                while lc[j + 1] == lc[j]:
+                    j += 1
+                assert lc[j] + b == max(doc_start[i], b)
+                assert (i < x) == (doc_start[i] < b)
+
+
 def test_full_range_plan_is_the_forward_plan():
     cu = workloads.cu_seqlens_from_lengths([300, 1, 0, 129, 77])
     a = swa.thd_attn_plan(cu, 8, 2, 128, 0)
@@ -92,6 +166,10 @@ def _worker(rank, world, port, result_dir):
     k, v = p["k"].float(), p["v"].float()
     kf, vf = cp.gather_kv(k[b:e].contiguous(), v[b:e].contiguous(), T)
     ok = torch.equal(kf, k) and torch.equal(vf, v)
+    # the asynchronous form (the overlapped forward's) gives the same tensors
+    _, _, finish = cp.gather_kv_async(k[b:e].contiguous(), v[b:e].contiguous(), T)
+    ka, va = finish()
+    ok = ok and torch.equal(ka, k) and torch.equal(va, v)
     with open(os.path.join(result_dir, f"r{rank}.txt"), "w") as f:
         f.write("ok" if ok else "mismatch")
     multirank.shutdown()
