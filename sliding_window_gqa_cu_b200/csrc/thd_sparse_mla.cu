@@ -12,8 +12,10 @@
 //
 // 1. Attention (thd_sparse_mla_attn_kernel): one CTA per (token, group of
 //    128 heads, half of the 512 latent columns).  The token's 128 query rows
-//    (128 x 576 bf16) are the A operand of S = Q kv^T: columns 0-255 in TMEM,
-//    columns 256-575 in shared memory (128-byte swizzled).  The selected kv
+//    (128 x 576 bf16) are the A operand of S = Q kv^T: columns 0-255 in TMEM
+//    (loaded by TMA into the second gather stage, which is still free, and
+//    moved into TMEM by the softmax warps), columns 256-575 in shared memory
+//    (128-byte swizzled).  The selected kv
 //    rows are gathered 64 at a time by eight gather warps, four per stage
 //    (16-byte cp.async copies, one kv row per warp instruction, into the
 //    128-byte-swizzled layout the tensor core reads; two stages, each
@@ -64,6 +66,12 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c,
+                                             uint32_t& d) {
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(addr)
+                 : "memory");
+}
+
 struct SmlaParams {
     const __nv_bfloat16* q;    // [T, H, 576]
     const __nv_bfloat16* kv;   // [Tg, 576]
@@ -93,7 +101,7 @@ constexpr int kTmQ = 0, kTmS = kQT / 2, kTmO = kTmS + 2 * kBN;
 constexpr int B_Q_READY = 0, B_QS_FULL = 1, B_FULL = 2, B_SFREE = B_FULL + kNST, B_EMPTY = B_SFREE + kNST,
               B_S_FULL = B_EMPTY + kNST,
               B_P_FULL = B_S_FULL + 2, B_O_FULL = B_P_FULL + 2, B_DRAIN = B_O_FULL + 1,
-              kNumBars = B_DRAIN + 1;
+              B_QT_FULL = B_DRAIN + 1, kNumBars = B_QT_FULL + 1;
 constexpr int kSmemQ = kNST * kStageBytes;                  // 1024-aligned
 constexpr int kSmemBias = kSmemQ + kQSChunks * kQSChunkBytes;  // float [kNST][64]
 constexpr int kSmemBar = kSmemBias + kNST * kBN * 4;
@@ -152,6 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1) thd_sparse_mla_attn_kernel(const 
 
     if (threadIdx.x == 0) {
         thd::mbar_init(bar(B_Q_READY), 4);
+        thd::mbar_init(bar(B_QT_FULL), 1);
         thd::mbar_init(bar(B_QS_FULL), 1);
         for (int s = 0; s < kNST; ++s) {
             thd::mbar_init(bar(B_FULL + s), kPW);  // the stage's gather warps
@@ -193,9 +202,12 @@ __global__ void __launch_bounds__(kThreads, 1) thd_sparse_mla_attn_kernel(const 
         constexpr int kRows = kBN / kPW;
         const int pw = warp - 4;
         const int s = pw / kPW;                 // this warp's stage
+        // Stage 1 first holds Q's TMEM columns on their way into TMEM: its
+        // gathers start once the softmax warps have read them.
         const int r0 = (pw % kPW) * kRows;
         const int32_t* irow = p.idx + t * p.K;
         bool ok = !skip;
+        if (ok && s == 1 && nch > 1) ok = thd::warp_wait(bar(B_Q_READY), 0, abort_flag, p.status);
         for (int c = s; ok && c < nch; c += kNST) {
             const uint32_t par = ((c / kNST) & 1) ^ 1;
             ok = thd::warp_wait(bar(B_SFREE + s), par, abort_flag, p.status);
@@ -272,9 +284,14 @@ __global__ void __launch_bounds__(kThreads, 1) thd_sparse_mla_attn_kernel(const 
             // issued (its S / P buffer), PV(k) needs P(k).  A PV that can go
             // is issued first: it frees the chunk's stage for the gather of
             // chunk k + 2.
-            // Q[:, kQT:] of the token's 128 heads: five 64-column boxes
-            // straight into the swizzled layout.
+            // Q[:, :kQT] of the token's 128 heads (four 64-column boxes) into
+            // stage 1, on their way into TMEM; Q[:, kQT:] (five boxes)
+            // straight into the swizzled layout the MMAs read.
             thd::tma_prefetch_desc(&tmap_q);
+            thd::mbar_arrive_expect_tx(bar(B_QT_FULL), (kQT / 64) * kQSChunkBytes);
+            for (int i = 0; i < kQT / 64; ++i)
+                thd::tma_load_3d(sbase + kStageBytes + i * kQSChunkBytes, &tmap_q, bar(B_QT_FULL), 64 * i,
+                                 hg * 128, static_cast<int>(t));
             thd::mbar_arrive_expect_tx(bar(B_QS_FULL), kQSChunks * kQSChunkBytes);
             for (int i = 0; i < kQSChunks; ++i)
                 thd::tma_load_3d(sbase + kSmemQ + i * kQSChunkBytes, &tmap_q, bar(B_QS_FULL), kQT + 64 * i,
@@ -328,6 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1) thd_sparse_mla_attn_kernel(const 
             }
             thd::mma_commit(bar(B_DRAIN));
             thd::drain_wait(bar(B_DRAIN), 0);
+            thd::drain_wait(bar(B_QT_FULL), 0);  // (landed long ago unless unwinding)
         }
         __syncwarp();
     } else {
@@ -336,26 +354,20 @@ __global__ void __launch_bounds__(kThreads, 1) thd_sparse_mla_attn_kernel(const 
         const int h = hg * 128 + row;
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
         bool ok = !skip;
+        if (ok) ok = thd::warp_wait(bar(B_QT_FULL), 0, abort_flag, p.status);
         if (ok) {
-            // Q row h, columns [0, kQT), into TMEM (bf16 pairs): batches of
-            // 64 columns, the next batch's loads in flight while this one is
-            // stored.  (Columns kQT and up arrive by TMA.)
-            const uint4* src = reinterpret_cast<const uint4*>(p.q + (t * p.H + h) * kQDim);
-            uint4 x[2][8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) x[0][u] = src[u];
+            // Q row h, columns [0, kQT), into TMEM (bf16 pairs), from the
+            // four 64-column boxes TMA put into stage 1 (128-byte swizzle:
+            // 16-byte unit u of row r at r * 128 + ((u ^ (r % 8)) * 16)).
+            // Arriving on Q_READY also hands stage 1 to its gather warps.
+            const uint32_t qt = sbase + kStageBytes + static_cast<uint32_t>(row) * 128;
 #pragma unroll
             for (int i = 0; i < kQT / 64; ++i) {
-                if (i + 1 < kQT / 64) {
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) x[(i + 1) & 1][u] = src[(i + 1) * 8 + u];
-                }
                 uint32_t w[32];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    w[4 * u] = x[i & 1][u].x; w[4 * u + 1] = x[i & 1][u].y;
-                    w[4 * u + 2] = x[i & 1][u].z; w[4 * u + 3] = x[i & 1][u].w;
-                }
+                for (int u = 0; u < 8; ++u)
+                    ld_shared_v4(qt + i * kQSChunkBytes + ((static_cast<uint32_t>(u) ^ static_cast<uint32_t>(row & 7)) << 4),
+                                 w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
                 thd::tmem_st32(lane_base + kTmQ + 32 * i, w);
             }
             thd::tmem_wait_st();
