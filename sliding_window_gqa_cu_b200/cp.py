@@ -129,6 +129,11 @@ def cp_rank_parts(q_local: torch.Tensor, k_local: torch.Tensor, v_local: torch.T
     D = q_local.shape[2]
     if scale is None:
         scale = D ** -0.5
+    if e == b:  # an empty shard still takes part in the collective
+        kv_before()
+        Hq = q_local.shape[1]
+        return (torch.empty((0, Hq, D), dtype=q_local.dtype, device=q_local.device),
+                torch.empty((0, Hq), dtype=torch.float32, device=q_local.device))
     out, lse = thd_attn_fwd(q_local, k_local, v_local, local_cu_seqlens(cu_seqlens, b, e), window,
                             scale, sinks)
     x = crossing_rows(cu_seqlens, b, e)

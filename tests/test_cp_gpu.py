@@ -128,8 +128,6 @@ def test_overlapped_parts_equal_the_oracle(lens, Hq, Hkv, D, window, sinks, worl
     T = int(p["T"])
     outs, lses = [], []
     for b, e in cp.shard_bounds(T, world):
-        if e == b:
-            continue
         o, l = cp.cp_rank_parts(q[b:e].contiguous(), k[b:e].contiguous(), v[b:e].contiguous(),
                                 p["cu_seqlens"], b, e, window, p["scale"], s, kv_before=lambda: (k, v))
         outs.append(o)
