@@ -223,3 +223,51 @@ def test_host_pipeline_rejects_bad_arguments_before_any_cuda_call(lib, kw, code)
 def test_stall_selftest_rejects_null_before_any_cuda_call(lib):
     lib.thd_attn_selftest_stall.argtypes = [ctypes.c_void_p]
     assert lib.thd_attn_selftest_stall(None) == -1
+
+
+# ----------------------------------------------- key-bounded range and merge ---
+
+def _range_keys(lib, cu=(0, 5, 9), qb=0, qe=9, k_end=5, D=64, ptr=0x10000):
+    cu = np.asarray(cu, dtype=np.int32)
+    lib.thd_attn_fwd_range_keys.argtypes = [ctypes.c_void_p] * 3 + [ctypes.POINTER(ctypes.c_int32)] + \
+        [ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64] + [ctypes.c_int] * 4 + \
+        [ctypes.c_float] + [ctypes.c_void_p] * 4
+    return lib.thd_attn_fwd_range_keys(ptr, ptr, ptr, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                       cu.size - 1, qb, qe, k_end, 4, 2, D, 0, 0.125, None, ptr, None,
+                                       None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k_end=10), -1),          # beyond the pack
+    (dict(k_end=-1), -1),
+    (dict(qb=5, qe=4), -1),        # empty-but-reversed row range
+    (dict(qe=10), -1),
+    (dict(cu=(0, 5, 3)), -1),
+    (dict(ptr=0x10008), -1),       # misaligned
+    (dict(D=96), -2),
+    (dict(qb=4, qe=4), 0),         # no rows: nothing to do
+    (dict(cu=(0,), qe=0, k_end=0), 0),
+])
+def test_range_keys_rejects_bad_arguments_before_any_cuda_call(lib, kw, code):
+    assert _range_keys(lib, **kw) == code
+
+
+def _merge(lib, rows=3, Hq=4, D=128, a=0x10000, la=0x20000, b=0x30000, lb=0x40000, o=0x50000,
+           lo=0x60000):
+    lib.thd_attn_merge.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64, ctypes.c_int, ctypes.c_int] + \
+        [ctypes.c_void_p] * 3
+    return lib.thd_attn_merge(a, la, b, lb, rows, Hq, D, o, lo, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(D=96), -2),
+    (dict(rows=-1), -1),
+    (dict(Hq=0), -1),
+    (dict(a=None), -1),
+    (dict(lo=None), -1),
+    (dict(b=0x30008), -1),         # misaligned bf16 part
+    (dict(la=0x20002), -1),        # misaligned fp32 LSE
+    (dict(rows=0, a=None, la=None), 0),   # nothing to merge
+])
+def test_merge_rejects_bad_arguments_before_any_launch(lib, kw, code):
+    assert _merge(lib, **kw) == code
