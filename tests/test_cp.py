@@ -181,6 +181,82 @@ def test_two_rank_gloo_kv_all_gather(tmp_path):
     assert [open(tmp_path / f"r{r}.txt").read() for r in range(2)] == ["ok", "ok"]
 
 
+# ------------------------------------- overlapped form, two gloo ranks on CPU --
+# The kernels need a GPU; here the three calls the overlapped forward makes are
+# replaced by fp64 stand-ins (the oracle's forward, a dense key-bounded
+# softmax from the oracle's mask, the log-sum-exp merge) so that its host
+# logic -- shard bounds, the own-slice pack, the crossing rows, k_end, the
+# asynchronous all-gather and the in-place merge -- runs on two real ranks.
+
+def _ref_fwd(q, k, v, cu_seqlens, window=0, scale=None, sinks=None, **_):
+    import oracle
+    o, l = oracle.attention(q.double().numpy(), k.double().numpy(), v.double().numpy(), cu_seqlens,
+                            window, scale, sinks)
+    return torch.from_numpy(o), torch.from_numpy(l)
+
+
+def _ref_range(q, k, v, cu_seqlens, q_begin, q_end, window=0, scale=None, sinks=None, k_end=None, **_):
+    """Rows [q_begin, q_end) against keys j < k_end (dense, fp64, no sinks)."""
+    import oracle
+    assert sinks is None
+    qa, ka, va = (t.double().numpy() for t in (q, k, v))
+    G = qa.shape[1] // ka.shape[1]
+    mask = oracle.dense_mask(cu_seqlens, window)[q_begin:q_end, :k_end]         # [n, k_end]
+    kx, vx = oracle.repeat_kv(ka[:k_end], G), oracle.repeat_kv(va[:k_end], G)
+    sc = np.where(mask[None], scale * np.einsum("ihc,jhc->hij", qa, kx), -np.inf)  # [Hq, n, k_end]
+    m = sc.max(axis=2, keepdims=True) if k_end > 0 else np.full(sc.shape[:2] + (1,), -np.inf)
+    ms = np.where(np.isfinite(m), m, 0.0)
+    w = np.exp(sc - ms)
+    Z = w.sum(axis=2, keepdims=True)
+    out = np.einsum("hij,jhc->ihc", np.where(Z > 0, w / np.where(Z > 0, Z, 1.0), 0.0), vx)
+    lse = np.where(Z[..., 0] > 0, np.log(np.where(Z[..., 0] > 0, Z[..., 0], 1.0)) + ms[..., 0], -np.inf)
+    return torch.from_numpy(out), torch.from_numpy(lse.T.copy())
+
+
+def _ref_merge(out_a, lse_a, out_b, lse_b, out=None, lse=None, **_):
+    m = torch.maximum(lse_a, lse_b)
+    ms = torch.where(torch.isfinite(m), m, torch.zeros_like(m))
+    wa, wb = torch.exp(lse_a - ms), torch.exp(lse_b - ms)
+    s = wa + wb
+    o = torch.where(s[..., None] > 0, (wa[..., None] * out_a + wb[..., None] * out_b) / s[..., None],
+                    torch.zeros_like(out_a))
+    l = torch.where(s > 0, ms + torch.log(s), torch.full_like(s, float("-inf")))
+    out.copy_(o)
+    lse.copy_(l)
+    return out, lse
+
+
+def _overlap_worker(rank, world, port, result_dir, lens, window, sinks):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    multirank.init("gloo", timeout_s=60)
+    import oracle
+    swa.thd_attn_fwd, swa.thd_attn_fwd_range, swa.thd_attn_merge = _ref_fwd, _ref_range, _ref_merge
+    p = workloads.random_pack(7, lens, 4, 2, 64, window, 0.125, sinks)
+    T = int(p["T"])
+    b, e = cp.shard_bounds(T, world)[rank]
+    q, k, v = (p[n].double() for n in "qkv")
+    o, l = cp.cp_attention_fwd_overlapped(q[b:e].contiguous(), k[b:e].contiguous(), v[b:e].contiguous(),
+                                          p["cu_seqlens"], window, 0.125, p["sinks"])
+    ref_o, ref_l = oracle.attention(p["q"], p["k"], p["v"], p["cu_seqlens"], window, 0.125, p["sinks"])
+    ok = (o.shape[0] == e - b and np.abs(o.numpy() - ref_o[b:e]).max(initial=0.0) < 1e-9 and
+          np.abs(l.numpy() - ref_l[b:e]).max(initial=0.0) < 1e-9)
+    with open(os.path.join(result_dir, f"r{rank}.txt"), "w") as f:
+        f.write("ok" if ok else "mismatch")
+    multirank.shutdown()
+
+
+@pytest.mark.parametrize("lens,window,sinks", [
+    ([300, 1, 0, 129, 78], 0, True),    # the shard boundary inside the first document
+    ([300, 1, 0, 129, 78], 40, False),  # a window shorter than the crossing part
+    ([254, 254], 0, True),              # the boundary on a document start: no keys before it
+])
+def test_two_rank_gloo_overlapped_forward(tmp_path, lens, window, sinks):
+    port = _free_port()
+    mp.spawn(_overlap_worker, args=(2, port, str(tmp_path), lens, window, sinks), nprocs=2, join=True)
+    assert [open(tmp_path / f"r{r}.txt").read() for r in range(2)] == ["ok", "ok"]
+
+
 # ----------------------------------------------------------- head sharding --
 
 @pytest.mark.parametrize("Hq,Hkv,world", [(64, 8, 8), (64, 8, 2), (32, 8, 4), (16, 1, 8),
