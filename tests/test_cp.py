@@ -5,7 +5,8 @@ exactly once, no row outside it, every visible key in its items' key tiles)
 and its key-bounded form, and the overlapped forward's split of a shard into
 its own-slice pack and the rows with keys on earlier ranks, checked by brute
 force against the window definition of FlintMagiPlan.attention ("flint.magi"
-page)."""
+page); and the overlapped forward itself on two gloo ranks, its GPU calls
+replaced by fp64 stand-ins, against the oracle."""
 import os
 import socket
 
