@@ -27,8 +27,10 @@ one line for that pass alone (``--workload`` selects the pack).
 Multi-GPU runs are launched with torchrun, one process per GPU; every rank
 runs its own pack of the same shape (no data-path collective; "weak"), or,
 with ``--shard heads``, its kv-head groups of one pack (cp.head_shard; no
-collective either; "strong").  The timed region is bracketed by a barrier and
-a device synchronisation, and the time is the max over ranks.
+collective either; "strong"), or, with ``--shard tokens``, its token shard of
+one pack (cp.cp_attention_fwd_overlapped: the K/V all-gather over NCCL under
+the own-slice part; "strong").  The timed region is bracketed by a barrier
+and a device synchronisation, and the time is the max over ranks.
 """
 from __future__ import annotations
 
@@ -87,9 +89,10 @@ def parse_args(argv=None):
                     default="fwd", help="what one step runs (default: the forward, the headline)")
     ap.add_argument("--no-extras", action="store_true",
                     help="headline only: leave out per_config and passes")
-    ap.add_argument("--shard", choices=["packs", "heads"], default="packs",
-                    help="multi-GPU form: every rank its own pack (weak scaling, default) or "
-                         "every rank its kv-head groups of one pack (strong scaling, no collective)")
+    ap.add_argument("--shard", choices=["packs", "heads", "tokens"], default="packs",
+                    help="multi-GPU form: every rank its own pack (weak scaling, default), "
+                         "every rank its kv-head groups of one pack (strong scaling, no collective) "
+                         "or its token shard of one pack (context parallel, overlapped K/V all-gather)")
     return ap.parse_args(argv)
 
 
@@ -318,7 +321,8 @@ def fwd_case(swa, cfg, args, info, device, stream, T_override=None):
     ``--shard heads`` every rank holds the same pack and keeps only its head
     slice (cp.head_shard): q/k/v/sinks/out/lse have the slice's head counts."""
     heads = getattr(args, "shard", "packs") == "heads"
-    seed = args.seed if heads else multirank.tensor_seed(args.seed, info.rank)
+    tokens = getattr(args, "shard", "packs") == "tokens"
+    seed = args.seed if heads or tokens else multirank.tensor_seed(args.seed, info.rank)
     pack = workloads.make_pack(cfg, args.seed, tensor_seed=seed, T_override=T_override)
     cu = pack["cu_seqlens"]
     if heads:
@@ -336,8 +340,21 @@ def fwd_case(swa, cfg, args, info, device, stream, T_override=None):
     out = torch.empty((T, Hq_r, cfg.D), dtype=torch.bfloat16, device=device)
     lse = torch.empty((T, Hq_r), dtype=torch.float32, device=device)
 
+    if tokens:
+        from sliding_window_gqa_cu_b200 import cp
+        b, e = cp.shard_bounds(T, info.world)[info.rank]
+        ql, kl, vl = q[b:e].contiguous(), k[b:e].contiguous(), v[b:e].contiguous()
+
+        def step():
+            cp.cp_attention_fwd_overlapped(ql, kl, vl, cu, cfg.window, cfg.scale, sinks)
+        # this rank's launches per step: the own-slice forward, plus the
+        # key-bounded range and the merge when a document crosses its start
+        step.launches = 1 + (2 if cp.crossing_rows(cu, b, e) > b else 0)
+        return pack, dict(q=q, k=k, v=v, sinks=sinks, out=out, lse=lse), step
+
     def step():
         swa.thd_attn_fwd(q, k, v, cu, cfg.window, cfg.scale, sinks, out=out, lse=lse, stream=stream)
+    step.launches = 1
     return pack, dict(q=q, k=k, v=v, sinks=sinks, out=out, lse=lse), step
 
 
@@ -480,7 +497,11 @@ def run_ours(args, info):
     max_ms, max_launch, h0, h1 = timed_loop(step, args, device, stream, f"thd_attn_fwd {cfg.name}")
     check_status(swa, stream, cfg.name)
     csum = clocks.summary(h0, h1)
-    value = multirank.aggregate_rate(flops * args.steps, info.world, max_ms / 1e3) / 1e12
+    if args.shard == "tokens":  # flops is the whole pack's, shared by the ranks
+        value = flops * args.steps / (max_ms / 1e3) / 1e12
+    else:
+        value = multirank.aggregate_rate(flops * args.steps, info.world, max_ms / 1e3) / 1e12
+    launches = step.launches
 
     # end to end through the public API with pinned host buffers
     e2e = None
@@ -518,9 +539,12 @@ def run_ours(args, info):
                "ms_per_step": e2e_ms / args.e2e_steps,
                "path": f"thd_attn_fwd_host, pinned host buffers, {E2E_CHUNKS} overlapped token ranges"}
 
-    achieved = flops / (max_launch / 1e3) / 1e12
+    # per GPU: the whole pack's flops over the ranks with --shard tokens
+    achieved = flops / (info.world if args.shard == "tokens" else 1) / (max_launch / 1e3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": traffic_per_launch(cfg.name),
+                "frac": achieved / peak,
+                # a full-pack launch's DRAM bytes: packs mode, or a single GPU
+                "traffic": traffic_per_launch(cfg.name) if args.shard == "packs" or info.world == 1 else None,
                 "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)" if peak_src == "measured"
                 else "fallback 1.59 PFLOP/s",
                 "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
@@ -568,16 +592,19 @@ def run_ours(args, info):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": info.world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
-            "higher_is_better": True, "scaling": "strong" if args.shard == "heads" else "weak",
+            "higher_is_better": True, "scaling": "weak" if args.shard == "packs" else "strong",
             "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": workload_config(cfg, cu, pairs, {
                 "parallelism": (f"head-sharded x{info.world} (one pack, no collective)"
-                                if args.shard == "heads" else f"pack-parallel x{info.world}"),
+                                if args.shard == "heads" else
+                                f"context-parallel x{info.world} (token shards of one pack, "
+                                f"K/V all-gather overlapped with the own-slice part)"
+                                if args.shard == "tokens" else f"pack-parallel x{info.world}"),
                 "per_rank_tflop": flops / 1e12}),
             "pct_of_peak": 100.0 * value / info.world / peak,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": args.steps, "clocks": {k: csum[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+            "gpu_launches": args.steps * launches, "clocks": {k: csum[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
             "first_call_ms_with_schedule_build": first_call_ms,
             "per_config": per_config, "passes": passes,
         }
@@ -601,7 +628,7 @@ def run_other_pass(args, info):
     import sliding_window_gqa_cu_b200 as swa
 
     if args.shard != "packs":
-        raise SystemExit("--shard heads applies to the forward only")
+        raise SystemExit("--shard heads / tokens apply to the forward only")
 
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device (the CUDA path has no CPU fallback)")
